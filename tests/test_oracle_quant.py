@@ -1,0 +1,260 @@
+"""Pins for the oracle's quantizers: the scaled-amax invariant (each tile's amax encodes to
+exactly 448), exact round trips on inputs whose scales are powers of two (which fixes the
+scale formula, its stored form and its layout), brute-force encoders, brute-force MX
+exponent minimality, and the statistics of stochastic rounding."""
+import numpy as np
+import pytest
+
+import workloads
+from oracle import formats as F
+from oracle import quant as Q
+from oracle import rht as RHT
+
+
+def exact_matrix(R, C, tr, tc, rng, top=448.0, grid="e4m3", jrange=(-12, 12)):
+    """Values on the element grid times a power of two per (tr x tc) tile, with one element
+    of each tile at +-top * 2^j: quantization of such a matrix is exact."""
+    if grid == "e4m3":
+        mags = F.e4m3_decode(rng.integers(0, 0x7F, (R, C)).astype(np.uint8))
+    else:
+        mags = F.E2M1_VALUES[rng.integers(0, 8, (R, C))]
+    sign = np.where(rng.random((R, C)) < 0.5, -1.0, 1.0)
+    x = mags * sign
+    js = rng.integers(jrange[0], jrange[1], (-(-R // tr), -(-C // tc)))
+    for i in range(js.shape[0]):
+        for j in range(js.shape[1]):
+            blk = x[i * tr:(i + 1) * tr, j * tc:(j + 1) * tc]
+            blk[0, 0] = top * (1 if rng.random() < 0.5 else -1)
+            blk *= 2.0 ** js[i, j]
+    return x.astype(np.float32), js
+
+
+def test_1x128_exact_roundtrip_pins_scale_and_layout():
+    rng = np.random.default_rng(0)
+    x, js = exact_matrix(24, 384, 1, 128, rng)
+    q, s = Q.quantize_1x128_rowwise(x)
+    assert s.shape == (3, 24)
+    assert np.array_equal(s, np.exp2(js.T).astype(np.float32))
+    deq = F.e4m3_decode(q) * np.repeat(s.T.astype(np.float64), 128, axis=1)
+    assert np.array_equal(deq, x.astype(np.float64))
+
+
+def test_1x128_amax_maps_to_448_on_real_inputs():
+    x = Q.as_f32(workloads.bf16_bits(workloads.tiny()["A"]))
+    q, s = Q.quantize_1x128_rowwise(x)
+    t = np.abs(x).reshape(256, 4, 128)
+    amax = t.max(-1, keepdims=True)
+    hit = (t == amax) & (amax > 0)
+    assert np.all((q.reshape(256, 4, 128)[hit] & 0x7F) == 0x7E)
+    # stored decode scale times 448 recovers amax to FP32 rounding
+    rel = np.abs(s.T.astype(np.float64) * 448.0 / amax[..., 0] - 1.0)
+    assert rel.max() < 2.0 ** -22
+
+
+def test_1x128_codes_match_bruteforce_encoder():
+    rng = np.random.default_rng(1)
+    x = (rng.standard_normal((3, 256)) * np.exp2(rng.integers(-10, 10, (3, 1)))).astype(np.float32)
+    q, _ = Q.quantize_1x128_rowwise(x)
+    t = x.reshape(3, 2, 128)
+    sf = (np.float32(448.0) / np.abs(t).max(-1)).astype(np.float32)
+    y = (t * sf[..., None]).astype(np.float32).reshape(3, 256)
+    assert np.array_equal(q, F.e4m3_encode_bruteforce(y).reshape(3, 256))
+
+
+def test_1x128_zero_tile_and_colwise_transpose():
+    rng = np.random.default_rng(2)
+    x, js = exact_matrix(256, 256, 128, 1, rng)
+    x[:128, 5] = 0.0
+    qc, sc = Q.quantize_1x128_colwise(x)
+    assert qc.shape == (256, 256) and sc.shape == (2, 256)
+    assert sc[0, 5] == 1.0 and np.all(qc[5, :128] == 0)
+    keep = np.ones(256, bool)
+    keep[5] = False
+    expect = np.exp2(js).astype(np.float32)
+    assert np.array_equal(sc[:, keep], expect[:, keep])
+    deq = F.e4m3_decode(qc) * np.repeat(sc.T.astype(np.float64), 128, axis=1)
+    assert np.array_equal(deq, x.T.astype(np.float64))
+
+
+def test_scale_overflow_clamps_to_flt_max():
+    x = np.zeros((1, 128), np.float32)
+    x[0, 0] = np.float32(1e-40)         # a subnormal amax: 448 / amax overflows FP32
+    q, s = Q.quantize_1x128_rowwise(x)
+    assert np.isfinite(s[0, 0]) and s[0, 0] == np.float32(1.0) / F.FLT_MAX
+
+
+def test_128x128_exact_and_transposed_layout():
+    rng = np.random.default_rng(3)
+    w, js = exact_matrix(256, 384, 128, 128, rng)
+    q, qt, s = Q.quantize_128x128(w)
+    assert s.shape == (3, 2) and np.array_equal(qt, q.T)
+    assert np.array_equal(s, np.exp2(js.T).astype(np.float32))
+    scale = np.exp2(np.repeat(np.repeat(js, 128, 0), 128, 1).astype(np.float64))
+    assert np.array_equal(F.e4m3_decode(q) * scale, w.astype(np.float64))
+
+
+def test_128x128_amax_maps_to_448():
+    w = Q.as_f32(workloads.bf16_bits(workloads.tiny()["B"]))
+    q, _, _ = Q.quantize_128x128(w)
+    for i in range(4):
+        for j in range(2):
+            blk = np.abs(w[128 * i:128 * i + 128, 128 * j:128 * j + 128])
+            hit = blk == blk.max()
+            assert np.all((q[128 * i:128 * i + 128, 128 * j:128 * j + 128][hit] & 0x7F) == 0x7E)
+
+
+def test_per_tensor_exact_and_amax():
+    rng = np.random.default_rng(4)
+    x = F.e4m3_decode(rng.integers(0, 0x7E, (64, 96)).astype(np.uint8)) * 2.0 ** -5
+    x[7, 9] = -448 * 2.0 ** -5
+    q, s = Q.quantize_tensor(x.astype(np.float32))
+    assert s == np.float32(2.0 ** -5) and q[7, 9] == 0xFE
+    assert np.array_equal(F.e4m3_decode(q) * float(s), x)
+
+
+# ----------------------------------------------------------------------------- MX
+def _mx_bruteforce(amax):
+    out = []
+    for a in np.asarray(amax, np.float32).astype(np.float64).ravel():
+        if a == 0:
+            out.append(-127)
+            continue
+        for e in range(-127, 128):
+            if a <= 448.0 * 2.0 ** e:
+                out.append(e)
+                break
+        else:
+            out.append(127)
+    return np.array(out)
+
+
+def test_mx_exponent_is_minimal_bruteforce():
+    rng = np.random.default_rng(5)
+    a = [0.0, 448.0, 448.0 * 2 ** -3, np.nextafter(np.float32(448.0), np.float32(1e9)),
+         np.float32(1e-40), np.float32(3e-45), np.float32(3.3e38), 1.0, 1.75, 1.7500001, 224.0]
+    a = np.concatenate([np.float32(a), (rng.random(3000) * np.exp2(rng.integers(-140, 120, 3000)))
+                        .astype(np.float32)])
+    assert np.array_equal(Q.mx_exponent(a), _mx_bruteforce(a))
+
+
+def test_mx_no_saturation_and_exact_roundtrip():
+    rng = np.random.default_rng(6)
+    x, js = exact_matrix(16, 256, 1, 32, rng)
+    q, e = Q.quantize_mx_rowwise(x)
+    assert np.array_equal(e.astype(np.int64) - 127, js)
+    deq = F.e4m3_decode(q) * np.repeat(F.e8m0_decode(e), 32, axis=1)
+    assert np.array_equal(deq, x.astype(np.float64))
+    # random inputs: the scaled amax lies in (224, 448] and nothing exceeds 448
+    xr = Q.as_f32(workloads.bf16_bits(workloads.tiny()["A"]))
+    q, e = Q.quantize_mx_rowwise(xr)
+    amax = np.abs(xr).reshape(256, 16, 32).max(-1)
+    scaled = amax.astype(np.float64) / F.e8m0_decode(e)
+    assert np.all((scaled > 224) & (scaled <= 448))
+    assert np.all(np.abs(xr).reshape(256, 16, 32) / F.e8m0_decode(e)[..., None] <= 448)
+
+
+def test_mx_colwise_is_transposed():
+    x = Q.as_f32(workloads.bf16_bits(workloads.tiny()["B"]))
+    qc, ec = Q.quantize_mx_colwise(x)
+    assert qc.shape == (256, 512) and ec.shape == (256, 16)
+    qr, er = Q.quantize_mx_rowwise(np.ascontiguousarray(x.T))
+    assert np.array_equal(qc, qr) and np.array_equal(ec, er)
+
+
+# ----------------------------------------------------------------------------- NVFP4
+def test_nvfp4_exact_grid_roundtrip():
+    rng = np.random.default_rng(7)
+    x, js = exact_matrix(8, 128, 1, 16, rng, top=6.0, grid="e2m1", jrange=(-5, 5))
+    q, sf, g = Q.quantize_nvfp4_rowwise(x)
+    deq = _deq_nvfp4(q, sf, g)
+    assert np.allclose(deq, x.astype(np.float64), rtol=2.0 ** -23, atol=0)
+    jmax = js.max()
+    assert np.array_equal(F.e4m3_decode(sf), 448.0 * np.exp2(js - jmax))
+
+
+def _deq_nvfp4(q, sf, g):
+    codes = F.unpack_e2m1(q)
+    return F.e2m1_decode(codes) * np.repeat(F.e4m3_decode(sf), 16, axis=1) * float(g)
+
+
+def test_nvfp4_scale_invariants_and_rne_bruteforce():
+    d = workloads.nvfp4(M=64, H=64, F=256, which=("dY",))
+    x = Q.as_f32(workloads.bf16_bits(d["dY"]))
+    q, sf, g = Q.quantize_nvfp4_rowwise(x)
+    dec = F.e4m3_decode(sf)
+    assert np.all(dec <= 448) and np.all(sf < 0x80)
+    # rebuild y from the stored scales and compare codes with the brute-force encoder
+    S_g = np.float32(np.float32(2688.0) / np.float32(np.abs(x).max()))
+    assert np.float32(np.float32(1.0) / S_g) == g
+    enc = np.where(sf == 0, 0, (S_g / dec.astype(np.float32))).astype(np.float32)
+    y = (x.reshape(64, 16, 16) * enc[..., None]).astype(np.float32).reshape(64, 256)
+    assert np.all(np.abs(y) <= 6.0 / (1 - 2.0 ** -4))
+    assert np.array_equal(F.unpack_e2m1(q), F.e2m1_encode_bruteforce(y).reshape(64, 256))
+
+
+def test_nvfp4_sr_is_unbiased_and_picks_neighbours():
+    n_blocks = 65536
+    v, w = np.float32(1.0), np.float32(0.3)
+    x = np.full((n_blocks, 16), w, np.float32)
+    x[:, 0] = v
+    x = x.reshape(1024, 1024)
+    q, sf, g = Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=6)
+    deq = _deq_nvfp4(q, sf, g).reshape(n_blocks, 16)[:, 1:].ravel()
+    scale = float(F.e4m3_decode(sf[0, 0])) * float(g)
+    y = float(np.float32(w * np.float32(np.float32(np.float32(2688.0) / v)
+                                        / np.float32(F.e4m3_decode(sf[0, 0])))))
+    lo, hi, _ = F.e2m1_grid_neighbours(np.array([y]))
+    vals = np.unique(deq / scale)
+    assert set(np.round(vals, 6)) <= {round(float(lo[0]), 6), round(float(hi[0]), 6)}
+    p = (y - lo[0]) / (hi[0] - lo[0])
+    sigma = np.sqrt(p * (1 - p)) * (hi[0] - lo[0])
+    mean = (deq / scale).mean()
+    assert abs(mean - y) < 4 * sigma / np.sqrt(deq.size)
+    assert deq.size > 900_000
+    # a different seed changes the draws, the same seed reproduces them
+    q2, _, _ = Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=6)
+    q3, _, _ = Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=7)
+    assert np.array_equal(q, q2) and not np.array_equal(q, q3)
+
+
+def test_nvfp4_rht_roundtrip_close_and_orthogonal_gemm():
+    rng = np.random.default_rng(8)
+    A = rng.standard_normal((32, 256)).astype(np.float32)
+    B = rng.standard_normal((24, 256)).astype(np.float32)
+    qa, sa, ga = Q.quantize_nvfp4_rowwise(A, rht=True, rht_seed=5)
+    qb, sb, gb = Q.quantize_nvfp4_rowwise(B, rht=True, rht_seed=5)
+    C_rht = _deq_nvfp4(qa, sa, ga) @ _deq_nvfp4(qb, sb, gb).T
+    qa0, sa0, ga0 = Q.quantize_nvfp4_rowwise(A)
+    qb0, sb0, gb0 = Q.quantize_nvfp4_rowwise(B)
+    C_plain = _deq_nvfp4(qa0, sa0, ga0) @ _deq_nvfp4(qb0, sb0, gb0).T
+    C = A.astype(np.float64) @ B.astype(np.float64).T
+    scale = np.sqrt(256.0)
+    assert np.abs(C_rht - C).max() < 0.25 * scale * 4
+    assert np.abs(C_plain - C).max() < 0.25 * scale * 4
+    # undoing the transform on the dequantized operand recovers A approximately
+    s = RHT.rht_signs(5)
+    Qm = np.diag(s.astype(np.float64)) @ __import__("scipy").linalg.hadamard(16) / 4.0
+    Ad = _deq_nvfp4(qa, sa, ga).reshape(32, 16, 16) @ Qm.T
+    assert np.abs(Ad.reshape(32, 256) - A).max() < 1.0
+
+
+def test_nvfp4_colwise_uses_tag_one():
+    x = np.full((32, 16), 0.3, np.float32)
+    x[0] = 1.0
+    qc, sc, gc = Q.quantize_nvfp4_colwise(x, sr=True, sr_seed=9)
+    qr, sr_, gr = Q.quantize_nvfp4_rowwise(np.ascontiguousarray(x.T), sr=True, sr_seed=9, tag=1)
+    assert np.array_equal(qc, qr) and np.array_equal(sc, sr_)
+    qr0, _, _ = Q.quantize_nvfp4_rowwise(np.ascontiguousarray(x.T), sr=True, sr_seed=9, tag=0)
+    assert not np.array_equal(qc, qr0)
+
+
+def test_sf_tiled_layout_is_a_permutation():
+    rng = np.random.default_rng(10)
+    for R, S in [(128, 4), (200, 7), (300, 33), (5, 1)]:
+        sf = rng.integers(1, 255, (R, S)).astype(np.uint8)
+        flat = Q.sf_to_tiled(sf)
+        assert flat.size == Q.sf_tiled_size(R, S)
+        assert np.array_equal(Q.sf_from_tiled(flat, R, S), sf)
+        assert np.count_nonzero(flat) == R * S
+        rr, cc = np.meshgrid(np.arange(R), np.arange(S), indexing="ij")
+        assert len(np.unique(Q.sf_tiled_offset(rr, cc, S))) == R * S
