@@ -1,0 +1,293 @@
+"""Python binding of libfp8q.so (the C ABI declared in include/fp8q.h).
+
+Argument marshalling only: every step of quantization and GEMM runs in the library's CUDA
+kernels.  PyTorch supplies device memory (outputs are allocated with torch) and the current
+CUDA stream.  There is no CPU fallback: if the library is missing or no CUDA device is
+present, the calls raise.
+
+Two layers, same names as the C ABI:
+  * ``fp8q_quantize_1x128(...)`` etc. take raw integers/pointers exactly like the C calls;
+  * ``quantize_1x128(x, ...)``, ``quantize_128x128``, ``quantize_mx32``, ``quantize_tensor``,
+    ``rht16_quantize_sr``, ``gemm`` take torch tensors, allocate the outputs and call them.
+"""
+import ctypes
+import os
+
+import torch
+
+__all__ = [
+    "FP8Q_OK", "FP8Q_BLOCKWISE", "FP8Q_MXFP8", "FP8Q_PERTENSOR", "FP8Q_NVFP4",
+    "FP8Q_FPROP", "FP8Q_DGRAD", "FP8Q_WGRAD", "FP8Q_SF_ROWMAJOR", "FP8Q_SF_MMA_TILED",
+    "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
+    "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
+    "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
+    "fp8q_status_string", "fp8q_version", "GemmArgs",
+    "quantize_1x128", "quantize_128x128", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
+    "gemm", "device_status", "EXPORTED_SYMBOLS",
+]
+
+FP8Q_OK = 0
+FP8Q_ERR_TIMEOUT = 6
+FP8Q_BLOCKWISE, FP8Q_MXFP8, FP8Q_PERTENSOR, FP8Q_NVFP4 = 0, 1, 2, 3
+FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD = 0, 1, 2
+FP8Q_SF_ROWMAJOR, FP8Q_SF_MMA_TILED = 0, 1
+FP4Q_ROW, FP4Q_COL = 1, 2
+
+EXPORTED_SYMBOLS = [
+    "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
+    "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
+    "fp8q_release_scratch", "fp8q_status_string", "fp8q_version",
+]
+
+library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
+
+
+class Fp8qError(RuntimeError):
+    def __init__(self, status, where):
+        self.status = status
+        super().__init__(f"{where}: status {status} ({_status_str(status)})")
+
+
+class GemmArgs(ctypes.Structure):
+    """Mirror of fp8q_gemm_args (field order and types as in include/fp8q.h)."""
+    _fields_ = [
+        ("recipe", ctypes.c_int), ("layout", ctypes.c_int),
+        ("M", ctypes.c_int64), ("N", ctypes.c_int64), ("K", ctypes.c_int64),
+        ("a", ctypes.c_void_p), ("a_scale", ctypes.c_void_p), ("lda", ctypes.c_int64), ("ld_sa", ctypes.c_int64),
+        ("b", ctypes.c_void_p), ("b_scale", ctypes.c_void_p), ("ldb", ctypes.c_int64), ("ld_sb", ctypes.c_int64),
+        ("a_global", ctypes.c_void_p), ("b_global", ctypes.c_void_p),
+        ("c", ctypes.c_void_p), ("ldc", ctypes.c_int64),
+        ("m_offsets", ctypes.c_void_p), ("num_groups", ctypes.c_int32),
+    ]
+
+
+_LIB = None
+_i64, _u64, _vp, _int = ctypes.c_int64, ctypes.c_uint64, ctypes.c_void_p, ctypes.c_int
+
+
+def lib():
+    """Loads libfp8q.so once; raises if it has not been built."""
+    global _LIB
+    if _LIB is None:
+        if not os.path.exists(library_path):
+            raise ImportError(f"{library_path} is missing: build it with "
+                              "`python -m fp4_precision_gemm_b200.build`")
+        L = ctypes.CDLL(library_path)
+        L.fp8q_quantize_1x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _i64, _vp]
+        L.fp8q_quantize_128x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
+        L.fp8q_quantize_mx32.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp]
+        L.fp8q_quantize_tensor.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
+        L.fp4q_rht16_quantize_sr.argtypes = [_vp, _i64, _i64, _i64, _int, _u64, _int, _u64,
+                                             _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
+        L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
+        L.fp8q_sf_bytes.argtypes = [_int, _i64, _i64, _int]
+        L.fp8q_sf_bytes.restype = ctypes.c_size_t
+        L.fp8q_get_device_status.argtypes = [_vp]
+        L.fp8q_release_scratch.argtypes = []
+        L.fp8q_status_string.argtypes = [_int]
+        L.fp8q_status_string.restype = ctypes.c_char_p
+        L.fp8q_version.argtypes = []
+        L.fp8q_version.restype = ctypes.c_char_p
+        for name in EXPORTED_SYMBOLS:
+            f = getattr(L, name)
+            if f.restype is ctypes.c_int or name in ("fp8q_quantize_1x128", "fp8q_quantize_128x128",
+                                                     "fp8q_quantize_mx32", "fp8q_quantize_tensor",
+                                                     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
+                                                     "fp8q_get_device_status", "fp8q_release_scratch"):
+                f.restype = ctypes.c_int
+        _LIB = L
+    return _LIB
+
+
+def _status_str(st):
+    try:
+        return lib().fp8q_status_string(st).decode()
+    except Exception:  # noqa: BLE001 - message only
+        return "?"
+
+
+def _check(st, where):
+    if st != FP8Q_OK:
+        raise Fp8qError(st, where)
+
+
+def _stream(stream=None):
+    if stream is None:
+        stream = torch.cuda.current_stream()
+    return ctypes.c_void_p(stream.cuda_stream)
+
+
+def _ptr(t):
+    return None if t is None else ctypes.c_void_p(t.data_ptr())
+
+
+# --------------------------------------------------------------------------- raw C calls
+def fp8q_quantize_1x128(x, rows, cols, ld_x, q_row, s_row, ld_s_row, q_col, s_col, ld_s_col, stream):
+    return lib().fp8q_quantize_1x128(x, rows, cols, ld_x, q_row, s_row, ld_s_row, q_col, s_col, ld_s_col, stream)
+
+
+def fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream):
+    return lib().fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream)
+
+
+def fp8q_quantize_mx32(x, rows, cols, ld_x, q_row, e_row, q_col, e_col, sf_layout, stream):
+    return lib().fp8q_quantize_mx32(x, rows, cols, ld_x, q_row, e_row, q_col, e_col, sf_layout, stream)
+
+
+def fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream):
+    return lib().fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream)
+
+
+def fp4q_rht16_quantize_sr(x, rows, cols, ld_x, rht, rht_seed, sr, sr_seed, q_row, sf_row, g_row,
+                           q_col, sf_col, g_col, sf_layout, stream):
+    return lib().fp4q_rht16_quantize_sr(x, rows, cols, ld_x, rht, rht_seed, sr, sr_seed, q_row, sf_row, g_row,
+                                        q_col, sf_col, g_col, sf_layout, stream)
+
+
+def fp8q_gemm_blockscaled(args, stream):
+    return lib().fp8q_gemm_blockscaled(ctypes.byref(args), stream)
+
+
+def fp8q_sf_bytes(recipe, outer, inner, layout):
+    return int(lib().fp8q_sf_bytes(recipe, outer, inner, layout))
+
+
+def fp8q_get_device_status(stream):
+    return lib().fp8q_get_device_status(stream)
+
+
+def fp8q_status_string(st):
+    return lib().fp8q_status_string(st).decode()
+
+
+def fp8q_version():
+    return lib().fp8q_version().decode()
+
+
+# --------------------------------------------------------------------------- tensor API
+def _check_bf16(x, name="x"):
+    if not (x.is_cuda and x.dtype == torch.bfloat16 and x.dim() == 2 and x.stride(1) == 1):
+        raise ValueError(f"{name} must be a 2-D row-major CUDA bf16 tensor")
+
+
+def quantize_1x128(x, rowwise=True, colwise=False, stream=None):
+    """1x128 tiles.  Returns dict with q_row (R, C) uint8, s_row (C/128, R) float32 and/or
+    q_col (C, R) uint8, s_col (R/128, C) float32."""
+    _check_bf16(x)
+    R, C = x.shape
+    out = {}
+    dev = x.device
+    if rowwise:
+        out["q_row"] = torch.empty((R, C), dtype=torch.uint8, device=dev)
+        out["s_row"] = torch.empty((C // 128, max(R, 1) + (-max(R, 1)) % 4), dtype=torch.float32, device=dev)
+    if colwise:
+        out["q_col"] = torch.empty((C, R), dtype=torch.uint8, device=dev)
+        out["s_col"] = torch.empty((R // 128, C + (-C) % 4), dtype=torch.float32, device=dev)
+    st = fp8q_quantize_1x128(_ptr(x), R, C, x.stride(0), _ptr(out.get("q_row")), _ptr(out.get("s_row")),
+                             out["s_row"].shape[1] if rowwise else 0, _ptr(out.get("q_col")),
+                             _ptr(out.get("s_col")), out["s_col"].shape[1] if colwise else 0, _stream(stream))
+    _check(st, "fp8q_quantize_1x128")
+    return out
+
+
+def quantize_128x128(w, transposed=True, plain=True, stream=None):
+    """128x128 blocks of W (K x N).  Returns q_t (N, K), q (K, N), s (N/128, K/128)."""
+    _check_bf16(w, "w")
+    K, N = w.shape
+    dev = w.device
+    out = {"s": torch.empty((N // 128, K // 128), dtype=torch.float32, device=dev)}
+    if transposed:
+        out["q_t"] = torch.empty((N, K), dtype=torch.uint8, device=dev)
+    if plain:
+        out["q"] = torch.empty((K, N), dtype=torch.uint8, device=dev)
+    st = fp8q_quantize_128x128(_ptr(w), K, N, w.stride(0), _ptr(out.get("q_t")), _ptr(out.get("q")),
+                               _ptr(out["s"]), _stream(stream))
+    _check(st, "fp8q_quantize_128x128")
+    return out
+
+
+def quantize_mx32(x, rowwise=True, colwise=False, sf_layout=FP8Q_SF_ROWMAJOR, stream=None):
+    """MXFP8.  Returns q_row (R, C) + e8m0_row, and/or q_col (C, R) + e8m0_col (flat uint8
+    buffers sized by fp8q_sf_bytes for the chosen layout)."""
+    _check_bf16(x)
+    R, C = x.shape
+    dev = x.device
+    out = {}
+    if rowwise:
+        out["q_row"] = torch.empty((R, C), dtype=torch.uint8, device=dev)
+        out["e8m0_row"] = torch.empty(fp8q_sf_bytes(FP8Q_MXFP8, R, C, sf_layout), dtype=torch.uint8, device=dev)
+    if colwise:
+        out["q_col"] = torch.empty((C, R), dtype=torch.uint8, device=dev)
+        out["e8m0_col"] = torch.empty(fp8q_sf_bytes(FP8Q_MXFP8, C, R, sf_layout), dtype=torch.uint8, device=dev)
+    st = fp8q_quantize_mx32(_ptr(x), R, C, x.stride(0), _ptr(out.get("q_row")), _ptr(out.get("e8m0_row")),
+                            _ptr(out.get("q_col")), _ptr(out.get("e8m0_col")), sf_layout, _stream(stream))
+    _check(st, "fp8q_quantize_mx32")
+    return out
+
+
+def quantize_tensor(x, stream=None):
+    """Per-tensor current scaling.  Returns q (R, C) uint8 and s_dec (1,) float32."""
+    _check_bf16(x)
+    R, C = x.shape
+    out = {"q": torch.empty((R, C), dtype=torch.uint8, device=x.device),
+           "s_dec": torch.empty((1,), dtype=torch.float32, device=x.device)}
+    st = fp8q_quantize_tensor(_ptr(x), R, C, x.stride(0), _ptr(out["q"]), _ptr(out["s_dec"]), _stream(stream))
+    _check(st, "fp8q_quantize_tensor")
+    return out
+
+
+def rht16_quantize_sr(x, rowwise=True, colwise=False, rht=0, rht_seed=0, sr=0, sr_seed=0,
+                      sf_layout=FP8Q_SF_ROWMAJOR, stream=None):
+    """NVFP4.  rht / sr are FP4Q_ROW | FP4Q_COL masks.  Returns q_row (R, C/2), sf_row,
+    g_row (1,) and/or q_col (C, R/2), sf_col, g_col (1,)."""
+    _check_bf16(x)
+    R, C = x.shape
+    dev = x.device
+    out = {}
+    if rowwise:
+        out["q_row"] = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+        out["sf_row"] = torch.empty(fp8q_sf_bytes(FP8Q_NVFP4, R, C, sf_layout), dtype=torch.uint8, device=dev)
+        out["g_row"] = torch.empty((1,), dtype=torch.float32, device=dev)
+    if colwise:
+        out["q_col"] = torch.empty((C, R // 2), dtype=torch.uint8, device=dev)
+        out["sf_col"] = torch.empty(fp8q_sf_bytes(FP8Q_NVFP4, C, R, sf_layout), dtype=torch.uint8, device=dev)
+        out["g_col"] = torch.empty((1,), dtype=torch.float32, device=dev)
+    st = fp4q_rht16_quantize_sr(_ptr(x), R, C, x.stride(0), rht, rht_seed, sr, sr_seed,
+                                _ptr(out.get("q_row")), _ptr(out.get("sf_row")), _ptr(out.get("g_row")),
+                                _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("g_col")),
+                                sf_layout, _stream(stream))
+    _check(st, "fp4q_rht16_quantize_sr")
+    return out
+
+
+def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
+         a_global=None, b_global=None, K=None, m_offsets=None, out=None, stream=None):
+    """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
+    Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16."""
+    M = a.shape[0]
+    grouped = m_offsets is not None
+    N = b.shape[1] if grouped else b.shape[0]
+    if K is None:
+        K = a.shape[1] * (2 if recipe == FP8Q_NVFP4 else 1)
+    c = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
+    args = GemmArgs()
+    args.recipe, args.layout = recipe, layout
+    args.M, args.N, args.K = M, N, K
+    args.a, args.lda = a.data_ptr(), a.stride(0)
+    args.b, args.ldb = b.data_ptr(), b.stride(-2)
+    args.a_scale = a_scale.data_ptr() if a_scale is not None else None
+    args.b_scale = b_scale.data_ptr() if b_scale is not None else None
+    args.ld_sa = ld_sa if ld_sa is not None else (a_scale.shape[-1] if (a_scale is not None and a_scale.dim() == 2) else 0)
+    args.ld_sb = ld_sb if ld_sb is not None else (b_scale.shape[-1] if (b_scale is not None and b_scale.dim() >= 2) else 0)
+    args.a_global = a_global.data_ptr() if a_global is not None else None
+    args.b_global = b_global.data_ptr() if b_global is not None else None
+    args.c, args.ldc = c.data_ptr(), c.stride(0)
+    args.m_offsets = m_offsets.data_ptr() if grouped else None
+    args.num_groups = (m_offsets.numel() - 1) if grouped else 0
+    _check(fp8q_gemm_blockscaled(args, _stream(stream)), "fp8q_gemm_blockscaled")
+    return c
+
+
+def device_status(stream=None):
+    """Synchronizes the stream; returns and clears the device status word."""
+    return fp8q_get_device_status(_stream(stream))

@@ -1,0 +1,151 @@
+// Device helpers shared by the quantize kernels: BF16 unpacking, E4M3 / E2M1 encoding,
+// the MX exponent rule, Philox4x32-10 and small reductions.  sm_100a only.
+#pragma once
+#include <cfloat>
+#include <cstdint>
+#include <cuda_runtime.h>
+
+namespace fp8q {
+
+// Status word codes written by kernels (match fp8q_status).
+constexpr uint32_t kDevTimeout = 6;
+
+// ------------------------------------------------------------------ BF16
+// A 32-bit word holds two BF16 values, the lower-addressed one in bits 0..15.
+__device__ __forceinline__ float bf16_lo(uint32_t w) { return __uint_as_float(w << 16); }
+__device__ __forceinline__ float bf16_hi(uint32_t w) { return __uint_as_float(w & 0xFFFF0000u); }
+
+// Packed |x| of two BF16 values (sign bits cleared): non-negative BF16 bit patterns order
+// like their values, so a SIMD unsigned 16-bit max gives the larger magnitude exactly.
+__device__ __forceinline__ uint32_t abs2(uint32_t w) { return w & 0x7FFF7FFFu; }
+__device__ __forceinline__ uint32_t max2(uint32_t a, uint32_t b) { return __vmaxu2(a, b); }
+__device__ __forceinline__ uint32_t hmax(uint32_t w) { return max(w & 0xFFFFu, w >> 16); }
+__device__ __forceinline__ float bf16_bits_to_float(uint32_t b16) { return __uint_as_float(b16 << 16); }
+
+__device__ __forceinline__ uint4 ldg_nc_v4(const void* p) {
+  uint4 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v4.u32 {%0, %1, %2, %3}, [%4];"
+               : "=r"(r.x), "=r"(r.y), "=r"(r.z), "=r"(r.w) : "l"(p));
+  return r;
+}
+
+// ------------------------------------------------------------------ E4M3
+// Two FP32 values -> two E4M3 codes, round to nearest even, saturating to +-448
+// ("satfinite"); `lo` lands in bits 0..7.  The PTX instruction puts its first source
+// operand in the upper byte.
+__device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
+// Tile scale: sf = 448 / amax (IEEE division); amax == 0 -> 1; overflow -> FLT_MAX.
+__device__ __forceinline__ float e4m3_sf(float amax) {
+  if (amax == 0.0f) return 1.0f;
+  float sf = __fdiv_rn(448.0f, amax);
+  return (sf > FLT_MAX) ? FLT_MAX : sf;
+}
+
+// E4M3 code -> FP32 (codes 0x7F/0xFF never occur here: the encoder saturates).
+__device__ __forceinline__ float e4m3_to_float(uint32_t c) {
+  uint32_t e = (c >> 3) & 0xF, m = c & 7;
+  float mag = (e == 0) ? (float)m * 0.001953125f                      // m * 2^-9
+                       : __uint_as_float(((e + 120u) << 23) | (m << 20));  // 2^(e-7)(1+m/8)
+  return (c & 0x80) ? -mag : mag;
+}
+
+// ------------------------------------------------------------------ MX (E8M0)
+// Smallest e with amax <= 448 * 2^e from the FP32 bits of amax (amax = 1.f * 2^E:
+// e = E - 8, plus one when the 23-bit fraction exceeds 0x600000 = 0.75); amax == 0 ->
+// -127; clamped to [-127, 127].
+__device__ __forceinline__ int mx_exponent(float amax) {
+  uint32_t b = __float_as_uint(amax) & 0x7FFFFFFFu;
+  if (b == 0) return -127;
+  int E;
+  uint32_t mant;
+  uint32_t ef = b >> 23;
+  if (ef == 0) {                       // FP32 subnormal: normalise
+    int lz = __clz(b);                 // most significant set bit at 31 - lz (< 23)
+    E = (31 - lz) - 149;
+    mant = (b << (lz - 8)) & 0x7FFFFFu;
+  } else {
+    E = (int)ef - 127;
+    mant = b & 0x7FFFFFu;
+  }
+  int e = E - 8 + (mant > 0x600000u ? 1 : 0);
+  return max(-127, min(127, e));
+}
+
+// 2^-e as an exact FP32 value for e in [-127, 127] (2^-127 is subnormal).
+__device__ __forceinline__ float pow2_neg(int e) {
+  int k = -e;
+  return (k >= -126) ? __uint_as_float((uint32_t)(k + 127) << 23) : __uint_as_float(0x00400000u);
+}
+
+// ------------------------------------------------------------------ E2M1
+// Magnitude grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}; code index = grid index.
+__device__ __forceinline__ int e2m1_floor_index(float a) {   // largest i with grid[i] <= a (a < 6)
+  return (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
+}
+__device__ __forceinline__ float e2m1_grid(int i) {
+  // 0, .5, 1, 1.5, 2, 3, 4, 6
+  return (i < 4) ? 0.5f * (float)i : (i == 4 ? 2.0f : (i == 5 ? 3.0f : (i == 6 ? 4.0f : 6.0f)));
+}
+
+// Round to nearest, ties to the even code, saturating at 6.  Returns the 4-bit code.
+__device__ __forceinline__ uint32_t e2m1_rne(float y) {
+  float a = fabsf(y);
+  uint32_t code;
+  if (a >= 6.0f) {
+    code = 7;
+  } else {
+    int i = e2m1_floor_index(a);
+    float mid = 0.5f * (e2m1_grid(i) + e2m1_grid(i + 1));       // exact grid midpoint
+    bool up = (a > mid) || (a == mid && (i & 1));
+    code = (uint32_t)(i + (up ? 1 : 0));
+  }
+  return code | ((__float_as_uint(y) >> 28) & 8u);
+}
+
+// Stochastic rounding with one 32-bit random word: up iff (word >> 8) * 2^-24 < p,
+// p = (|y| - lo) / (hi - lo) (exact: the gaps are powers of two).
+__device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t word) {
+  float a = fabsf(y);
+  uint32_t code;
+  if (a >= 6.0f) {
+    code = 7;
+  } else {
+    int i = e2m1_floor_index(a);
+    float lo = e2m1_grid(i);
+    float inv_gap = (i < 4) ? 2.0f : (i < 6 ? 1.0f : 0.5f);
+    float p = (a - lo) * inv_gap;
+    float u = (float)(word >> 8) * 5.9604644775390625e-08f;   // 2^-24
+    code = (uint32_t)(i + (u < p ? 1 : 0));
+  }
+  return code | ((__float_as_uint(y) >> 28) & 8u);
+}
+
+// ------------------------------------------------------------------ Philox4x32-10
+// Salmon, Moraes, Dror, Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11).
+__device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    if (r) {
+      k0 += 0x9E3779B9u;
+      k1 += 0xBB67AE85u;
+    }
+    uint32_t hi0 = __umulhi(0xD2511F53u, c.x), lo0 = 0xD2511F53u * c.x;
+    uint32_t hi1 = __umulhi(0xCD9E8D57u, c.z), lo1 = 0xCD9E8D57u * c.z;
+    c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// ------------------------------------------------------------------ MMA-tiled scale layout
+// Byte offset of scale (row r, scale column c) with `s4` = ceil(scale columns / 4) atoms
+// per 128-row band.
+__device__ __forceinline__ int64_t sf_tiled_offset(int64_t r, int64_t c, int64_t s4) {
+  return (((r >> 7) * s4 + (c >> 2)) << 9) + ((r & 31) << 4) + (((r >> 5) & 3) << 2) + (c & 3);
+}
+
+}  // namespace fp8q

@@ -1,0 +1,78 @@
+// Host-side launch interfaces of the kernels (internal to the library).
+#pragma once
+#include <cstdint>
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+namespace fp8q {
+
+enum { kTile1x128 = 0, kTile128 = 1, kTileMX = 2 };
+
+struct TileQuantParams {
+  const uint16_t* x;
+  int64_t rows, cols, ld_x;
+  uint8_t* q_row;
+  void* s_row;      // float* (1x128, 128x128) or uint8_t* (MX)
+  int64_t ld_s_row;  // 1x128: scale row stride; 128x128: K/128
+  uint8_t* q_col;
+  void* s_col;
+  int64_t ld_s_col;
+  int tiles_c;      // 128-column tiles per 128-row band
+  int sf_tiled;     // MX scale bytes in the MMA-tiled layout
+};
+
+cudaError_t launch_tile_quant(int mode, bool row, bool col, const TileQuantParams& p,
+                              int64_t tiles, cudaStream_t s);
+
+// Per-tensor current scaling: amax pass into *amax_bits (zeroed by the caller), then cast.
+cudaError_t launch_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x,
+                               uint32_t* amax_bits, cudaStream_t s);
+cudaError_t launch_tensor_cast(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x,
+                               const uint32_t* amax_bits, uint8_t* q, float* s_dec,
+                               cudaStream_t s);
+
+struct Fp4QuantParams {
+  const uint16_t* x;
+  int64_t rows, cols, ld_x;
+  int rht_row, rht_col, sr_row, sr_col;
+  uint32_t rht_k0, rht_k1, sr_k0, sr_k1;
+  uint8_t* q_row;
+  uint8_t* sf_row;
+  float* g_row;
+  uint8_t* q_col;
+  uint8_t* sf_col;
+  float* g_col;
+  int sf_tiled;
+  int tiles_c;
+  uint32_t* amax_bits;  // [0]: rowwise output's global amax, [1]: colwise output's
+};
+
+cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
+cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
+
+// ------------------------------------------------------------------ GEMM
+struct GemmParams {
+  int recipe;       // fp8q_recipe
+  int layout;       // fp8q_layout
+  int M, N, K;
+  const float* sa;  // BLOCKWISE: A decode scales, sa[kb * ld_sa + m]
+  int64_t ld_sa;
+  const float* sb;  // BLOCKWISE: B scales (indexed per layout)
+  int64_t ld_sb;
+  const float* a_global;
+  const float* b_global;
+  uint16_t* c;      // BF16 row-major
+  int64_t ldc;
+  const uint8_t* sfa;  // MX / NVFP4: MMA-tiled scale images
+  const uint8_t* sfb;
+  int64_t sfa_s4, sfb_s4;  // atoms per 128-row band (ceil(scale columns / 4))
+  const int32_t* m_offsets;
+  int num_groups;
+  int tiles_m, tiles_n;    // output tile grid (non-grouped)
+  uint32_t* status;        // device status word
+};
+
+cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
+                        const CUtensorMap& tma_sb, int num_sms, cudaStream_t s);
+
+}  // namespace fp8q

@@ -1,0 +1,318 @@
+// NVFP4 quantization with the 16x16 random Hadamard transform and stochastic rounding.
+//
+// "NVIDIA developed a method to train neural networks in 4-bit precision", section "How it
+// works": 4-bit (E2M1) values, 16x16 random Hadamard transforms applied to gradient
+// inputs, stochastic rounding.  The two-level scale (E4M3 per 16 elements, FP32 per
+// tensor) keeps every block scale inside the E4M3 range: S_g = 2688 / G maps the tensor
+// amax G to 448 * 6.
+//
+// Two passes over the BF16 input: (1) the global amax of each requested output (after its
+// transform), one atomicMax per CTA into the library's scratch words; (2) recompute the
+// transform, per-16 block amax, E4M3 block scale, encode scale, and E2M1 codes by
+// round-to-nearest-even or by Philox4x32-10 stochastic rounding.
+//
+// One CTA (256 threads) handles a 128x128 tile.  Warp w owns rows 16w..16w+15, lane l
+// owns columns 4l..4l+3, so a thread holds a 16x4 sub-block:
+//   * colwise (along rows) 16-element groups and blocks are entirely in-thread, so the
+//     transform's butterflies and the block amax need no shuffles;
+//   * rowwise 16-element groups span 4 lanes (2 xor-shuffles for the amax, and for the
+//     two upper butterfly stages when the rowwise transform is on);
+//   * one Philox call yields the 4 words of 4 consecutive output elements in either
+//     direction.
+// The transposed colwise codes are staged in shared memory and stored as 64-byte rows.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace fp8q {
+
+namespace {
+
+constexpr uint32_t kRhtCounterTag = 0x52485431u;
+
+__device__ __forceinline__ uint2 ldg_nc_v2(const void* p) {
+  uint2 r;
+  asm volatile("ld.global.nc.L1::no_allocate.v2.u32 {%0, %1}, [%2];" : "=r"(r.x), "=r"(r.y) : "l"(p));
+  return r;
+}
+
+__device__ __forceinline__ float flip(float v, uint32_t signs, int i) {
+  return __uint_as_float(__float_as_uint(v) ^ (((signs >> i) & 1u) << 31));
+}
+
+// Butterflies h = 1, 2, 4, 8 over 16 in-thread values, then the 1/4 normalisation.
+__device__ __forceinline__ void fwht16(float (&e)[16]) {
+#pragma unroll
+  for (int h = 1; h < 16; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 16; ++k) {
+      if ((k & h) == 0) {
+        const float a = e[k], b = e[k + h];
+        e[k] = __fadd_rn(a, b);
+        e[k + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 16; ++k) e[k] = __fmul_rn(e[k], 0.25f);
+}
+
+// Rowwise transform of one row's 4 values held by this lane (positions 4*(lane&3)..+3 of
+// the 16-element group); the partner lanes supply the other 12.
+__device__ __forceinline__ void rht_row4(float (&e)[4], uint32_t signs, int lane) {
+  const int base = (lane & 3) * 4;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) e[j] = flip(e[j], signs, base + j);
+#pragma unroll
+  for (int h = 1; h < 4; h <<= 1) {
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      if ((k & h) == 0) {
+        const float a = e[k], b = e[k + h];
+        e[k] = __fadd_rn(a, b);
+        e[k + h] = __fsub_rn(a, b);
+      }
+    }
+  }
+#pragma unroll
+  for (int s = 1; s <= 2; s <<= 1) {          // h = 4 (lane ^ 1), h = 8 (lane ^ 2)
+    const bool upper = (lane & s) != 0;
+#pragma unroll
+    for (int k = 0; k < 4; ++k) {
+      const float o = __shfl_xor_sync(0xFFFFFFFFu, e[k], s);
+      e[k] = upper ? __fsub_rn(o, e[k]) : __fadd_rn(e[k], o);
+    }
+  }
+#pragma unroll
+  for (int k = 0; k < 4; ++k) e[k] = __fmul_rn(e[k], 0.25f);
+}
+
+__device__ __forceinline__ float global_scale(uint32_t amax_bits) {
+  const float G = __uint_as_float(amax_bits);
+  if (G == 0.0f) return 1.0f;
+  const float s = __fdiv_rn(2688.0f, G);
+  return (s > FLT_MAX) ? FLT_MAX : s;
+}
+
+// E4M3 block scale and the matching encode scale for block amax `m`.
+__device__ __forceinline__ void block_scale(float m, float S_g, uint32_t& sb, float& enc) {
+  const float t = __fmul_rn(__fdiv_rn(m, 6.0f), S_g);
+  sb = cvt_e4m3x2(t, 0.0f) & 0xFFu;
+  enc = (sb == 0) ? 0.0f : __fdiv_rn(S_g, e4m3_to_float(sb));
+}
+
+__device__ __forceinline__ uint32_t rht_signs(const Fp4QuantParams& P) {
+  return philox4x32_10(make_uint4(0, 0, 0, kRhtCounterTag), P.rht_k0, P.rht_k1).x & 0xFFFFu;
+}
+
+struct Tile {
+  int64_t r0, c0, col;
+  bool cok;
+  int lane, w;
+};
+
+__device__ __forceinline__ Tile tile_coords(const Fp4QuantParams& P) {
+  Tile T;
+  T.lane = threadIdx.x & 31;
+  T.w = threadIdx.x >> 5;
+  T.r0 = (int64_t)(blockIdx.x / P.tiles_c) * 128;
+  T.c0 = (int64_t)(blockIdx.x % P.tiles_c) * 128;
+  T.col = T.c0 + T.lane * 4;
+  T.cok = T.col < P.cols;
+  return T;
+}
+
+__device__ __forceinline__ void load16x4(const Fp4QuantParams& P, const Tile& T, float (&x)[16][4]) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) {
+    const int64_t row = T.r0 + T.w * 16 + i;
+    const uint2 v = (T.cok && row < P.rows) ? ldg_nc_v2(P.x + row * P.ld_x + T.col) : make_uint2(0, 0);
+    x[i][0] = bf16_lo(v.x);
+    x[i][1] = bf16_hi(v.x);
+    x[i][2] = bf16_lo(v.y);
+    x[i][3] = bf16_hi(v.y);
+  }
+}
+
+__device__ __forceinline__ void block_max_atomic(float m, uint32_t* dst) {
+  __shared__ float red[8];
+  uint32_t b = __float_as_uint(m);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) b = max(b, __shfl_xor_sync(0xFFFFFFFFu, b, s));
+  __syncthreads();
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = __uint_as_float(b);
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t r = __float_as_uint(red[0]);
+    for (int k = 1; k < 8; ++k) r = max(r, __float_as_uint(red[k]));
+    if (r) atomicMax(dst, r);
+  }
+}
+
+}  // namespace
+
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(256) fp4_amax_kernel(const __grid_constant__ Fp4QuantParams P) {
+  const Tile T = tile_coords(P);
+  float x[16][4];
+  load16x4(P, T, x);
+  const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
+  float m_plain = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m_plain = fmaxf(m_plain, fabsf(x[i][j]));
+  if (ROW) {
+    float m = m_plain;
+    if (P.rht_row) {
+      m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) {
+        float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
+        rht_row4(e, signs, T.lane);
+#pragma unroll
+        for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(e[j]));
+      }
+    }
+    block_max_atomic(m, P.amax_bits);
+  }
+  if (COL) {
+    float m = m_plain;
+    if (P.rht_col) {
+      m = 0.0f;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        float e[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) e[i] = flip(x[i][j], signs, i);
+        fwht16(e);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+      }
+    }
+    block_max_atomic(m, P.amax_bits + 1);
+  }
+}
+
+template <bool ROW, bool COL>
+__global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
+  __shared__ __align__(16) uint8_t tq[COL ? 128 * 64 : 16];
+  const Tile T = tile_coords(P);
+  float x[16][4];
+  load16x4(P, T, x);
+  const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
+
+  if (ROW) {
+    const float S_g = global_scale(P.amax_bits[0]);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_row = __frcp_rn(S_g);
+    const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int64_t row = T.r0 + T.w * 16 + i;
+      float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
+      if (P.rht_row) rht_row4(e, signs, T.lane);
+      float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+      uint32_t sb;
+      float enc;
+      block_scale(m, S_g, sb, enc);
+      uint32_t codes = 0;
+      if (P.sr_row) {
+        const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u),
+                                      P.sr_k0, P.sr_k1);
+        codes = e2m1_sr(__fmul_rn(e[0], enc), r.x) | (e2m1_sr(__fmul_rn(e[1], enc), r.y) << 4) |
+                (e2m1_sr(__fmul_rn(e[2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[3], enc), r.w) << 12);
+      } else {
+        codes = e2m1_rne(__fmul_rn(e[0], enc)) | (e2m1_rne(__fmul_rn(e[1], enc)) << 4) |
+                (e2m1_rne(__fmul_rn(e[2], enc)) << 8) | (e2m1_rne(__fmul_rn(e[3], enc)) << 12);
+      }
+      if (row < P.rows && T.cok) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)codes;
+      if ((T.lane & 3) == 0) {
+        const int64_t kc = T.col >> 4;
+        if (P.sf_tiled) {
+          if (kc < s4 * 4) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+        } else if (row < P.rows && kc < nsf) {
+          P.sf_row[row * nsf + kc] = (uint8_t)sb;
+        }
+      }
+    }
+  }
+
+  if (COL) {
+    const float S_g = global_scale(P.amax_bits[1]);
+    if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_col = __frcp_rn(S_g);
+    const int64_t nsf = P.rows >> 4, s4 = (nsf + 3) >> 2;
+    const int64_t kr = (T.r0 >> 4) + T.w;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int64_t cg = T.col + j;
+      float e[16];
+#pragma unroll
+      for (int i = 0; i < 16; ++i) e[i] = P.rht_col ? flip(x[i][j], signs, i) : x[i][j];
+      if (P.rht_col) fwht16(e);
+      float m = 0.0f;
+#pragma unroll
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+      uint32_t sb;
+      float enc;
+      block_scale(m, S_g, sb, enc);
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int q = 0; q < 4; ++q) {
+        uint32_t c4;
+        if (P.sr_col) {
+          const uint64_t blk = (uint64_t)(cg * P.rows + T.r0 + T.w * 16 + 4 * q) >> 2;
+          const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 1u),
+                                        P.sr_k0, P.sr_k1);
+          c4 = e2m1_sr(__fmul_rn(e[4 * q], enc), r.x) | (e2m1_sr(__fmul_rn(e[4 * q + 1], enc), r.y) << 4) |
+               (e2m1_sr(__fmul_rn(e[4 * q + 2], enc), r.z) << 8) |
+               (e2m1_sr(__fmul_rn(e[4 * q + 3], enc), r.w) << 12);
+        } else {
+          c4 = e2m1_rne(__fmul_rn(e[4 * q], enc)) | (e2m1_rne(__fmul_rn(e[4 * q + 1], enc)) << 4) |
+               (e2m1_rne(__fmul_rn(e[4 * q + 2], enc)) << 8) | (e2m1_rne(__fmul_rn(e[4 * q + 3], enc)) << 12);
+        }
+        if (q < 2) lo |= c4 << (16 * q);
+        else hi |= c4 << (16 * (q - 2));
+      }
+      const int c = T.lane * 4 + j;
+      *(uint2*)&tq[c * 64 + ((T.w ^ ((c >> 2) & 7)) * 8)] = make_uint2(lo, hi);
+      if (P.sf_tiled) {
+        if (kr < s4 * 4) P.sf_col[sf_tiled_offset(cg, kr, s4)] = (uint8_t)sb;
+      } else if (cg < P.cols && kr < nsf) {
+        P.sf_col[cg * nsf + kr] = (uint8_t)sb;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int c = pass * 64 + (threadIdx.x >> 2), h = threadIdx.x & 3;
+      const int64_t cg = T.c0 + c, rg = T.r0 + 32 * h;
+      const uint2 a = *(const uint2*)&tq[c * 64 + (((2 * h) ^ ((c >> 2) & 7)) * 8)];
+      const uint2 b = *(const uint2*)&tq[c * 64 + (((2 * h + 1) ^ ((c >> 2) & 7)) * 8)];
+      uint8_t* dst = P.q_col + cg * (P.rows >> 1) + (rg >> 1);
+      if (cg < P.cols) {
+        if (rg + 32 <= P.rows) *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
+        else if (rg + 16 <= P.rows) *(uint2*)dst = a;
+      }
+    }
+  }
+}
+
+cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
+  const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
+  if (row && col) fp4_amax_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else if (row) fp4_amax_kernel<true, false><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else fp4_amax_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
+  const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
+  if (row && col) fp4_quant_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else if (row) fp4_quant_kernel<true, false><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else fp4_quant_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  return cudaGetLastError();
+}
+
+}  // namespace fp8q

@@ -1,0 +1,217 @@
+/*
+ * fp8q.h - C ABI of the B200 (sm_100a) library for online fine-grained quantization and
+ * block-scaled low-precision GEMM.
+ *
+ * Sources of the operations (pages cited by title and section):
+ *   [DSV3]  "Can you explain the role of FP8 precision in DeepSeek-V3 training":
+ *           "Fine-grained quantization" (1x128 activation tiles, 128x128 weight blocks,
+ *           one scale each), "Online quantization" (scales from the live amax),
+ *           "Increased accumulation precision" (partial sums promoted to FP32 at fixed
+ *           intervals), "Unified E4M3 format" (E4M3 for all tensors), "Mixed-precision
+ *           framework" (the compute-heavy GEMMs in FP8).
+ *   [NeMo]  "Accelerating FP8 training performance with the NVIDIA NeMo framework":
+ *           per-tensor and MXFP8 (blocks of 32 values) scaling recipes.
+ *   [NVFP4] "NVIDIA developed a method to train neural networks in 4-bit precision",
+ *           "How it works": 4-bit values, 16x16 random Hadamard transforms on gradient
+ *           inputs, stochastic rounding.
+ *
+ * Conventions for every call:
+ *   - Tensor pointers are DEVICE pointers owned by the caller; the library never frees
+ *     or keeps them.  BF16 inputs are raw bit patterns (uint16).  Matrices are row-major.
+ *   - `stream` is a cudaStream_t passed as void* (NULL = legacy default stream).  Every
+ *     call is asynchronous on that stream: it validates its arguments on the host,
+ *     enqueues its kernels and returns.
+ *   - The return value reports host-side validation and launch only.  A kernel that gives
+ *     up (a bounded wait that ran out) records a code in a per-device status word that
+ *     fp8q_get_device_status() reads; faults surface as CUDA errors on the next sync.
+ *   - Inputs are assumed finite; NaN/Inf inputs give unspecified codes but never fault.
+ *   - The library allocates no device memory for tensors.  Calls that need a global amax
+ *     (per-tensor and NVFP4 quantization) and the status word use a small per-device
+ *     scratch pool the library allocates on first use and keeps until
+ *     fp8q_release_scratch() or process exit.
+ *
+ * Quantization rules (the readings the pages leave open, shared by the CPU oracle):
+ *   E4M3 is OCP "E4M3FN" (max 448), encoded round-to-nearest-even with saturation.
+ *   1x128 / 128x128 / per-tensor: sf = 448 / amax (FP32 IEEE division; amax == 0 -> 1;
+ *   overflow -> FLT_MAX), codes = E4M3(fp32(x * sf)), stored decode scale = 1 / sf.
+ */
+#ifndef FP8Q_H
+#define FP8Q_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FP8Q_OK = 0,
+  FP8Q_ERR_NULL = 1,        /* a required pointer is NULL                            */
+  FP8Q_ERR_SHAPE = 2,       /* a size, stride or block-multiple requirement fails     */
+  FP8Q_ERR_ALIGN = 3,       /* a pointer or leading dimension is not 16-byte aligned  */
+  FP8Q_ERR_UNSUPPORTED = 4, /* valid request this build does not implement            */
+  FP8Q_ERR_CUDA = 5,        /* a CUDA runtime/driver call or kernel launch failed     */
+  FP8Q_ERR_TIMEOUT = 6      /* (device status) a bounded wait inside a kernel ran out */
+} fp8q_status;
+
+/* Byte layout of MX (E8M0) and NVFP4 (E4M3) scale factors. */
+typedef enum {
+  FP8Q_SF_ROWMAJOR = 0,  /* sf[r * n_sf_cols + c]                                     */
+  FP8Q_SF_MMA_TILED = 1  /* per 128 rows x 4 scale columns, 512 contiguous bytes:
+                            offset = ((r/128) * ceil(n_sf_cols/4) + c/4) * 512
+                                     + (r%32) * 16 + ((r%128)/32) * 4 + c%4;
+                            rows padded to 128 and scale columns to 4, padding bytes 0.
+                            This is the image the block-scaled tensor-core MMA reads
+                            into tensor memory; the MX and NVFP4 GEMMs require it.       */
+} fp8q_sf_layout;
+
+typedef enum {
+  FP8Q_BLOCKWISE = 0,  /* [DSV3] 1x128 x 128x128 (or 1x128 x 1x128) FP32 scales, E4M3 */
+  FP8Q_MXFP8 = 1,      /* [NeMo] E4M3 with E8M0 scales per 32 along K                  */
+  FP8Q_PERTENSOR = 2,  /* [NeMo] E4M3 with one FP32 decode scale per operand           */
+  FP8Q_NVFP4 = 3       /* [NVFP4] E2M1, E4M3 scales per 16 along K, FP32 tensor scale  */
+} fp8q_recipe;
+
+/* Selects how the blockwise B scales are indexed (the A scales are always 1x128). */
+typedef enum {
+  FP8Q_FPROP = 0,  /* B = W^T (N x K codes); sb[(n/128) * ld_sb + k/128]  (128x128)    */
+  FP8Q_DGRAD = 1,  /* B = W   (N x K codes); sb[(k/128) * ld_sb + n/128]  (128x128)    */
+  FP8Q_WGRAD = 2   /* B = dY^T (N x K codes, K = tokens); sb[(k/128) * ld_sb + n] (1x128)*/
+} fp8q_layout;
+
+/* NVFP4 per-direction flags for `rht` and `sr`. */
+#define FP4Q_ROW 1  /* apply to the rowwise output (quantized along columns)           */
+#define FP4Q_COL 2  /* apply to the colwise output (quantized along rows, transposed)  */
+
+/* [DSV3] "Fine-grained quantization", "Online quantization": 1x128 tiles.
+ * x: BF16 rows x cols, row stride ld_x elements (ld_x % 8 == 0, x 16-byte aligned).
+ * Rowwise (needs cols % 128 == 0; any rows >= 0): one scale per 128 consecutive
+ *   elements of a row -> q_row[r * cols + c] (E4M3, contiguous rows x cols) and
+ *   s_row[(c/128) * ld_s_row + r] (FP32 decode scales, MN-major, ld_s_row >= rows,
+ *   ld_s_row % 4 == 0).
+ * Colwise (needs rows % 128 == 0; cols % 16 == 0): one scale per 128 consecutive
+ *   elements of a column, output transposed: q_col[c * rows + r] (cols x rows,
+ *   K-major in the row index: the wgrad operands) and s_col[(r/128) * ld_s_col + c]
+ *   (ld_s_col >= cols, % 4 == 0).
+ * Either output pair may be NULL (not produced); both NULL is FP8Q_ERR_NULL.
+ * x is read once for both outputs.  rows == 0 or cols == 0 -> FP8Q_OK, nothing launched. */
+fp8q_status fp8q_quantize_1x128(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                uint8_t* q_row, float* s_row, int64_t ld_s_row,
+                                uint8_t* q_col, float* s_col, int64_t ld_s_col,
+                                void* stream);
+
+/* [DSV3] "Fine-grained quantization": 128x128 weight blocks.
+ * w: BF16 K x N (K % 128 == 0, N % 128 == 0), row stride ld_w (% 8 == 0).
+ * q_t: N x K codes (the FPROP B operand); q: K x N codes (the DGRAD B operand); the two
+ * hold the same codes transposed; either may be NULL.  s: FP32 decode scales
+ * [N/128][K/128] (s[(n/128) * (K/128) + k/128]), required. */
+fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t ld_w,
+                                  uint8_t* q_t, uint8_t* q, float* s, void* stream);
+
+/* [NeMo] MXFP8: 32-element blocks, E8M0 scale = smallest e with amax <= 448 * 2^e
+ * (amax == 0 -> e = -127; e clamped to [-127, 127]; byte e + 127), codes
+ * E4M3(fp32(x * 2^-e)).
+ * Rowwise (cols % 32 == 0): q_row rows x cols, e8m0_row for (rows, cols/32).
+ * Colwise (rows % 32 == 0, cols % 16 == 0): transposed q_col cols x rows, e8m0_col for
+ *   (cols, rows/32).
+ * Scale bytes use `sf_layout`; size buffers with fp8q_sf_bytes(FP8Q_MXFP8, outer, inner,
+ * layout) (outer = rows of the code matrix, inner = its columns).  Either pair may be NULL. */
+fp8q_status fp8q_quantize_mx32(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                               uint8_t* q_row, uint8_t* e8m0_row,
+                               uint8_t* q_col, uint8_t* e8m0_col,
+                               fp8q_sf_layout sf_layout, void* stream);
+
+/* [NeMo] per-tensor current scaling: amax of the whole tensor, then codes
+ * q[r * cols + c] and one FP32 decode scale *s_dec (device).  cols % 8 == 0.
+ * Two kernels (amax, cast) on `stream`; the amax lives in the library's scratch pool. */
+fp8q_status fp8q_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                 uint8_t* q, float* s_dec, void* stream);
+
+/* [NVFP4] 4-bit quantization with optional 16x16 random Hadamard transform and
+ * stochastic rounding.
+ *   G = amax of the (transformed) tensor; S_g = 2688 / G (G == 0 -> 1);
+ *   per 16 elements along the quantized dim: sb = E4M3(fp32(amax_b / 6) * S_g),
+ *   enc = S_g / decode(sb) (0 if sb == 0), y = x * enc, q = E2M1(y) by
+ *   round-to-nearest-even or stochastic rounding; stored g_dec = 1 / S_g.
+ *   RHT (per direction in `rht`, FP4Q_ROW / FP4Q_COL): 16 signs from Philox4x32-10
+ *   (counter (0,0,0,0x52485431), key rht_seed, word 0 bits 0..15, 1 -> -1); each group of
+ *   16 along the quantized dim is sign-flipped, passed through the butterflies h = 1, 2,
+ *   4, 8 in FP32 and scaled by 1/4.
+ *   SR (per direction in `sr`): random word = Philox4x32-10 output word (idx & 3) for
+ *   counter (idx>>2 low, idx>>2 high, 0, tag), key sr_seed; idx = linear index of the
+ *   element in that output; tag 0 rowwise, 1 colwise; u = (word >> 8) * 2^-24; round up
+ *   iff u < (|y| - lo) / (hi - lo).
+ * Rowwise (cols % 16 == 0): q_row rows x cols/2 bytes (even element in the low nibble),
+ *   sf_row scale bytes for (rows, cols/16), *g_dec_row.
+ * Colwise (rows % 16 == 0, cols % 16 == 0): transposed, q_col cols x rows/2, sf_col for
+ *   (cols, rows/16), *g_dec_col.
+ * Either triple may be NULL.  Two passes over x (global amax, then quantize). */
+fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                   int rht, uint64_t rht_seed, int sr, uint64_t sr_seed,
+                                   uint8_t* q_row, uint8_t* sf_row, float* g_dec_row,
+                                   uint8_t* q_col, uint8_t* sf_col, float* g_dec_col,
+                                   fp8q_sf_layout sf_layout, void* stream);
+
+/* Arguments of fp8q_gemm_blockscaled: C[M x N] = A[M x K] . B[N x K]^T, both operands
+ * K-major codes, C BF16 row-major (ldc >= N, ldc % 8 == 0, c 16-byte aligned).
+ *   BLOCKWISE [DSV3] "Increased accumulation precision": for every 128-element K chunk the
+ *     tensor cores form the E4M3 partial product in FP32 and CUDA cores add it into an
+ *     FP32 accumulator with the chunk's scales applied:
+ *       C[m,n] = bf16( sum_kb sa[kb * ld_sa + m] * sb(kb, n) * partial_kb[m,n] ),
+ *     sb by `layout`.  K % 128 == 0.  a_scale/b_scale are float*.
+ *   MXFP8: codes E4M3, scales E8M0 in FP8Q_SF_MMA_TILED layout for (M, K/32) and
+ *     (N, K/32), applied by the hardware.  K % 32 == 0.
+ *   PERTENSOR: codes E4M3; C = (*a_global) * (*b_global) * (A . B^T).  K % 16 == 0.
+ *   NVFP4: packed E2M1 (lda/ldb in BYTES, K/2 bytes per row), E4M3 scales in
+ *     FP8Q_SF_MMA_TILED layout for (M, K/16) and (N, K/16), C scaled by
+ *     (*a_global) * (*b_global).  K % 32 == 0.
+ * lda/ldb: row strides in bytes (% 16 == 0).  a/b 16-byte aligned.
+ * Grouped (MoE, BLOCKWISE/FPROP only) when num_groups > 0: m_offsets[0..G] (device int32,
+ *   non-decreasing, m_offsets[0] == 0, m_offsets[G] == M) delimit each expert's rows of A
+ *   and C; B is [G][N][K] (expert g at b + g * N * ldb) and b_scale [G][N/128][K/128]
+ *   (expert g at g * (N/128) * ld_sb floats).  The kernel reads the offsets on the device
+ *   and builds its tile schedule there (at most M/128 + G row tiles), so the host needs
+ *   no copy of them.
+ * M, N >= 0 arbitrary (tails masked at the store). */
+typedef struct {
+  fp8q_recipe recipe;
+  fp8q_layout layout;
+  int64_t M, N, K;
+  const void* a;
+  const void* a_scale;
+  int64_t lda, ld_sa;
+  const void* b;
+  const void* b_scale;
+  int64_t ldb, ld_sb;
+  const float* a_global;
+  const float* b_global;
+  void* c;
+  int64_t ldc;
+  const int32_t* m_offsets;
+  int32_t num_groups;
+} fp8q_gemm_args;
+
+fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);
+
+/* Bytes of a scale-factor buffer: recipe MXFP8 (inner/32 scale columns) or NVFP4
+ * (inner/16), `outer` rows, in `layout`.  Returns 0 for other recipes. */
+size_t fp8q_sf_bytes(fp8q_recipe recipe, int64_t outer, int64_t inner, fp8q_sf_layout layout);
+
+/* Synchronizes `stream`, returns and clears the current device's status word
+ * (FP8Q_OK, or FP8Q_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call). */
+fp8q_status fp8q_get_device_status(void* stream);
+
+/* Frees the current device's scratch pool (after a device sync).  Optional. */
+fp8q_status fp8q_release_scratch(void);
+
+const char* fp8q_status_string(fp8q_status s);
+
+/* Library version, e.g. "fp8q 0.1.0 sm_100a". */
+const char* fp8q_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FP8Q_H */

@@ -32,14 +32,19 @@ def rht_signs(rht_seed):
 
 
 def fwht16_stages(v):
-    """In-place-order butterflies h = 1, 2, 4, 8 on the last axis (length 16), FP32."""
+    """Butterflies h = 1, 2, 4, 8 on the last axis (length 16), FP32.
+
+    For stage h the 16 positions split into 16 / (2h) blocks of [i .. i+h) (bit h clear)
+    followed by [i+h .. i+2h) (bit h set); each pair becomes (a + b, a - b)."""
     v = np.array(v, dtype=np.float32, copy=True)
+    lead = v.shape[:-1]
     for h in (1, 2, 4, 8):
-        idx = np.array([i for i in range(16) if (i & h) == 0])
-        a = v[..., idx].copy()
-        b = v[..., idx + h].copy()
-        v[..., idx] = a + b          # float32 + float32 -> float32 (round to nearest even)
-        v[..., idx + h] = a - b
+        w = v.reshape(lead + (16 // (2 * h), 2, h))
+        a = w[..., 0, :].copy()
+        b = w[..., 1, :].copy()
+        w[..., 0, :] = a + b          # float32 + float32 -> float32 (round to nearest even)
+        w[..., 1, :] = a - b
+        v = w.reshape(lead + (16,))
     return v
 
 

@@ -1,0 +1,147 @@
+"""The C-ABI library loads on a machine without a GPU, exports every function include/fp8q.h
+declares, and its host-side validation rejects bad arguments with the documented status
+codes before touching the device (no compute call is made here)."""
+import ctypes
+import os
+import re
+import subprocess
+
+import pytest
+
+import fp4_precision_gemm_b200 as fq
+
+HEADER = os.path.join(os.path.dirname(os.path.dirname(os.path.abspath(__file__))), "include", "fp8q.h")
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(fq.library_path):
+        from fp4_precision_gemm_b200 import build
+        build.build()
+    return fq.lib()
+
+
+def declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"\b(fp[48]q_[a-z0-9_]+)\s*\(", src)))
+
+
+def test_header_declares_the_entry_points():
+    names = declared_functions()
+    for required in ("fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32",
+                     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(L):
+    out = subprocess.run(["nm", "-D", "--defined-only", fq.library_path], capture_output=True, text=True,
+                         check=True).stdout
+    exported = {line.split()[-1] for line in out.splitlines() if " T " in line}
+    for name in declared_functions():
+        assert name in exported, name
+        assert hasattr(L, name)
+    assert set(fq.EXPORTED_SYMBOLS) <= exported
+
+
+def test_version_and_status_strings(L):
+    assert fq.fp8q_version().startswith("fp8q ")
+    assert "sm_100a" in fq.fp8q_version()
+    for st in range(7):
+        assert fq.fp8q_status_string(st)
+
+
+def test_sf_bytes(L):
+    assert fq.fp8q_sf_bytes(fq.FP8Q_MXFP8, 256, 512, fq.FP8Q_SF_ROWMAJOR) == 256 * 16
+    assert fq.fp8q_sf_bytes(fq.FP8Q_MXFP8, 200, 96, fq.FP8Q_SF_MMA_TILED) == 256 * 4
+    assert fq.fp8q_sf_bytes(fq.FP8Q_NVFP4, 300, 656, fq.FP8Q_SF_MMA_TILED) == 384 * 44
+    assert fq.fp8q_sf_bytes(fq.FP8Q_BLOCKWISE, 300, 656, fq.FP8Q_SF_MMA_TILED) == 0
+
+
+P = ctypes.c_void_p
+ALIGNED = P(0x10000)          # never dereferenced: validation fails before any launch
+MISALIGNED = P(0x10008)
+
+
+def test_quantize_validation_codes(L):
+    s = P(0)
+    # no outputs at all
+    assert fq.fp8q_quantize_1x128(ALIGNED, 128, 128, 128, None, None, 0, None, None, 0, s) == 1
+    # rowwise needs cols % 128 == 0
+    assert fq.fp8q_quantize_1x128(ALIGNED, 128, 100, 104, ALIGNED, ALIGNED, 128, None, None, 0, s) == 2
+    # ld_x must be >= cols and a multiple of 8
+    assert fq.fp8q_quantize_1x128(ALIGNED, 128, 128, 100, ALIGNED, ALIGNED, 128, None, None, 0, s) == 2
+    # input must be 16-byte aligned
+    assert fq.fp8q_quantize_1x128(MISALIGNED, 128, 128, 128, ALIGNED, ALIGNED, 128, None, None, 0, s) == 3
+    # colwise needs rows % 128 == 0
+    assert fq.fp8q_quantize_1x128(ALIGNED, 100, 128, 128, None, None, 0, ALIGNED, ALIGNED, 128, s) == 2
+    # 128x128 needs both dims multiple of 128 and a scale pointer
+    assert fq.fp8q_quantize_128x128(ALIGNED, 128, 200, 200, ALIGNED, None, ALIGNED, s) == 2
+    assert fq.fp8q_quantize_128x128(ALIGNED, 128, 128, 128, ALIGNED, None, None, s) == 1
+    # MX: bad layout enum, and colwise rows % 32
+    assert fq.fp8q_quantize_mx32(ALIGNED, 64, 64, 64, ALIGNED, ALIGNED, None, None, 7, s) == 4
+    assert fq.fp8q_quantize_mx32(ALIGNED, 48, 64, 64, None, None, ALIGNED, ALIGNED, 0, s) == 2
+    # per-tensor: cols % 8
+    assert fq.fp8q_quantize_tensor(ALIGNED, 4, 12, 16, ALIGNED, ALIGNED, s) == 2
+    # NVFP4: unknown flag bits, cols % 16, partial output triple
+    assert fq.fp4q_rht16_quantize_sr(ALIGNED, 16, 16, 16, 4, 0, 0, 0, ALIGNED, ALIGNED, ALIGNED,
+                                     None, None, None, 0, s) == 4
+    assert fq.fp4q_rht16_quantize_sr(ALIGNED, 16, 24, 24, 0, 0, 0, 0, ALIGNED, ALIGNED, ALIGNED,
+                                     None, None, None, 0, s) == 2
+    assert fq.fp4q_rht16_quantize_sr(ALIGNED, 16, 16, 16, 0, 0, 0, 0, ALIGNED, None, ALIGNED,
+                                     None, None, None, 0, s) == 1
+
+
+def test_quantize_empty_is_ok_without_launch(L):
+    s = P(0)
+    assert fq.fp8q_quantize_1x128(ALIGNED, 0, 128, 128, ALIGNED, ALIGNED, 0, None, None, 0, s) == 0
+    assert fq.fp8q_quantize_128x128(ALIGNED, 0, 128, 128, ALIGNED, None, ALIGNED, s) == 0
+    assert fq.fp8q_quantize_mx32(ALIGNED, 0, 64, 64, ALIGNED, ALIGNED, None, None, 0, s) == 0
+
+
+def _args(**kw):
+    a = fq.GemmArgs()
+    a.recipe, a.layout = fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP
+    a.M, a.N, a.K = 256, 256, 512
+    a.a = a.b = a.c = a.a_scale = a.b_scale = 0x10000
+    a.lda = a.ldb = 512
+    a.ld_sa, a.ld_sb, a.ldc = 256, 4, 256
+    for k, v in kw.items():
+        setattr(a, k, v)
+    return a
+
+
+def test_gemm_validation_codes(L):
+    s = P(0)
+    assert fq.fp8q_gemm_blockscaled(_args(K=500), s) == 2                    # K % 128
+    assert fq.fp8q_gemm_blockscaled(_args(recipe=fq.FP8Q_NVFP4, K=384, lda=192, ldb=192), s) == 2
+    assert fq.fp8q_gemm_blockscaled(_args(ldc=100), s) == 2                  # ldc < N
+    assert fq.fp8q_gemm_blockscaled(_args(lda=520), s) == 2                  # lda % 16
+    assert fq.fp8q_gemm_blockscaled(_args(a=0x10004), s) == 3                # alignment
+    assert fq.fp8q_gemm_blockscaled(_args(a_scale=None), s) == 1
+    assert fq.fp8q_gemm_blockscaled(_args(recipe=9), s) == 4
+    assert fq.fp8q_gemm_blockscaled(_args(recipe=fq.FP8Q_PERTENSOR), s) == 1  # globals missing
+    assert fq.fp8q_gemm_blockscaled(_args(layout=fq.FP8Q_DGRAD, ld_sb=1), s) == 2
+    assert fq.fp8q_gemm_blockscaled(_args(layout=fq.FP8Q_WGRAD, ld_sb=100), s) == 2
+    # grouped only for the blockwise FPROP layout
+    assert fq.fp8q_gemm_blockscaled(_args(recipe=fq.FP8Q_MXFP8, m_offsets=0x10000, num_groups=2), s) == 4
+    assert fq.fp8q_gemm_blockscaled(_args(num_groups=2, m_offsets=None), s) == 1
+    assert L.fp8q_gemm_blockscaled(None, s) == 1
+    # M == 0 or N == 0: nothing to do
+    assert fq.fp8q_gemm_blockscaled(_args(M=0), s) == 0
+    assert fq.fp8q_gemm_blockscaled(_args(N=0), s) == 0
+
+
+def test_product_path_has_no_cpu_fallback():
+    """The binding must raise when the library is absent instead of computing on the host."""
+    import importlib
+    src = open(os.path.join(os.path.dirname(fq.__file__), "__init__.py")).read()
+    assert "oracle" not in src and "numpy" not in src
+    mod = importlib.import_module("fp4_precision_gemm_b200")
+    saved_path, saved_lib = mod.library_path, mod._LIB
+    try:
+        mod.library_path, mod._LIB = "/nonexistent/libfp8q.so", None
+        with pytest.raises(ImportError):
+            mod.lib()
+    finally:
+        mod.library_path, mod._LIB = saved_path, saved_lib

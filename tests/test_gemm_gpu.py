@@ -1,0 +1,311 @@
+"""Block-scaled GEMMs vs the CPU oracle, through the C ABI.
+
+The GPU GEMM consumes operands produced by the GPU quantize kernels (bit-exact with the
+oracle, tested separately); the oracle quantizes the same BF16 inputs itself and computes
+the FP64 product of its dequantized operands.  Acceptance, elementwise:
+    |C_gpu - C_ref| <= 2^-7 |C_ref| + 1e-4 (|A_dq| |B_dq|^T)
+on every element of small shapes (ragged M/N tails, several tiles, many K chunks, more
+tiles than SMs) and on 64 sampled 128x128 tiles of the full-size workloads."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import gemm as G
+from oracle import quant as Q
+
+pytestmark = pytest.mark.gpu
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def check(c_gpu, c_ref, t, what):
+    got = host(c_gpu.float()).astype(np.float64) if isinstance(c_gpu, torch.Tensor) else c_gpu
+    v = G.tolerance_violation(got, c_ref, t)
+    worst = float(v.max())
+    if worst > 0:
+        i = np.unravel_index(int(np.argmax(v)), v.shape)
+        raise AssertionError(f"{what}: {int((v > 0).sum())} elements outside tolerance; worst at {i}: "
+                             f"gpu={got[i]} ref={c_ref[i]} T={t[i]}")
+
+
+def bf(shape, sigma, seed, frac=0.0, fac=1.0):
+    return workloads.normal_bf16(shape, sigma, seed, frac, fac)
+
+
+# ----------------------------------------------------------------------------- blockwise
+@pytest.mark.parametrize("M,K,N", [(256, 512, 256), (300, 384, 384), (256, 4096, 512), (1, 128, 128)])
+def test_blockwise_fprop(cuda_lib, M, K, N):
+    fq = cuda_lib
+    X, W = bf((M, K), 1.0, M + K, 1e-3, 50.0), bf((K, N), 0.02, K + N)
+    qx = fq.quantize_1x128(X.cuda())
+    qw = fq.quantize_128x128(W.cuda())
+    c = fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"], b_scale=qw["s"])
+    assert fq.device_status() == 0
+    ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+    _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+    check(c, ref, t, "fprop")
+
+
+@pytest.mark.parametrize("M,Kw,Nw", [(300, 384, 512), (256, 256, 1024)])
+def test_blockwise_dgrad(cuda_lib, M, Kw, Nw):
+    """dX = dY . W^T with W (Kw x Nw): GEMM N = Kw, K = Nw, B = W's K x N codes."""
+    fq = cuda_lib
+    dY, W = bf((M, Nw), 1e-3, M + Nw), bf((Kw, Nw), 0.02, Kw * 3 + Nw)
+    qd = fq.quantize_1x128(dY.cuda())
+    qw = fq.quantize_128x128(W.cuda())
+    c = fq.gemm(qd["q_row"], qw["q"], fq.FP8Q_BLOCKWISE, fq.FP8Q_DGRAD, a_scale=qd["s_row"], b_scale=qw["s"],
+                ld_sb=Kw // 128)
+    od, osd = Q.quantize_1x128_rowwise(workloads.bf16_bits(dY))
+    ow, _, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_a_1x128(od, osd), G.dequant_b_blockwise(ow, osw, G.DGRAD))
+    check(c, ref, t, "dgrad")
+
+
+@pytest.mark.parametrize("T,Kf,N", [(256, 208, 400), (1024, 256, 512)])
+def test_blockwise_wgrad(cuda_lib, T, Kf, N):
+    """dW = X^T . dY: both operands 1x128 along tokens (colwise, transposed)."""
+    fq = cuda_lib
+    X, dY = bf((T, Kf), 1.0, T + Kf, 1e-3, 50.0), bf((T, N), 1e-3, 2 * T + N)
+    qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
+    qd = fq.quantize_1x128(dY.cuda(), rowwise=False, colwise=True)
+    c = fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                b_scale=qd["s_col"])
+    ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
+    od, osd = Q.quantize_1x128_colwise(workloads.bf16_bits(dY))
+    ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od, osd, G.WGRAD))
+    check(c, ref, t, "wgrad")
+
+
+def test_blockwise_more_tiles_than_sms(cuda_lib):
+    """2048 x 4096 output = 256 tiles: every CTA runs the persistent loop more than once."""
+    fq = cuda_lib
+    M, K, N = 2048, 256, 4096
+    X, W = bf((M, K), 1.0, 91), bf((K, N), 0.02, 92)
+    qx = fq.quantize_1x128(X.cuda())
+    qw = fq.quantize_128x128(W.cuda())
+    c = fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"], b_scale=qw["s"])
+    ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+    _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+    check(c, ref, t, "fprop persistent")
+
+
+def test_grouped_fprop_ragged_experts(cuda_lib):
+    fq = cuda_lib
+    counts = [130, 0, 1, 257, 60, 128]
+    K, N, Gn = 384, 256, len(counts)
+    offs = np.concatenate([[0], np.cumsum(counts)]).astype(np.int32)
+    M = int(offs[-1])
+    A = bf((M, K), 1.0, 31)
+    Ws = [bf((K, N), 0.006, 40 + g) for g in range(Gn)]
+    qa = fq.quantize_1x128(A.cuda())
+    qws = [fq.quantize_128x128(w.cuda()) for w in Ws]
+    B = torch.stack([q["q_t"] for q in qws])              # (G, N, K)
+    SB = torch.stack([q["s"] for q in qws])               # (G, N/128, K/128)
+    c = fq.gemm(qa["q_row"], B, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qa["s_row"], b_scale=SB,
+                ld_sb=K // 128, m_offsets=torch.from_numpy(offs).cuda())
+    oa, osa = Q.quantize_1x128_rowwise(workloads.bf16_bits(A))
+    got = host(c.float()).astype(np.float64)
+    for g in range(Gn):
+        r0, r1 = offs[g], offs[g + 1]
+        if r1 == r0:
+            continue
+        _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(Ws[g]))
+        rows = np.arange(r0, r1)
+        ref, t = G.reference(G.dequant_a_1x128(oa, osa, rows=rows), G.dequant_b_blockwise(owt, osw, G.FPROP))
+        check(got[r0:r1], ref, t, f"grouped expert {g}")
+
+
+# ----------------------------------------------------------------------------- other recipes
+@pytest.mark.parametrize("M,K,N", [(300, 512, 400), (256, 1024, 256)])
+def test_mxfp8(cuda_lib, M, K, N):
+    fq = cuda_lib
+    A, W = bf((M, K), 1.0, M + 7 * K), bf((K, N), 0.02, N + K)
+    qa = fq.quantize_mx32(A.cuda(), rowwise=True, sf_layout=fq.FP8Q_SF_MMA_TILED)
+    qb = fq.quantize_mx32(W.cuda(), rowwise=False, colwise=True, sf_layout=fq.FP8Q_SF_MMA_TILED)
+    c = fq.gemm(qa["q_row"], qb["q_col"], fq.FP8Q_MXFP8, a_scale=qa["e8m0_row"], b_scale=qb["e8m0_col"])
+    oa, ea = Q.quantize_mx_rowwise(workloads.bf16_bits(A))
+    ob, eb = Q.quantize_mx_colwise(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_mx(oa, ea), G.dequant_mx(ob, eb))
+    check(c, ref, t, "mxfp8")
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 512, 400)])
+def test_per_tensor(cuda_lib, M, K, N):
+    fq = cuda_lib
+    A, W = bf((M, K), 1.0, 3 * M + K), bf((K, N), 0.02, 5 * N + K)
+    Wt = W.t().contiguous()
+    qa = fq.quantize_tensor(A.cuda())
+    qb = fq.quantize_tensor(Wt.cuda())
+    c = fq.gemm(qa["q"], qb["q"], fq.FP8Q_PERTENSOR, a_global=qa["s_dec"], b_global=qb["s_dec"])
+    oa, sa = Q.quantize_tensor(workloads.bf16_bits(A))
+    ob, sb = Q.quantize_tensor(workloads.bf16_bits(Wt))
+    ref, t = G.reference(G.dequant_tensor(oa, sa), G.dequant_tensor(ob, sb))
+    check(c, ref, t, "per-tensor")
+
+
+@pytest.mark.parametrize("M,K,N,rht", [(300, 512, 400, False), (256, 1024, 256, True)])
+def test_nvfp4(cuda_lib, M, K, N, rht):
+    fq = cuda_lib
+    A, B = bf((M, K), 1e-3, M + 11 * K, 5e-4, 100.0), bf((N, K), 0.02, N + 13 * K)
+    flag = fq.FP4Q_ROW if rht else 0
+    qa = fq.rht16_quantize_sr(A.cuda(), rht=flag, rht_seed=5, sr=fq.FP4Q_ROW, sr_seed=6,
+                              sf_layout=fq.FP8Q_SF_MMA_TILED)
+    qb = fq.rht16_quantize_sr(B.cuda(), rht=flag, rht_seed=5, sf_layout=fq.FP8Q_SF_MMA_TILED)
+    c = fq.gemm(qa["q_row"], qb["q_row"], fq.FP8Q_NVFP4, a_scale=qa["sf_row"], b_scale=qb["sf_row"],
+                a_global=qa["g_row"], b_global=qb["g_row"], K=K)
+    oa, sa, ga = Q.quantize_nvfp4_rowwise(workloads.bf16_bits(A), rht=rht, rht_seed=5, sr=True, sr_seed=6)
+    ob, sb, gb = Q.quantize_nvfp4_rowwise(workloads.bf16_bits(B), rht=rht, rht_seed=5)
+    ref, t = G.reference(G.dequant_nvfp4(oa, sa, ga), G.dequant_nvfp4(ob, sb, gb))
+    check(c, ref, t, "nvfp4")
+
+
+def test_k_zero_gives_zeros(cuda_lib):
+    fq = cuda_lib
+    a = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
+    s = torch.ones((1, 4), dtype=torch.float32, device="cuda")
+    out = torch.full((4, 8), 7.0, dtype=torch.bfloat16, device="cuda")
+    fq.gemm(a, a[:, :0].new_zeros((8, 128)), fq.FP8Q_BLOCKWISE, a_scale=s, b_scale=s, K=0, out=out)
+    assert float(out.abs().max()) == 0.0
+
+
+# ----------------------------------------------------------------------------- full size, sampled
+def _tiles(M, N, seed):
+    return G.sample_tiles(M, N, 64, seed=seed)
+
+
+def test_llama8b_fprop_dgrad_wgrad_sampled(cuda_lib):
+    """The bench's three GEMMs at M=8192, hidden 4096, FFN 14336 on 64 sampled tiles each."""
+    fq = cuda_lib
+    d = workloads.llama8b(device="cuda")
+    X, W, dY = d["X"], d["W"], d["dY"]
+    qx = fq.quantize_1x128(X, rowwise=True, colwise=True)
+    qw = fq.quantize_128x128(W)
+    qd = fq.quantize_1x128(dY, rowwise=True, colwise=True)
+    Xb, Wb, dYb = workloads.bf16_bits(X), workloads.bf16_bits(W), workloads.bf16_bits(dY)
+    # FPROP (8192, 4096, 14336)
+    c = host(fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"],
+                     b_scale=qw["s"]).float())
+    for m0, n0 in _tiles(8192, 14336, 2):
+        oa, sa = Q.quantize_1x128_rowwise(Xb[m0:m0 + 128])
+        _, owt, sw = Q.quantize_128x128(Wb[:, n0:n0 + 128])
+        ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"fprop tile {m0},{n0}")
+    # DGRAD (8192, 14336, 4096): B = W (4096 x 14336)
+    c = host(fq.gemm(qd["q_row"], qw["q"], fq.FP8Q_BLOCKWISE, fq.FP8Q_DGRAD, a_scale=qd["s_row"],
+                     b_scale=qw["s"], ld_sb=4096 // 128).float())
+    for m0, n0 in _tiles(8192, 4096, 3):
+        oa, sa = Q.quantize_1x128_rowwise(dYb[m0:m0 + 128])
+        ow, _, sw = Q.quantize_128x128(Wb[n0:n0 + 128])            # W rows n0.. (its K), all N
+        ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ow, sw, G.DGRAD))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"dgrad tile {m0},{n0}")
+    # WGRAD (4096, 8192, 14336): A = X^T, B = dY^T, K = tokens
+    c = host(fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                     b_scale=qd["s_col"]).float())
+    for m0, n0 in _tiles(4096, 14336, 4):
+        oa, sa = Q.quantize_1x128_colwise(Xb[:, m0:m0 + 128])
+        ob, sb = Q.quantize_1x128_colwise(dYb[:, n0:n0 + 128])
+        ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"wgrad tile {m0},{n0}")
+    assert fq.device_status() == 0
+
+
+def test_mxfp8_and_per_tensor_fullsize_sampled(cuda_lib):
+    fq = cuda_lib
+    d = workloads.mxfp8(device="cuda")
+    for i, (M, K, N) in enumerate(workloads.MXFP8_GEMMS):
+        A, W = d[f"A{i}"], d[f"W{i}"]
+        qa = fq.quantize_mx32(A, rowwise=True, sf_layout=1)
+        qb = fq.quantize_mx32(W, rowwise=False, colwise=True, sf_layout=1)
+        c = host(fq.gemm(qa["q_row"], qb["q_col"], fq.FP8Q_MXFP8, a_scale=qa["e8m0_row"],
+                         b_scale=qb["e8m0_col"]).float())
+        Ab, Wb = workloads.bf16_bits(A), workloads.bf16_bits(W)
+        for m0, n0 in _tiles(M, N, 10 + i)[:16]:
+            oa, ea = Q.quantize_mx_rowwise(Ab[m0:m0 + 128])
+            ob, eb = Q.quantize_mx_colwise(Wb[:, n0:n0 + 128])
+            ref, t = G.reference(G.dequant_mx(oa, ea), G.dequant_mx(ob, eb))
+            check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"mxfp8 {i} tile {m0},{n0}")
+        del qa, qb
+    # per-tensor comparison variant on the first shape
+    A, W = d["A0"], d["W0"]
+    qa = fq.quantize_tensor(A)
+    Wt = W.t().contiguous()
+    qb = fq.quantize_tensor(Wt)
+    c = host(fq.gemm(qa["q"], qb["q"], fq.FP8Q_PERTENSOR, a_global=qa["s_dec"], b_global=qb["s_dec"]).float())
+    oa, sa = Q.quantize_tensor(workloads.bf16_bits(A))
+    ob, sb = Q.quantize_tensor(workloads.bf16_bits(Wt))       # global scales over whole tensors
+    for m0, n0 in _tiles(8192, 4096, 20)[:8]:
+        ref, t = G.reference(G.dequant_tensor(oa[m0:m0 + 128], sa), G.dequant_tensor(ob[n0:n0 + 128], sb))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"per-tensor tile {m0},{n0}")
+
+
+def test_moe_grouped_fullsize_sampled(cuda_lib):
+    """DeepSeek-V3 expert GEMMs: 32 experts, 16384 tokens x top-8, up and down projections."""
+    fq = cuda_lib
+    for proj in ("up", "down"):
+        d = workloads.moe(device="cuda", proj=proj)
+        A, W, offs = d["A"], d["W"], d["offsets"]
+        Gn, K, N = W.shape
+        qa = fq.quantize_1x128(A)
+        B = torch.empty((Gn, N, K), dtype=torch.uint8, device="cuda")
+        SB = torch.empty((Gn, N // 128, K // 128), dtype=torch.float32, device="cuda")
+        for g in range(Gn):
+            q = fq.quantize_128x128(W[g], plain=False)
+            B[g].copy_(q["q_t"])
+            SB[g].copy_(q["s"])
+        c = host(fq.gemm(qa["q_row"], B, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qa["s_row"], b_scale=SB,
+                         ld_sb=K // 128, m_offsets=offs.cuda()).float())
+        tiles = G.sample_group_tiles(offs.numpy(), N, 64, seed=4)
+        Ab = workloads.bf16_bits(A)
+        for g, m0, m1, n0 in tiles[:24]:
+            oa, sa = Q.quantize_1x128_rowwise(Ab[m0:m1])
+            _, owt, sw = Q.quantize_128x128(workloads.bf16_bits(W[g][:, n0:n0 + 128]))
+            ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+            check(c[m0:m1, n0:n0 + 128].astype(np.float64), ref, t, f"moe {proj} expert {g} tile {m0},{n0}")
+        del qa, B, SB, d
+
+
+def test_nvfp4_fullsize_sampled(cuda_lib):
+    """Llama-3.1-405B-shaped NVFP4 dgrad (8192, 53248, 16384) and wgrad (16384, 8192, 53248)."""
+    fq = cuda_lib
+    d = workloads.nvfp4(device="cuda")
+    X, W, dY = d["X"], d["W"], d["dY"]
+    Xb, Wb, dYb = workloads.bf16_bits(X), workloads.bf16_bits(W), workloads.bf16_bits(dY)
+    qd = fq.rht16_quantize_sr(dY, rowwise=True, colwise=True, rht=fq.FP4Q_COL, rht_seed=5, sr=3, sr_seed=6,
+                              sf_layout=1)
+    qw = fq.rht16_quantize_sr(W, rowwise=True, sf_layout=1)
+    c = host(fq.gemm(qd["q_row"], qw["q_row"], fq.FP8Q_NVFP4, a_scale=qd["sf_row"], b_scale=qw["sf_row"],
+                     a_global=qd["g_row"], b_global=qw["g_row"], K=53248).float())
+    tiles = _tiles(8192, 16384, 5)[:8]
+    rows_a = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
+    rows_b = np.unique(np.concatenate([np.arange(n0, n0 + 128) for _, n0 in tiles]))
+    oa, sa, ga = Q.quantize_nvfp4_rowwise(dYb, sr=True, sr_seed=6, rows=rows_a)
+    ob, sb, gb = Q.quantize_nvfp4_rowwise(Wb, rows=rows_b)
+    ia = {r: i for i, r in enumerate(rows_a)}
+    ib = {r: i for i, r in enumerate(rows_b)}
+    for m0, n0 in tiles:
+        ra = [ia[r] for r in range(m0, m0 + 128)]
+        rb = [ib[r] for r in range(n0, n0 + 128)]
+        ref, t = G.reference(G.dequant_nvfp4(oa[ra], sa[ra], ga), G.dequant_nvfp4(ob[rb], sb[rb], gb))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"nvfp4 dgrad tile {m0},{n0}")
+    del qw, c
+    qx = fq.rht16_quantize_sr(X, rowwise=False, colwise=True, rht=fq.FP4Q_COL, rht_seed=5, sf_layout=1)
+    c = host(fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_NVFP4, a_scale=qx["sf_col"], b_scale=qd["sf_col"],
+                     a_global=qx["g_col"], b_global=qd["g_col"], K=8192).float())
+    tiles = _tiles(16384, 53248, 6)[:8]
+    cols_a = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
+    cols_b = np.unique(np.concatenate([np.arange(n0, n0 + 128) for _, n0 in tiles]))
+    oa, sa, ga = Q.quantize_nvfp4_colwise(Xb, rht=True, rht_seed=5, rows=cols_a)
+    ob, sb, gb = Q.quantize_nvfp4_colwise(dYb, rht=True, rht_seed=5, sr=True, sr_seed=6, rows=cols_b)
+    ia = {r: i for i, r in enumerate(cols_a)}
+    ib = {r: i for i, r in enumerate(cols_b)}
+    for m0, n0 in tiles:
+        ra = [ia[r] for r in range(m0, m0 + 128)]
+        rb = [ib[r] for r in range(n0, n0 + 128)]
+        ref, t = G.reference(G.dequant_nvfp4(oa[ra], sa[ra], ga), G.dequant_nvfp4(ob[rb], sb[rb], gb))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"nvfp4 wgrad tile {m0},{n0}")
+    assert fq.device_status() == 0

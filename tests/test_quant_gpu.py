@@ -1,0 +1,236 @@
+"""Quantize kernels vs the CPU oracle, bit-exact (codes and scales), through the C ABI.
+
+Small shapes span several 128x128 tiles with ragged tails; the edge cases cover all-zero
+tiles, subnormal and maximal BF16 magnitudes and signed zeros; full-size workloads are
+checked on sampled row and column bands (the oracle quantizes the same bands from the same
+BF16 inputs)."""
+import numpy as np
+import pytest
+import torch
+
+import workloads
+from oracle import quant as Q
+
+pytestmark = pytest.mark.gpu
+
+
+def f32bits(a):
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
+
+
+def host(t):
+    return t.detach().cpu().numpy()
+
+
+def crafted_bf16(R, C, seed):
+    """Random data plus edge cases: a zero tile, subnormal magnitudes, BF16 max, -0.0."""
+    x = workloads.normal_bf16((R, C), 1.0, seed, 1e-3, 100.0).float()
+    x[:min(R, 128), :min(C, 128)] = 0.0
+    if R > 130 and C > 256:
+        x[130, 128:256] = torch.tensor(1e-40)                       # subnormal amax tile
+        x[131, 128:256] = torch.tensor(3.3e38)                      # near BF16 max
+        x[132, 128:192] = -0.0
+    return x.to(torch.bfloat16)
+
+
+# ----------------------------------------------------------------------------- 1x128
+@pytest.mark.parametrize("R,C,row,col", [
+    (300, 640, True, False), (384, 656, False, True), (384, 640, True, True),
+    (1, 128, True, False), (128, 16, False, True), (256, 512, True, True)])
+def test_1x128_parity(cuda_lib, R, C, row, col):
+    fq = cuda_lib
+    x = crafted_bf16(R, C, seed=R * 1000 + C)
+    out = fq.quantize_1x128(x.cuda(), rowwise=row, colwise=col)
+    bits = workloads.bf16_bits(x)
+    if row:
+        q, s = Q.quantize_1x128_rowwise(bits)
+        assert np.array_equal(host(out["q_row"]), q)
+        assert np.array_equal(f32bits(host(out["s_row"])[:, :R]), f32bits(s))
+    if col:
+        q, s = Q.quantize_1x128_colwise(bits)
+        assert np.array_equal(host(out["q_col"]), q)
+        assert np.array_equal(f32bits(host(out["s_col"])[:, :C]), f32bits(s))
+
+
+def test_1x128_strided_input(cuda_lib):
+    fq = cuda_lib
+    big = workloads.normal_bf16((256, 1024), 1.0, 77).cuda()
+    x = big[:, 128:640]                                   # row stride 1024 != cols
+    out = fq.quantize_1x128(x, rowwise=True, colwise=True)
+    bits = workloads.bf16_bits(x)
+    q, s = Q.quantize_1x128_rowwise(bits)
+    assert np.array_equal(host(out["q_row"]), q)
+    qc, sc = Q.quantize_1x128_colwise(bits)
+    assert np.array_equal(host(out["q_col"]), qc)
+
+
+# ----------------------------------------------------------------------------- 128x128
+@pytest.mark.parametrize("K,N", [(384, 640), (128, 128), (512, 256)])
+def test_128x128_parity(cuda_lib, K, N):
+    fq = cuda_lib
+    w = crafted_bf16(K, N, seed=K + N)
+    out = fq.quantize_128x128(w.cuda())
+    q, qt, s = Q.quantize_128x128(workloads.bf16_bits(w))
+    assert np.array_equal(host(out["q"]), q)
+    assert np.array_equal(host(out["q_t"]), qt)
+    assert np.array_equal(f32bits(host(out["s"])), f32bits(s))
+
+
+# ----------------------------------------------------------------------------- MX
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("R,C,row,col", [(300, 672, True, False), (352, 656, False, True),
+                                         (384, 640, True, True), (64, 32, True, True)])
+def test_mx32_parity(cuda_lib, layout, R, C, row, col):
+    fq = cuda_lib
+    x = crafted_bf16(R, C, seed=5 * R + C)
+    out = fq.quantize_mx32(x.cuda(), rowwise=row, colwise=col, sf_layout=layout)
+    bits = workloads.bf16_bits(x)
+    if row:
+        q, e = Q.quantize_mx_rowwise(bits)
+        assert np.array_equal(host(out["q_row"]), q)
+        want = Q.sf_to_tiled(e) if layout == 1 else e.ravel()
+        assert np.array_equal(host(out["e8m0_row"]), want)
+    if col:
+        q, e = Q.quantize_mx_colwise(bits)
+        assert np.array_equal(host(out["q_col"]), q)
+        want = Q.sf_to_tiled(e) if layout == 1 else e.ravel()
+        assert np.array_equal(host(out["e8m0_col"]), want)
+
+
+# ----------------------------------------------------------------------------- per tensor
+@pytest.mark.parametrize("R,C", [(300, 648), (1, 8), (128, 4096)])
+def test_per_tensor_parity(cuda_lib, R, C):
+    fq = cuda_lib
+    x = workloads.normal_bf16((R, C), 1.0, R + 3 * C, 1e-3, 50.0)
+    out = fq.quantize_tensor(x.cuda())
+    q, s = Q.quantize_tensor(workloads.bf16_bits(x))
+    assert np.array_equal(host(out["q"]), q)
+    assert f32bits(host(out["s_dec"]))[0] == f32bits(np.float32([s]))[0]
+
+
+# ----------------------------------------------------------------------------- NVFP4
+NV_CASES = [
+    # R, C, row, col, rht, sr
+    (300, 656, True, False, 0, 0),
+    (300, 656, True, False, 1, 1),
+    (368, 656, False, True, 0, 0),
+    (368, 656, False, True, 2, 2),
+    (384, 640, True, True, 2, 3),        # gradient recipe: rowwise SR, colwise RHT + SR
+    (384, 640, True, True, 3, 0),
+    (16, 16, True, True, 3, 3),
+]
+
+
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("R,C,row,col,rht,sr", NV_CASES)
+def test_nvfp4_parity(cuda_lib, layout, R, C, row, col, rht, sr):
+    fq = cuda_lib
+    x = workloads.normal_bf16((R, C), 1e-3, 11 * R + C, 5e-4, 100.0)
+    out = fq.rht16_quantize_sr(x.cuda(), rowwise=row, colwise=col, rht=rht, rht_seed=5, sr=sr, sr_seed=6,
+                               sf_layout=layout)
+    bits = workloads.bf16_bits(x)
+    if row:
+        q, sf, g = Q.quantize_nvfp4_rowwise(bits, rht=bool(rht & 1), rht_seed=5, sr=bool(sr & 1), sr_seed=6)
+        assert np.array_equal(host(out["q_row"]), q)
+        want = Q.sf_to_tiled(sf) if layout == 1 else sf.ravel()
+        assert np.array_equal(host(out["sf_row"]), want)
+        assert f32bits(host(out["g_row"]))[0] == f32bits(np.float32([g]))[0]
+    if col:
+        q, sf, g = Q.quantize_nvfp4_colwise(bits, rht=bool(rht & 2), rht_seed=5, sr=bool(sr & 2), sr_seed=6)
+        assert np.array_equal(host(out["q_col"]), q)
+        want = Q.sf_to_tiled(sf) if layout == 1 else sf.ravel()
+        assert np.array_equal(host(out["sf_col"]), want)
+        assert f32bits(host(out["g_col"]))[0] == f32bits(np.float32([g]))[0]
+
+
+def test_nvfp4_zero_tensor(cuda_lib):
+    fq = cuda_lib
+    x = torch.zeros((32, 32), dtype=torch.bfloat16, device="cuda")
+    out = fq.rht16_quantize_sr(x, rowwise=True, colwise=True, rht=3, sr=3, rht_seed=1, sr_seed=2)
+    assert int(host(out["q_row"]).max()) == 0 and int(host(out["sf_row"]).max()) == 0
+    assert host(out["g_row"])[0] == 1.0 and host(out["g_col"])[0] == 1.0
+
+
+# ----------------------------------------------------------------------------- full size, sampled
+def _bands(n, size, rng, k=3):
+    starts = sorted({0, (n // size - 1) * size, int(rng.integers(0, n // size)) * size})
+    return np.concatenate([np.arange(s, s + size) for s in starts[:k]])
+
+
+def test_llama8b_fused_1x128_sampled(cuda_lib):
+    """X 8192x4096 (fused rowwise + transposed colwise, the bench's launch) and dY."""
+    fq = cuda_lib
+    d = workloads.llama8b()
+    rng = np.random.default_rng(2)
+    for name in ("X", "dY"):
+        x = d[name]
+        out = fq.quantize_1x128(x.cuda(), rowwise=True, colwise=True)
+        bits = workloads.bf16_bits(x)
+        rows = _bands(bits.shape[0], 128, rng)
+        q, s = Q.quantize_1x128_rowwise(bits[rows])
+        assert np.array_equal(host(out["q_row"][torch.from_numpy(rows).cuda()]), q)
+        assert np.array_equal(f32bits(host(out["s_row"])[:, rows]), f32bits(s))
+        cols = _bands(bits.shape[1], 128, rng)
+        qc, sc = Q.quantize_1x128_colwise(bits[:, cols])
+        assert np.array_equal(host(out["q_col"][torch.from_numpy(cols).cuda()]), qc)
+        assert np.array_equal(f32bits(host(out["s_col"])[:, cols]), f32bits(sc))
+        del out
+    w = d["W"]
+    out = fq.quantize_128x128(w.cuda())
+    bits = workloads.bf16_bits(w)
+    cols = _bands(bits.shape[1], 128, rng)
+    q, qt, s = Q.quantize_128x128(bits[:, cols])
+    assert np.array_equal(host(out["q"])[:, cols], q)
+    assert np.array_equal(host(out["q_t"][torch.from_numpy(cols).cuda()]), qt)
+    assert np.array_equal(f32bits(host(out["s"])[cols[::128] // 128]), f32bits(s))
+
+
+def test_mxfp8_fullsize_sampled(cuda_lib):
+    fq = cuda_lib
+    d = workloads.mxfp8(which=[2])
+    rng = np.random.default_rng(3)
+    a, w = d["A2"], d["W2"]                           # A 8192x14336, W 14336x4096
+    out = fq.quantize_mx32(a.cuda(), rowwise=True, sf_layout=1)
+    bits = workloads.bf16_bits(a)
+    rows = _bands(bits.shape[0], 128, rng)
+    q, e = Q.quantize_mx_rowwise(bits[rows])
+    assert np.array_equal(host(out["q_row"][torch.from_numpy(rows).cuda()]), q)
+    tiled = host(out["e8m0_row"])
+    ncols = bits.shape[1] // 32
+    rr, cc = np.meshgrid(rows, np.arange(ncols), indexing="ij")
+    assert np.array_equal(tiled[Q.sf_tiled_offset(rr, cc, ncols)], e)
+    out = fq.quantize_mx32(w.cuda(), rowwise=False, colwise=True, sf_layout=1)
+    bits = workloads.bf16_bits(w)
+    cols = _bands(bits.shape[1], 128, rng)
+    q, e = Q.quantize_mx_colwise(bits[:, cols])
+    assert np.array_equal(host(out["q_col"][torch.from_numpy(cols).cuda()]), q)
+    tiled = host(out["e8m0_col"])
+    nsf = bits.shape[0] // 32
+    rr, cc = np.meshgrid(cols, np.arange(nsf), indexing="ij")
+    assert np.array_equal(tiled[Q.sf_tiled_offset(rr, cc, nsf)], e)
+
+
+def test_nvfp4_gradient_fullsize_sampled(cuda_lib):
+    """dY 8192x53248: rowwise SR (dgrad A) and colwise RHT + SR (wgrad B) in one call."""
+    fq = cuda_lib
+    d = workloads.nvfp4(which=("dY",), device="cuda")
+    x = d["dY"]
+    out = fq.rht16_quantize_sr(x, rowwise=True, colwise=True, rht=2, rht_seed=5, sr=3, sr_seed=6, sf_layout=1)
+    bits = workloads.bf16_bits(x)
+    rng = np.random.default_rng(5)
+    rows = _bands(bits.shape[0], 128, rng, k=2)
+    q, sf, g = Q.quantize_nvfp4_rowwise(bits, sr=True, sr_seed=6, rows=rows)
+    assert np.array_equal(host(out["q_row"][torch.from_numpy(rows).cuda()]), q)
+    assert f32bits(host(out["g_row"]))[0] == f32bits(np.float32([g]))[0]
+    tiled = host(out["sf_row"])
+    nsf = bits.shape[1] // 16
+    rr, cc = np.meshgrid(rows, np.arange(nsf), indexing="ij")
+    assert np.array_equal(tiled[Q.sf_tiled_offset(rr, cc, nsf)], sf)
+    cols = _bands(bits.shape[1], 128, rng, k=2)
+    q, sf, g = Q.quantize_nvfp4_colwise(bits, rht=True, rht_seed=5, sr=True, sr_seed=6, rows=cols)
+    assert np.array_equal(host(out["q_col"][torch.from_numpy(cols).cuda()]), q)
+    assert f32bits(host(out["g_col"]))[0] == f32bits(np.float32([g]))[0]
+    tiled = host(out["sf_col"])
+    nsf = bits.shape[0] // 16
+    rr, cc = np.meshgrid(cols, np.arange(nsf), indexing="ij")
+    assert np.array_equal(tiled[Q.sf_tiled_offset(rr, cc, nsf)], sf)
