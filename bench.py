@@ -1,0 +1,717 @@
+"""Benchmark of the hot path: online fine-grained quantization + block-scaled GEMM on B200.
+
+Default workload (one "step"), Llama-3-8B up-projection, blockwise recipe, forward and
+backward with M = 8192 tokens, hidden K = 4096, FFN N = 14336:
+  quantize X (1x128 rowwise + fused transposed colwise), quantize W (128x128, both
+  layouts), quantize dY (1x128 rowwise + colwise), GEMM fprop, dgrad, wgrad.
+Other workloads (--workload): tiny, mxfp8, moe, nvfp4 (one JSON line each).
+
+Metric: block-scaled GEMM TFLOP/s (the step's GEMM FLOPs over the whole step's device time,
+quantization included) with per-kernel TFLOP/s and GB/s as fractions of the roofline.
+
+Contract: python bench.py --gpus N --steps K --warmup W [--impl ours|reference]
+  * N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs the step on
+    its own tokens (weak scaling, no data-path collective); timing is the max over ranks.
+  * Inputs live in HBM before the timed region; the L2 is flushed (256 MiB write) between
+    steps, outside the per-step events.
+  * --impl reference times the CPU oracle (rank 0 only) on a bounded sample of the step.
+"""
+import argparse
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+import torch
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+import workloads  # noqa: E402
+
+METRIC = "block-scaled FP8 GEMM TFLOPS & quantize GB/s on 1 B200, % of roofline"
+FALLBACK_PEAKS = {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0}
+FP8_PER_BF16 = 2.0   # nominal dense FP8 : BF16 tensor throughput ratio on B200
+FP4_PER_BF16 = 4.0   # nominal dense FP4 : BF16
+
+
+def load_peaks():
+    p = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    if os.path.exists(p):
+        with open(p) as f:
+            d = json.load(f)
+        return d, "measured"
+    return dict(FALLBACK_PEAKS), "fallback"
+
+
+# ============================================================================ steps
+class Launch:
+    """One kernel launch in a step: `fn()` enqueues it on the current stream."""
+
+    def __init__(self, name, fn, kernel, flop=0.0, bytes_=0.0):
+        self.name, self.fn, self.kernel, self.flop, self.bytes = name, fn, kernel, flop, bytes_
+
+
+def b_1x128_fused(r, c):
+    return r * c * (2 + 1 + 1) + 2 * r * c / 128 * 4
+
+
+def b_1x128_row(r, c):
+    return r * c * (2 + 1) + r * c / 128 * 4
+
+
+def b_128(k, n):
+    return k * n * (2 + 1 + 1) + (k // 128) * (n // 128) * 4
+
+
+def b_mx(r, c):
+    return r * c * (2 + 1) + r * c / 32
+
+
+class LlamaStep:
+    name = "llama8b"
+    workload = "llama3-8b up-proj blockwise fwd+bwd: X 8192x4096, W 4096x14336, dY 8192x14336"
+
+    def __init__(self, fq, rank, M=8192, K=4096, N=14336):
+        self.fq, self.M, self.K, self.N = fq, M, K, N
+        d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
+        if rank:   # other ranks: their own tokens, the same weights
+            g = workloads.llama8b(device="cuda", M=M, K=K, N=N)
+            d["X"] = workloads.normal_bf16((M, K), 1.0, 10_000 + rank, 1e-3, 50.0, "cuda")
+            d["dY"] = workloads.normal_bf16((M, N), 1e-3, 20_000 + rank, device="cuda")
+            del g
+        self.X, self.W, self.dY = d["X"], d["W"], d["dY"]
+        dev = self.X.device
+        u8, f32 = torch.uint8, torch.float32
+        self.qx_r, self.qx_c = torch.empty((M, K), dtype=u8, device=dev), torch.empty((K, M), dtype=u8, device=dev)
+        self.sx_r, self.sx_c = torch.empty((K // 128, M), dtype=f32, device=dev), torch.empty((M // 128, K), dtype=f32, device=dev)
+        self.qw_t, self.qw = torch.empty((N, K), dtype=u8, device=dev), torch.empty((K, N), dtype=u8, device=dev)
+        self.sw = torch.empty((N // 128, K // 128), dtype=f32, device=dev)
+        self.qd_r, self.qd_c = torch.empty((M, N), dtype=u8, device=dev), torch.empty((N, M), dtype=u8, device=dev)
+        self.sd_r, self.sd_c = torch.empty((N // 128, M), dtype=f32, device=dev), torch.empty((M // 128, N), dtype=f32, device=dev)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty((K, N), dtype=torch.bfloat16, device=dev)
+        self.gemm_flop = 3 * 2.0 * M * N * K
+
+    def inputs(self):
+        return [self.X, self.W, self.dY]
+
+    def outputs(self):
+        return [self.Y, self.dX, self.dW]
+
+    def launches(self):
+        fq, M, K, N = self.fq, self.M, self.K, self.N
+        P = lambda t: t.data_ptr()  # noqa: E731
+
+        def q1x128(x, qr, sr, qc, sc, R, C):
+            def f():
+                st = fq.fp8q_quantize_1x128(P(x), R, C, C, P(qr), P(sr), sr.shape[1], P(qc), P(sc), sc.shape[1],
+                                            fq._stream())
+                assert st == 0, st
+            return f
+
+        def q128():
+            st = fq.fp8q_quantize_128x128(P(self.W), K, N, N, P(self.qw_t), P(self.qw), P(self.sw), fq._stream())
+            assert st == 0, st
+
+        def gemm(a, b, layout, sa, sb, ld_sb, c):
+            def f():
+                fq.gemm(a, b, fq.FP8Q_BLOCKWISE, layout, a_scale=sa, b_scale=sb, ld_sb=ld_sb, out=c)
+            return f
+
+        return [
+            Launch("quantize_1x128 X (row+col)", q1x128(self.X, self.qx_r, self.sx_r, self.qx_c, self.sx_c, M, K),
+                   "quantize", bytes_=b_1x128_fused(M, K)),
+            Launch("quantize_128x128 W (both layouts)", q128, "quantize", bytes_=b_128(K, N)),
+            Launch("quantize_1x128 dY (row+col)", q1x128(self.dY, self.qd_r, self.sd_r, self.qd_c, self.sd_c, M, N),
+                   "quantize", bytes_=b_1x128_fused(M, N)),
+            Launch("gemm blockwise fprop", gemm(self.qx_r, self.qw_t, fq.FP8Q_FPROP, self.sx_r, self.sw, K // 128, self.Y),
+                   "gemm_blockwise", flop=2.0 * M * N * K),
+            Launch("gemm blockwise dgrad", gemm(self.qd_r, self.qw, fq.FP8Q_DGRAD, self.sd_r, self.sw, K // 128, self.dX),
+                   "gemm_blockwise", flop=2.0 * M * N * K),
+            Launch("gemm blockwise wgrad", gemm(self.qx_c, self.qd_c, fq.FP8Q_WGRAD, self.sx_c, self.sd_c, N, self.dW),
+                   "gemm_blockwise", flop=2.0 * M * N * K),
+        ]
+
+    def cpu_sample(self, tiles=1):
+        """Oracle on a bounded sample: the operands of `tiles` output tiles of each GEMM
+        are quantized by the oracle from the BF16 inputs, then the FP64 reference tiles."""
+        from oracle import gemm as G
+        from oracle import quant as Q
+        M, K, N = self.M, self.K, self.N
+        Xb, Wb, dYb = (workloads.bf16_bits(t) for t in (self.X, self.W, self.dY))
+        t0 = time.perf_counter()
+        flop = 0.0
+        for m0, n0 in G.sample_tiles(M, N, tiles, seed=2):
+            oa, sa = Q.quantize_1x128_rowwise(Xb[m0:m0 + 128])
+            _, owt, sw = Q.quantize_128x128(Wb[:, n0:n0 + 128])
+            G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+            flop += 2.0 * 128 * 128 * K
+        for m0, n0 in G.sample_tiles(M, K, tiles, seed=3):
+            oa, sa = Q.quantize_1x128_rowwise(dYb[m0:m0 + 128])
+            ow, _, sw = Q.quantize_128x128(Wb[n0:n0 + 128])
+            G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ow, sw, G.DGRAD))
+            flop += 2.0 * 128 * 128 * N
+        for m0, n0 in G.sample_tiles(K, N, tiles, seed=4):
+            oa, sa = Q.quantize_1x128_colwise(Xb[:, m0:m0 + 128])
+            ob, sb = Q.quantize_1x128_colwise(dYb[:, n0:n0 + 128])
+            G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
+            flop += 2.0 * 128 * 128 * M
+        dt = time.perf_counter() - t0
+        return flop, dt, (f"{tiles} sampled 128x128 output tile(s) of each of fprop/dgrad/wgrad, operands "
+                          "quantized by the oracle from the BF16 inputs, FP64 reference product")
+
+
+class TinyStep(LlamaStep):
+    name = "tiny"
+    workload = "tiny blockwise fprop: A 256x512, B 512x256"
+
+    def __init__(self, fq, rank):
+        self.fq = fq
+        d = workloads.tiny(device="cuda")
+        self.A, self.B = d["A"], d["B"]
+        dev = self.A.device
+        self.qa = torch.empty((256, 512), dtype=torch.uint8, device=dev)
+        self.sa = torch.empty((4, 256), dtype=torch.float32, device=dev)
+        self.qbt = torch.empty((256, 512), dtype=torch.uint8, device=dev)
+        self.sb = torch.empty((2, 4), dtype=torch.float32, device=dev)
+        self.C = torch.empty((256, 256), dtype=torch.bfloat16, device=dev)
+        self.gemm_flop = 2.0 * 256 * 256 * 512
+
+    def inputs(self):
+        return [self.A, self.B]
+
+    def outputs(self):
+        return [self.C]
+
+    def launches(self):
+        fq = self.fq
+        P = lambda t: t.data_ptr()  # noqa: E731
+
+        def qa():
+            assert fq.fp8q_quantize_1x128(P(self.A), 256, 512, 512, P(self.qa), P(self.sa), 256, None, None, 0,
+                                          fq._stream()) == 0
+
+        def qb():
+            assert fq.fp8q_quantize_128x128(P(self.B), 512, 256, 256, P(self.qbt), None, P(self.sb), fq._stream()) == 0
+
+        def g():
+            fq.gemm(self.qa, self.qbt, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=self.sa, b_scale=self.sb, out=self.C)
+
+        return [Launch("quantize_1x128 A", qa, "quantize", bytes_=b_1x128_row(256, 512)),
+                Launch("quantize_128x128 B", qb, "quantize", bytes_=256 * 512 * 3.0),
+                Launch("gemm blockwise fprop", g, "gemm_blockwise", flop=self.gemm_flop)]
+
+    def cpu_sample(self, tiles=1):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        t0 = time.perf_counter()
+        oa, sa = Q.quantize_1x128_rowwise(workloads.bf16_bits(self.A))
+        _, owt, sw = Q.quantize_128x128(workloads.bf16_bits(self.B))
+        G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+        return self.gemm_flop, time.perf_counter() - t0, "the whole tiny step"
+
+
+class MxStep:
+    name = "mxfp8"
+    workload = "MXFP8 (and per-tensor) GEMMs (M,K,N) = (8192,4096,4096), (8192,4096,14336), (8192,14336,4096)"
+
+    def __init__(self, fq, rank):
+        self.fq = fq
+        d = workloads.mxfp8(device="cuda")
+        self.items = []
+        for i, (M, K, N) in enumerate(workloads.MXFP8_GEMMS):
+            A, W = d[f"A{i}"], d[f"W{i}"]
+            dev = A.device
+            it = {"M": M, "K": K, "N": N, "A": A, "W": W, "Wt": W.t().contiguous(),
+                  "qa": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                  "ea": torch.empty(fq.fp8q_sf_bytes(fq.FP8Q_MXFP8, M, K, 1), dtype=torch.uint8, device=dev),
+                  "qb": torch.empty((N, K), dtype=torch.uint8, device=dev),
+                  "eb": torch.empty(fq.fp8q_sf_bytes(fq.FP8Q_MXFP8, N, K, 1), dtype=torch.uint8, device=dev),
+                  "ta": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                  "tb": torch.empty((N, K), dtype=torch.uint8, device=dev),
+                  "sa": torch.empty((1,), dtype=torch.float32, device=dev),
+                  "sb": torch.empty((1,), dtype=torch.float32, device=dev),
+                  "C": torch.empty((M, N), dtype=torch.bfloat16, device=dev),
+                  "C2": torch.empty((M, N), dtype=torch.bfloat16, device=dev)}
+            self.items.append(it)
+        self.gemm_flop = sum(2.0 * 2 * it["M"] * it["N"] * it["K"] for it in self.items)
+
+    def inputs(self):
+        return [t for it in self.items for t in (it["A"], it["W"])]
+
+    def outputs(self):
+        return [t for it in self.items for t in (it["C"], it["C2"])]
+
+    def launches(self):
+        fq = self.fq
+        P = lambda t: t.data_ptr()  # noqa: E731
+        out = []
+        for i, it in enumerate(self.items):
+            M, K, N = it["M"], it["K"], it["N"]
+
+            def qa(it=it, M=M, K=K):
+                assert fq.fp8q_quantize_mx32(P(it["A"]), M, K, K, P(it["qa"]), P(it["ea"]), None, None, 1,
+                                             fq._stream()) == 0
+
+            def qb(it=it, K=K, N=N):
+                assert fq.fp8q_quantize_mx32(P(it["W"]), K, N, N, None, None, P(it["qb"]), P(it["eb"]), 1,
+                                             fq._stream()) == 0
+
+            def g(it=it):
+                fq.gemm(it["qa"], it["qb"], fq.FP8Q_MXFP8, a_scale=it["ea"], b_scale=it["eb"], out=it["C"])
+
+            def ta(it=it, M=M, K=K):
+                assert fq.fp8q_quantize_tensor(P(it["A"]), M, K, K, P(it["ta"]), P(it["sa"]), fq._stream()) == 0
+
+            def tb(it=it, K=K, N=N):
+                assert fq.fp8q_quantize_tensor(P(it["Wt"]), N, K, K, P(it["tb"]), P(it["sb"]), fq._stream()) == 0
+
+            def g2(it=it):
+                fq.gemm(it["ta"], it["tb"], fq.FP8Q_PERTENSOR, a_global=it["sa"], b_global=it["sb"], out=it["C2"])
+
+            out += [Launch(f"quantize_mx32 A{i} rowwise", qa, "quantize", bytes_=b_mx(M, K)),
+                    Launch(f"quantize_mx32 W{i} colwise", qb, "quantize", bytes_=b_mx(K, N)),
+                    Launch(f"gemm mxfp8 {M}x{K}x{N}", g, "gemm_mxfp8", flop=2.0 * M * N * K),
+                    Launch(f"quantize_tensor A{i}", ta, "quantize", bytes_=5.0 * M * K),
+                    Launch(f"quantize_tensor W{i}^T", tb, "quantize", bytes_=5.0 * K * N),
+                    Launch(f"gemm per-tensor {M}x{K}x{N}", g2, "gemm_pertensor", flop=2.0 * M * N * K)]
+        return out
+
+    def cpu_sample(self, tiles=1):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        t0 = time.perf_counter()
+        flop = 0.0
+        for i, it in enumerate(self.items):
+            Ab, Wb = workloads.bf16_bits(it["A"]), workloads.bf16_bits(it["W"])
+            for m0, n0 in G.sample_tiles(it["M"], it["N"], tiles, seed=10 + i):
+                oa, ea = Q.quantize_mx_rowwise(Ab[m0:m0 + 128])
+                ob, eb = Q.quantize_mx_colwise(Wb[:, n0:n0 + 128])
+                G.reference(G.dequant_mx(oa, ea), G.dequant_mx(ob, eb))
+                flop += 2.0 * 128 * 128 * it["K"]
+        return flop, time.perf_counter() - t0, f"{tiles} sampled MXFP8 output tile(s) per GEMM, oracle-quantized"
+
+
+class MoeStep:
+    name = "moe"
+    workload = "DeepSeek-V3 MoE grouped blockwise fprop: 32 experts, 16384 tokens x top-8, up 7168->2048, down 2048->7168"
+
+    def __init__(self, fq, rank):
+        self.fq = fq
+        self.parts = []
+        for proj in ("up", "down"):
+            d = workloads.moe(device="cuda", proj=proj)
+            A, W, offs = d["A"], d["W"], d["offsets"].cuda()
+            Gn, K, N = W.shape
+            M = A.shape[0]
+            dev = A.device
+            self.parts.append({"proj": proj, "A": A, "W": W, "offs": offs, "G": Gn, "K": K, "N": N, "M": M,
+                               "qa": torch.empty((M, K), dtype=torch.uint8, device=dev),
+                               "sa": torch.empty((K // 128, M), dtype=torch.float32, device=dev),
+                               "B": torch.empty((Gn, N, K), dtype=torch.uint8, device=dev),
+                               "SB": torch.empty((Gn, N // 128, K // 128), dtype=torch.float32, device=dev),
+                               "C": torch.empty((M, N), dtype=torch.bfloat16, device=dev)})
+        self.gemm_flop = sum(2.0 * p["M"] * p["N"] * p["K"] for p in self.parts)
+
+    def inputs(self):
+        return [t for p in self.parts for t in (p["A"], p["W"])]
+
+    def outputs(self):
+        return [p["C"] for p in self.parts]
+
+    def launches(self):
+        fq = self.fq
+        P = lambda t: t.data_ptr()  # noqa: E731
+        out = []
+        for p in self.parts:
+            M, K, N, Gn = p["M"], p["K"], p["N"], p["G"]
+
+            def qa(p=p, M=M, K=K):
+                assert fq.fp8q_quantize_1x128(P(p["A"]), M, K, K, P(p["qa"]), P(p["sa"]), M, None, None, 0,
+                                              fq._stream()) == 0
+
+            def qw(p=p, K=K, N=N, Gn=Gn):
+                for g in range(Gn):
+                    assert fq.fp8q_quantize_128x128(P(p["W"][g]), K, N, N, P(p["B"][g]), None, P(p["SB"][g]),
+                                                    fq._stream()) == 0
+
+            def g_(p=p, K=K):
+                fq.gemm(p["qa"], p["B"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=p["sa"], b_scale=p["SB"],
+                        ld_sb=K // 128, m_offsets=p["offs"], out=p["C"])
+
+            out += [Launch(f"quantize_1x128 A_{p['proj']}", qa, "quantize", bytes_=b_1x128_row(M, K)),
+                    Launch(f"quantize_128x128 W_{p['proj']} x{Gn}", qw, "quantize",
+                           bytes_=Gn * (K * N * 3.0 + (K // 128) * (N // 128) * 4)),
+                    Launch(f"gemm grouped blockwise {p['proj']}", g_, "gemm_grouped", flop=2.0 * M * N * K)]
+        return out
+
+    def launch_count(self):
+        return sum(2 + p["G"] for p in self.parts)
+
+    def cpu_sample(self, tiles=1):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        t0 = time.perf_counter()
+        flop = 0.0
+        for p in self.parts:
+            Ab = workloads.bf16_bits(p["A"])
+            for g, m0, m1, n0 in G.sample_group_tiles(p["offs"].cpu().numpy(), p["N"], tiles, seed=4):
+                oa, sa = Q.quantize_1x128_rowwise(Ab[m0:m1])
+                _, owt, sw = Q.quantize_128x128(workloads.bf16_bits(p["W"][g][:, n0:n0 + 128]))
+                G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+                flop += 2.0 * (m1 - m0) * 128 * p["K"]
+        return flop, time.perf_counter() - t0, f"{tiles} sampled grouped output tile(s) per projection"
+
+
+class Nvfp4Step:
+    name = "nvfp4"
+    workload = "NVFP4 Llama-3.1-405B shapes: dgrad (8192,53248,16384), wgrad (16384,8192,53248)"
+
+    def __init__(self, fq, rank, M=8192, H=16384, F=53248):
+        self.fq, self.M, self.H, self.F = fq, M, H, F
+        d = workloads.nvfp4(device="cuda", M=M, H=H, F=F)
+        self.X, self.W, self.dY = d["X"], d["W"], d["dY"]
+        dev = self.X.device
+        u8 = torch.uint8
+        sfb = lambda o, i: torch.empty(fq.fp8q_sf_bytes(fq.FP8Q_NVFP4, o, i, 1), dtype=u8, device=dev)  # noqa: E731
+        self.qd_r, self.sd_r = torch.empty((M, F // 2), dtype=u8, device=dev), sfb(M, F)
+        self.qd_c, self.sd_c = torch.empty((F, M // 2), dtype=u8, device=dev), sfb(F, M)
+        self.qw, self.sw = torch.empty((H, F // 2), dtype=u8, device=dev), sfb(H, F)
+        self.qx_c, self.sx_c = torch.empty((H, M // 2), dtype=u8, device=dev), sfb(H, M)
+        self.g = torch.empty((4,), dtype=torch.float32, device=dev)
+        self.dX = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty((H, F), dtype=torch.bfloat16, device=dev)
+        self.gemm_flop = 2 * 2.0 * M * H * F
+
+    def inputs(self):
+        return [self.X, self.W, self.dY]
+
+    def outputs(self):
+        return [self.dX, self.dW]
+
+    def launches(self):
+        fq, M, H, F = self.fq, self.M, self.H, self.F
+        P = lambda t: t.data_ptr()  # noqa: E731
+        g = self.g
+
+        def qd():
+            assert fq.fp4q_rht16_quantize_sr(P(self.dY), M, F, F, fq.FP4Q_COL, 5, fq.FP4Q_ROW | fq.FP4Q_COL, 6,
+                                             P(self.qd_r), P(self.sd_r), P(g[0:1]), P(self.qd_c), P(self.sd_c),
+                                             P(g[1:2]), 1, fq._stream()) == 0
+
+        def qw():
+            assert fq.fp4q_rht16_quantize_sr(P(self.W), H, F, F, 0, 5, 0, 6, P(self.qw), P(self.sw), P(g[2:3]),
+                                             None, None, None, 1, fq._stream()) == 0
+
+        def qx():
+            assert fq.fp4q_rht16_quantize_sr(P(self.X), M, H, H, fq.FP4Q_COL, 5, 0, 6, None, None, None,
+                                             P(self.qx_c), P(self.sx_c), P(g[3:4]), 1, fq._stream()) == 0
+
+        def dgrad():
+            fq.gemm(self.qd_r, self.qw, fq.FP8Q_NVFP4, a_scale=self.sd_r, b_scale=self.sw, a_global=g[0:1],
+                    b_global=g[2:3], K=F, out=self.dX)
+
+        def wgrad():
+            fq.gemm(self.qx_c, self.qd_c, fq.FP8Q_NVFP4, a_scale=self.sx_c, b_scale=self.sd_c, a_global=g[3:4],
+                    b_global=g[1:2], K=M, out=self.dW)
+
+        nv2 = lambda r, c: r * c * 4.0 + 2 * r * c * (0.5 + 1 / 16)  # noqa: E731  two outputs
+        nv1 = lambda r, c: r * c * 4.0 + r * c * (0.5 + 1 / 16)      # noqa: E731  one output
+        return [Launch("fp4q quantize dY (row SR + col RHT SR)", qd, "quantize_nvfp4", bytes_=nv2(M, F)),
+                Launch("fp4q quantize W (row RNE)", qw, "quantize_nvfp4", bytes_=nv1(H, F)),
+                Launch("fp4q quantize X (col RHT RNE)", qx, "quantize_nvfp4", bytes_=nv1(M, H)),
+                Launch("gemm nvfp4 dgrad", dgrad, "gemm_nvfp4", flop=2.0 * M * H * F),
+                Launch("gemm nvfp4 wgrad", wgrad, "gemm_nvfp4", flop=2.0 * M * H * F)]
+
+    def cpu_sample(self, tiles=1):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        t0 = time.perf_counter()
+        dYb = workloads.bf16_bits(self.dY[:1024])
+        Wb = workloads.bf16_bits(self.W[:1024])
+        # global amax over the sampled slabs stands in for the full tensors' (sample timing only)
+        oa, sa, ga = Q.quantize_nvfp4_rowwise(dYb, sr=True, sr_seed=6, rows=list(range(128)))
+        ob, sb, gb = Q.quantize_nvfp4_rowwise(Wb, rows=list(range(128)))
+        G.reference(G.dequant_nvfp4(oa, sa, ga), G.dequant_nvfp4(ob, sb, gb))
+        flop = 2.0 * 128 * 128 * self.F
+        return flop, time.perf_counter() - t0, "1 dgrad output tile; amax over 1024-row slabs"
+
+
+STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step}
+
+
+# ============================================================================ measurement
+class ClockSampler:
+    """nvidia-smi samples of SM clock and throttle reasons while the timed region runs."""
+
+    Q = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.hw_slowdown,"
+         "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+         "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def start(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.Q}",
+                                          "--format=csv,noheader,nounits", "-lms", "50"],
+                                         stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"], "samples": 0}
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except subprocess.TimeoutExpired:
+            self.proc.kill()
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) == 7:
+                    try:
+                        rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                    except ValueError:
+                        pass
+        os.unlink(self.path)
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": reasons, "samples": 0}
+        return {"sm_mhz": statistics.median(r[0] for r in rows), "sm_max_mhz": max(r[1] for r in rows),
+                "reasons": reasons, "samples": len(rows)}
+
+
+def run_ours(args, rank, world, local_rank):
+    import fp4_precision_gemm_b200 as fq
+    torch.cuda.set_device(local_rank)
+    fq.lib()
+    step = STEPS[args.workload](fq, rank)
+    launches = step.launches()
+    n_launch = getattr(step, "launch_count", lambda: len(launches))()
+    flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    stream = torch.cuda.current_stream()
+
+    def barrier():
+        if world > 1:
+            torch.distributed.barrier()
+
+    for _ in range(args.warmup):
+        for L in launches:
+            L.fn()
+    torch.cuda.synchronize()
+    assert fq.device_status() == 0
+    ev = [[(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in launches]
+          for _ in range(args.steps)]
+    barrier()
+    torch.cuda.synchronize()
+    sampler = ClockSampler(local_rank)
+    sampler.start()
+    time.sleep(0.15)
+    t_wall = time.perf_counter()
+    for k in range(args.steps):
+        flush.fill_(k & 0xFF)                     # L2 flush (256 MiB write), outside the events
+        for L, (a, b) in zip(launches, ev[k]):
+            a.record(stream)
+            L.fn()
+            b.record(stream)
+    torch.cuda.synchronize()
+    t_wall = time.perf_counter() - t_wall
+    clocks = sampler.stop()
+    barrier()
+    per = [[a.elapsed_time(b) for (a, b) in row] for row in ev]          # ms
+    step_ms = [ev[k][0][0].elapsed_time(ev[k][-1][1]) for k in range(args.steps)]
+    ms = sum(step_ms) / len(step_ms)
+    if world > 1:
+        t = torch.tensor([ms], device="cuda")
+        torch.distributed.all_reduce(t, op=torch.distributed.ReduceOp.MAX)
+        ms = float(t.item())
+    status = fq.device_status()
+
+    # per-kernel statistics (mean over the timed steps)
+    peaks, src = load_peaks()
+    fp8_peak = peaks["bf16_tflops"] * FP8_PER_BF16
+    fp4_peak = peaks["bf16_tflops"] * FP4_PER_BF16
+    kern = []
+    for i, L in enumerate(launches):
+        t_ms = statistics.mean(r[i] for r in per)
+        d = {"name": L.name, "kernel": L.kernel, "ms": round(t_ms, 4)}
+        if L.flop:
+            tf = L.flop / (t_ms * 1e-3) / 1e12
+            peak = fp4_peak if "nvfp4" in L.kernel else fp8_peak
+            d.update({"tflops": round(tf, 1), "frac": round(tf / peak, 3)})
+        if L.bytes:
+            gbs = L.bytes / (t_ms * 1e-3) / 1e9
+            d.update({"gbs": round(gbs, 1), "frac": round(gbs / peaks["hbm_gbs"], 3)})
+        kern.append(d)
+    # dominant kernel: the GEMM family with the largest share of the step
+    fam = {}
+    for d, L in zip(kern, launches):
+        f = fam.setdefault(L.kernel, {"ms": 0.0, "flop": 0.0, "bytes": 0.0})
+        f["ms"] += d["ms"]
+        f["flop"] += L.flop
+        f["bytes"] += L.bytes
+    dom = max(fam, key=lambda k: fam[k]["ms"])
+    f = fam[dom]
+    if f["flop"]:
+        peak = fp4_peak if "nvfp4" in dom else fp8_peak
+        ach = f["flop"] / (f["ms"] * 1e-3) / 1e12
+        roof = {"kernel": dom, "bound": "tensor", "achieved": round(ach, 1), "peak": round(peak, 1),
+                "unit": "TFLOP/s", "frac": round(ach / peak, 3), "traffic": None,
+                "peak_source": f"{src}: bf16_tflops x {FP4_PER_BF16 if 'nvfp4' in dom else FP8_PER_BF16:g} "
+                               "(nominal dense ratio), burst figure"}
+    else:
+        ach = f["bytes"] / (f["ms"] * 1e-3) / 1e9
+        roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
+                "frac": round(ach / peaks["hbm_gbs"], 3), "traffic": None, "peak_source": f"{src}: hbm_gbs"}
+    roof["traffic"] = traffic_for(dom, args.workload)
+
+    e2e = measure_e2e(step, launches, stream, args) if (not args.no_e2e) else None
+    value = world * step.gemm_flop / (ms * 1e-3) / 1e12
+    out = {
+        "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "fp8_e4m3" if args.workload != "nvfp4" else "fp4_e2m1",
+        "data": "synthetic (seeded normal BF16 with outliers; see workloads.py)",
+        "config": {"workload": step.workload, "l2": "flushed between steps (256 MiB write)",
+                   "gemm_tflop_per_step": round(step.gemm_flop / 1e12, 4),
+                   "parallelism": f"dp{world} (independent replicas, no collective)"},
+        "roofline": roof, "kernels": kern, "gpu_launches": n_launch * args.steps,
+        "clocks": clocks, "e2e": e2e, "device_status": status, "wall_s_timed_region": round(t_wall, 3),
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        out["cpu_baseline"] = cpu_baseline(step)
+    return out
+
+
+TRAFFIC_FILE = os.path.join(ROOT, "profiles", "traffic.json")
+
+
+def traffic_for(kernel, workload):
+    """DRAM bytes per launch from the committed ncu summary, when one exists for this kernel
+    and workload (null otherwise)."""
+    try:
+        with open(TRAFFIC_FILE) as f:
+            d = json.load(f)
+        return d.get(workload, {}).get(kernel)
+    except (OSError, ValueError):
+        return None
+
+
+def measure_e2e(step, launches, stream, args):
+    """Same step through the C ABI with the inputs in pinned HOST memory: H2D copies, the
+    kernels, D2H copies of the results, all inside the timed region."""
+    ins = step.inputs()
+    outs = step.outputs()
+    h_in = [t.cpu().pin_memory() for t in ins]
+    h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs]
+    bi = sum(t.numel() * t.element_size() for t in ins)
+    bo = sum(t.numel() * t.element_size() for t in outs)
+    reps = max(2, min(args.steps, 5))
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        for d, h in zip(ins, h_in):
+            d.copy_(h, non_blocking=True)
+        for L in launches:
+            L.fn()
+        for d, h in zip(outs, h_out):
+            h.copy_(d, non_blocking=True)
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    return {"value": round(step.gemm_flop / (ms * 1e-3) / 1e12, 2), "unit": "TFLOP/s",
+            "ms_per_step": round(ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
+
+
+def cpu_baseline(step):
+    threads = torch.get_num_threads()
+    try:
+        import numpy as np  # noqa: F401
+        from threadpoolctl import threadpool_info
+        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        blas = threads
+    flop, dt, what = step.cpu_sample()
+    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": int(blas), "kind": "oracle",
+            "sample": what, "seconds": round(dt, 2)}
+
+
+def run_reference(args, rank, world):
+    """The CPU oracle as it stands, timed on the host cores on a bounded sample per step."""
+    if rank != 0:
+        return None
+    torch.cuda.set_device(0) if torch.cuda.is_available() else None
+    import fp4_precision_gemm_b200 as fq
+    step = STEPS[args.workload](fq, 0) if torch.cuda.is_available() else None
+    if step is None:
+        return {"impl": "reference", "unavailable": "the oracle's inputs are generated on a CUDA device"}
+    for _ in range(args.warmup):
+        step.cpu_sample()
+    flops, secs = 0.0, 0.0
+    what = ""
+    for _ in range(args.steps):
+        f, dt, what = step.cpu_sample()
+        flops += f
+        secs += dt
+    value = flops / secs / 1e12
+    cb = cpu_baseline(step)
+    return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
+            "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
+            "data": "synthetic (seeded normal BF16 with outliers; see workloads.py)",
+            "config": {"workload": step.workload, "sample": what},
+            "cpu_baseline": {"value": round(value, 6), "unit": "TFLOP/s", "cores": cb["cores"], "kind": "oracle",
+                             "sample": what},
+            "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=3)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", choices=sorted(STEPS) + ["all"], default="llama8b")
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    args.warmup = max(args.warmup, 3)
+
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1 and args.impl == "ours":
+        import datetime
+        torch.cuda.set_device(local_rank)
+        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                             device_id=torch.device("cuda", local_rank))
+    names = sorted(STEPS) if args.workload == "all" else [args.workload]
+    for name in names:
+        args.workload = name
+        if args.impl == "reference":
+            out = run_reference(args, rank, world)
+        else:
+            out = run_ours(args, rank, world, local_rank)
+        if rank == 0 and out is not None:
+            print(json.dumps(out), flush=True)
+    if world > 1 and args.impl == "ours":
+        torch.distributed.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

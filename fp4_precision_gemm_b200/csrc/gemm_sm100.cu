@@ -356,25 +356,34 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint32_t pb = chunk & 1;
           if (!mbar_wait(&pfull[pb], (chunk >> 1) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
           tc_fence_after();
+          // two 16-column TMEM loads in flight per wait
 #pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(t_lane + pb * kBN + c * 16, r);
-            tmem_ld_wait(r);
+          for (int c = 0; c < 8; c += 2) {
+            uint32_t r0[16], r1[16];
+            tmem_ld_32x32b_x16(t_lane + pb * kBN + c * 16, r0);
+            tmem_ld_32x32b_x16(t_lane + pb * kBN + c * 16 + 16, r1);
+            tmem_ld_wait(r0);
+            tmem_ld_wait(r1);
             if (kWg) {
               const float2 s2 = make_float2(sa, sa);
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float2 b2 = *reinterpret_cast<const float2*>(sbw + c * 16 + 2 * i);
-                const float2 pr = __fmul2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), b2);
-                acc[c * 8 + i] = __ffma2_rn(pr, s2, acc[c * 8 + i]);
+                const float2 b0 = *reinterpret_cast<const float2*>(sbw + c * 16 + 2 * i);
+                const float2 b1 = *reinterpret_cast<const float2*>(sbw + c * 16 + 16 + 2 * i);
+                const float2 p0 = __fmul2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])), b0);
+                const float2 p1 = __fmul2_rn(make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])), b1);
+                acc[c * 8 + i] = __ffma2_rn(p0, s2, acc[c * 8 + i]);
+                acc[c * 8 + 8 + i] = __ffma2_rn(p1, s2, acc[c * 8 + 8 + i]);
               }
             } else {
               const float2 s2 = make_float2(scale, scale);
 #pragma unroll
-              for (int i = 0; i < 8; ++i)
-                acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1])), s2,
+              for (int i = 0; i < 8; ++i) {
+                acc[c * 8 + i] = __ffma2_rn(make_float2(__uint_as_float(r0[2 * i]), __uint_as_float(r0[2 * i + 1])), s2,
                                             acc[c * 8 + i]);
+                acc[c * 8 + 8 + i] = __ffma2_rn(make_float2(__uint_as_float(r1[2 * i]), __uint_as_float(r1[2 * i + 1])),
+                                                s2, acc[c * 8 + 8 + i]);
+              }
             }
           }
           tc_fence_before();

@@ -291,9 +291,18 @@ __global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ 
       const uint2 a = *(const uint2*)&tq[c * 64 + (((2 * h) ^ ((c >> 2) & 7)) * 8)];
       const uint2 b = *(const uint2*)&tq[c * 64 + (((2 * h + 1) ^ ((c >> 2) & 7)) * 8)];
       uint8_t* dst = P.q_col + cg * (P.rows >> 1) + (rg >> 1);
+      // the transposed row stride is rows/2 bytes: 16-byte aligned only when rows % 32 == 0
       if (cg < P.cols) {
-        if (rg + 32 <= P.rows) *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
-        else if (rg + 16 <= P.rows) *(uint2*)dst = a;
+        if (rg + 32 <= P.rows) {
+          if (((P.rows >> 1) & 15) == 0) {
+            *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
+          } else {
+            *(uint2*)dst = a;
+            *(uint2*)(dst + 8) = b;
+          }
+        } else if (rg + 16 <= P.rows) {
+          *(uint2*)dst = a;
+        }
       }
     }
   }
