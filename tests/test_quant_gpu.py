@@ -144,10 +144,17 @@ def test_nvfp4_parity(cuda_lib, layout, R, C, row, col, rht, sr):
 
 
 def test_nvfp4_zero_tensor(cuda_lib):
+    """All-zero input: G = 0 -> S_g = 1, every block scale 0, every magnitude 0.  The
+    transform's sign flips turn some zeros into -0.0, whose code (0x8) the oracle gives too."""
     fq = cuda_lib
-    x = torch.zeros((32, 32), dtype=torch.bfloat16, device="cuda")
-    out = fq.rht16_quantize_sr(x, rowwise=True, colwise=True, rht=3, sr=3, rht_seed=1, sr_seed=2)
-    assert int(host(out["q_row"]).max()) == 0 and int(host(out["sf_row"]).max()) == 0
+    x = torch.zeros((32, 32), dtype=torch.bfloat16)
+    out = fq.rht16_quantize_sr(x.cuda(), rowwise=True, colwise=True, rht=3, sr=3, rht_seed=1, sr_seed=2)
+    bits = workloads.bf16_bits(x)
+    q, sf, g = Q.quantize_nvfp4_rowwise(bits, rht=True, rht_seed=1, sr=True, sr_seed=2)
+    assert np.array_equal(host(out["q_row"]), q) and np.array_equal(host(out["sf_row"]), sf.ravel())
+    q, sf, g = Q.quantize_nvfp4_colwise(bits, rht=True, rht_seed=1, sr=True, sr_seed=2)
+    assert np.array_equal(host(out["q_col"]), q) and np.array_equal(host(out["sf_col"]), sf.ravel())
+    assert int((host(out["q_row"]) & 0x77).max()) == 0 and int(host(out["sf_row"]).max()) == 0
     assert host(out["g_row"])[0] == 1.0 and host(out["g_col"])[0] == 1.0
 
 
