@@ -20,8 +20,8 @@ __all__ = [
     "FP8Q_FPROP", "FP8Q_DGRAD", "FP8Q_WGRAD", "FP8Q_SF_ROWMAJOR", "FP8Q_SF_MMA_TILED",
     "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
-    "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
-    "fp8q_status_string", "fp8q_version", "GemmArgs",
+    "fp8q_quantize_tensor_noalloc", "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
+    "fp8q_get_device_status", "fp8q_status_string", "fp8q_version", "GemmArgs",
     "quantize_1x128", "quantize_128x128", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
     "gemm", "device_status", "EXPORTED_SYMBOLS",
 ]
@@ -36,7 +36,7 @@ FP4Q_ROW, FP4Q_COL = 1, 2
 EXPORTED_SYMBOLS = [
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
-    "fp8q_release_scratch", "fp8q_status_string", "fp8q_version",
+    "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -77,6 +77,7 @@ def lib():
         L.fp8q_quantize_128x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
         L.fp8q_quantize_mx32.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_quantize_tensor.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
+        L.fp8q_quantize_tensor_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
         L.fp4q_rht16_quantize_sr.argtypes = [_vp, _i64, _i64, _i64, _int, _u64, _int, _u64,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
@@ -136,6 +137,12 @@ def fp8q_quantize_mx32(x, rows, cols, ld_x, q_row, e_row, q_col, e_col, sf_layou
 
 def fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream):
     return lib().fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream)
+
+
+def fp8q_quantize_tensor_noalloc(x, rows, cols, ld_x, q, s_dec, stream):
+    """Per-tensor quantization that allocates no device memory (scratch in the library's
+    fixed device array); for callers that cannot let a library allocate."""
+    return lib().fp8q_quantize_tensor_noalloc(x, rows, cols, ld_x, q, s_dec, stream)
 
 
 def fp4q_rht16_quantize_sr(x, rows, cols, ld_x, rht, rht_seed, sr, sr_seed, q_row, sf_row, g_row,

@@ -5,6 +5,9 @@
 // on the FP32 bit pattern, which orders like the value for non-negative floats) and a cast.
 // Both are 2-D grids over (16-byte column chunks, rows) so no thread divides by the row
 // length; the row loop strides by gridDim.y.
+#include <mutex>
+
+#include "../../include/fp8q.h"
 #include "common.cuh"
 #include "kernels.h"
 
@@ -74,4 +77,64 @@ cudaError_t launch_tensor_cast(const uint16_t* x, int64_t rows, int64_t cols, in
   return cudaGetLastError();
 }
 
+// ------------------------------------------------------------------ allocation-free variant
+// Scratch of fp8q_quantize_tensor_noalloc: a fixed array in the library's own device
+// globals, so the call never allocates.  Word 0 holds the running amax of the current call.
+namespace {
+constexpr int kNoAllocWords = 64;  // 256 bytes on every device that loads the library
+constexpr int kNoAllocMaxDevices = 64;
+static __device__ __align__(256) uint32_t g_noalloc_scratch[kNoAllocWords];
+uint32_t* g_noalloc_addr[kNoAllocMaxDevices] = {};
+std::mutex g_noalloc_mutex;
+
+// Device address of g_noalloc_scratch on the current device (the host-side symbol is only
+// a stand-in); looked up once per device, with that device current.
+cudaError_t noalloc_scratch(uint32_t** out) {
+  int dev = 0;
+  cudaError_t e = cudaGetDevice(&dev);
+  if (e != cudaSuccess) return e;
+  if (dev < 0 || dev >= kNoAllocMaxDevices) return cudaErrorInvalidDevice;
+  std::lock_guard<std::mutex> lock(g_noalloc_mutex);
+  if (g_noalloc_addr[dev] == nullptr) {
+    void* p = nullptr;
+    e = cudaGetSymbolAddress(&p, g_noalloc_scratch);
+    if (e != cudaSuccess) return e;
+    g_noalloc_addr[dev] = static_cast<uint32_t*>(p);
+  }
+  *out = g_noalloc_addr[dev];
+  return cudaSuccess;
+}
+}  // namespace
+
 }  // namespace fp8q
+
+extern "C" fp8q_status fp8q_quantize_tensor_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                                    uint8_t* q, float* s_dec, void* stream) {
+  using namespace fp8q;
+  if (rows < 0 || cols < 0 || rows >= (1ll << 31) || cols >= (1ll << 31)) return FP8Q_ERR_SHAPE;
+  if (!q || !s_dec) return FP8Q_ERR_NULL;
+  if (rows > 0 && cols > 0) {
+    if (!x) return FP8Q_ERR_NULL;
+    if (ld_x < cols || ld_x % 8 != 0) return FP8Q_ERR_SHAPE;
+    if ((reinterpret_cast<uintptr_t>(x) & 15u) != 0) return FP8Q_ERR_ALIGN;
+  }
+  if (cols % 8 != 0) return FP8Q_ERR_SHAPE;
+  if ((reinterpret_cast<uintptr_t>(q) & 15u) != 0) return FP8Q_ERR_ALIGN;
+  constexpr int kWordsNeeded = 1;  // one amax word per call
+  static_assert(kWordsNeeded <= kNoAllocWords, "scratch array too small");
+  if (kWordsNeeded > kNoAllocWords) return FP8Q_ERR_UNSUPPORTED;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint32_t* amax = nullptr;
+  if (noalloc_scratch(&amax) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (rows == 0 || cols == 0) {
+    const float one = 1.0f;  // empty tensor: amax 0 -> sf 1 -> decode scale 1
+    if (cudaMemcpyAsync(s_dec, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess) return FP8Q_ERR_CUDA;
+    return cudaStreamSynchronize(s) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+  }
+  // the array keeps the previous call's amax: clear the word before this call's reduction
+  if (cudaMemsetAsync(amax, 0, kWordsNeeded * sizeof(uint32_t), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  cudaError_t e = launch_tensor_amax(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax, s);
+  if (e == cudaSuccess) e = launch_tensor_cast(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax, q, s_dec, s);
+  return e == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
+}
+

@@ -128,6 +128,28 @@ fp8q_status fp8q_quantize_mx32(const void* x, int64_t rows, int64_t cols, int64_
 fp8q_status fp8q_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
                                  uint8_t* q, float* s_dec, void* stream);
 
+/* Allocation-free variant of fp8q_quantize_tensor (no counterpart in the pages: it is a
+ * library-integration entry point, not part of the method).  Same arguments, rules and
+ * results as fp8q_quantize_tensor.
+ * Who needs it: callers that cannot let a library allocate device memory - for example an
+ * application whose allocator owns all device memory and forbids foreign cudaMalloc calls,
+ * or one that runs under a fixed memory budget where a lazy allocation on first use could
+ * fail at an arbitrary point (and cudaMalloc/cudaFree may synchronize the device).
+ * fp8q_quantize_tensor allocates the library's scratch pool on its first call per device;
+ * this entry point calls no cudaMalloc, cudaFree or allocating library routine.  Its
+ * scratch is a fixed 256-byte array (64 words) in the library's device globals, present on
+ * every GPU that loads the library until the process exits; one call needs 1 word (the
+ * running amax), and a request needing more than the array holds is rejected with
+ * FP8Q_ERR_UNSUPPORTED.
+ * The first call on a device looks up the array's device address (cudaGetSymbolAddress,
+ * with that device current); make that first call before any stream capture.
+ * Every call shares the array and it keeps the last call's contents: each call clears the
+ * amax word on `stream` before using it.  Calls that overlap on the GPU (different streams
+ * without ordering, or different host threads) race on the array and may return wrong
+ * scales; serialize them. */
+fp8q_status fp8q_quantize_tensor_noalloc(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                         uint8_t* q, float* s_dec, void* stream);
+
 /* [NVFP4] 4-bit quantization with optional 16x16 random Hadamard transform and
  * stochastic rounding.
  *   G = amax of the (transformed) tensor; S_g = 2688 / G (G == 0 -> 1);
