@@ -358,11 +358,13 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (!make_map(&ma, a->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, a->M, a->lda, 128, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_CUDA;
-  if (!make_map(&mb, a->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, b_rows, a->ldb, 128, 256,
+  // B box rows = the kernel's tile width: 192 for the blockwise (promotion) kernel, 256 otherwise
+  const uint32_t bn = (a->recipe == FP8Q_BLOCKWISE) ? kBlockwiseTileN : 256;
+  if (!make_map(&mb, a->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, b_rows, a->ldb, 128, bn,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_CUDA;
   if (a->recipe == FP8Q_BLOCKWISE && a->layout == FP8Q_WGRAD) {
-    if (!make_map(&msb, a->b_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a->N, a->K / 128, a->ld_sb * 4, 256, 1,
+    if (!make_map(&msb, a->b_scale, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a->N, a->K / 128, a->ld_sb * 4, bn, 1,
                   CU_TENSOR_MAP_SWIZZLE_NONE))
       return FP8Q_ERR_CUDA;
   } else {

@@ -51,6 +51,10 @@ cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMM
+// Output tile width of the blockwise (FP32-promotion) kernel; the B and wgrad-scale TMA boxes
+// are built with it.
+constexpr uint32_t kBlockwiseTileN = 192;
+
 struct GemmParams {
   int recipe;       // fp8q_recipe
   int layout;       // fp8q_layout
