@@ -358,9 +358,11 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (!make_map(&ma, a->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, a->M, a->lda, 128, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_CUDA;
-  // B box rows = the kernel's tile width: 192 for the blockwise (promotion) kernel, 256 otherwise
+  // B box rows: each CTA of a blockwise pair loads half of the 192-column tile; the other
+  // kernel loads its whole 256-column tile.  The wgrad scale box spans the full tile width.
   const uint32_t bn = (a->recipe == FP8Q_BLOCKWISE) ? kBlockwiseTileN : 256;
-  if (!make_map(&mb, a->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, b_rows, a->ldb, 128, bn,
+  const uint32_t b_box = (a->recipe == FP8Q_BLOCKWISE) ? kBlockwiseTileN / 2 : 256;
+  if (!make_map(&mb, a->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, b_rows, a->ldb, 128, b_box,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_CUDA;
   if (a->recipe == FP8Q_BLOCKWISE && a->layout == FP8Q_WGRAD) {

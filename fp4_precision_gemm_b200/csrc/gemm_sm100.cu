@@ -310,7 +310,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive(accempty);
+      if (lane == 0) mbar_arrive_relaxed(accempty);
     }
   }
 
@@ -323,35 +323,86 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ blockwise (promotion) kernel
-// 128 x 192 output tiles; warps 0-11 promote (warp w: TMEM lanes 32*(w%4).., columns
-// 64*(w/4)..), warp 12 drives TMA, warp 13 allocates TMEM and issues the MMAs.  With at most
-// four warps per SM sub-partition each thread may use 128 registers: its 64 FP32
-// accumulators stay in registers for the whole tile and a chunk's 64 partial columns are
-// drained from TMEM in two 32-column loads.  Two 192-column TMEM partial buffers alternate
-// per 128-element K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted.
+// CTA pairs (clusters of 2) share 256 x 192 output tiles with the pair MMA
+// (tcgen05.mma.cta_group::2, M = 256): each CTA loads its own 128 rows of A and its half (96
+// rows) of B, so an SM moves 28 KB per 128-element K chunk instead of 40 KB, and each CTA's
+// TMEM receives its 128 rows of the chunk's partial.  The leader CTA's single MMA thread
+// issues for both; the TMA completions of both CTAs are counted on the leader's barrier and
+// the MMA commits arrive on both CTAs' barriers (multicast commit, no multicast loads).
+// In each CTA warps 0-11 promote (warp w: TMEM lanes 32*(w%4).., columns 64*(w/4)..),
+// warp 12 drives TMA, warp 13 owns TMEM (and, in the leader, issues the MMAs).  With at
+// most four warps per SM sub-partition a thread may use 128 registers: its 64 FP32
+// accumulators stay in registers for the whole tile.  Two 192-column TMEM partial buffers
+// alternate per K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted.
 namespace {
 
-constexpr int kBwBN = (int)kBlockwiseTileN;
+constexpr int kBwBN = (int)kBlockwiseTileN;     // 192 output columns per pair tile
+constexpr int kBwHalfBN = kBwBN / 2;            // B rows loaded by each CTA
+constexpr int kBwPairM = 2 * kBM;               // 256 output rows per pair tile
 constexpr int kBwEpiWarps = 12;
 constexpr int kBwProducerWarp = 12, kBwMmaWarp = 13;
 constexpr int kBwThreads = 14 * 32;
-constexpr int kBwStages = 5;
-constexpr int kBwSb = 4;                        // wgrad B-scale ring
-constexpr uint32_t kBwBStage = kBwBN * kBKB;    // 24 KB
+constexpr int kBwStages = 7;
+constexpr int kBwSb = 10;                       // scale ring: chunks of A/B scales staged ahead
+// One scale-ring slot: [wgrad B scales, 192 floats][A scales of the CTA's 128 rows][B scales
+// of the three 64-column groups (fprop/dgrad)], padded to a multiple of 128 bytes.
+constexpr uint32_t kSlotSbw = 0, kSlotSa = kBwBN * 4, kSlotSb = kSlotSa + kBM * 4;
+constexpr uint32_t kSlotBytes = ((kSlotSb + 16 + 127) / 128) * 128;
+constexpr uint32_t kBwBStage = kBwHalfBN * kBKB;  // 12 KB
 
 template <int L>
 struct BwSmem {
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + kBwStages * kAStage;
-  static constexpr uint32_t sbw = b + kBwStages * kBwBStage;
-  static constexpr uint32_t sbw_bytes = (L == kWgrad) ? kBwSb * kBwBN * 4 : 0;
-  static constexpr uint32_t bars = sbw + sbw_bytes;
+  static constexpr uint32_t ring = b + kBwStages * kBwBStage;
+  static constexpr uint32_t bars = ring + kBwSb * kSlotBytes;
   static constexpr uint32_t n_bars = 2 * kBwStages + 2 + 2 + 2 * kBwSb + 1;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t groups = misc + 16;
   static constexpr uint32_t total = groups + 2 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t alloc = total + 1024;
 };
+
+// Pair tile t: 256 rows x 192 columns, rasterized like tile_of; grouped GEMMs enumerate each
+// expert's 256-row tiles.  Returns this CTA's 128-row half.
+__device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
+                                             const int* offs, uint32_t rank) {
+  const int per = kGroupM * p.tiles_n;
+  const int grp = t / per, first = grp * kGroupM;
+  const int gsz = min(row_tiles - first, kGroupM);
+  const int local = t - grp * per;
+  const int rt = first + local % gsz, nt = local / gsz;
+  Tile T;
+  T.n0 = nt * kBwBN;
+  int end;
+  if (p.num_groups > 0) {
+    int g = 0;
+    while (g + 1 < p.num_groups && prefix[g + 1] <= rt) ++g;
+    T.g = g;
+    T.m0 = offs[g] + (rt - prefix[g]) * kBwPairM;
+    end = offs[g + 1];
+  } else {
+    T.g = 0;
+    T.m0 = rt * kBwPairM;
+    end = p.M;
+  }
+  T.m0 += (int)rank * kBM;
+  T.mend = min(end, T.m0 + kBM);
+  return T;
+}
+
+__device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefix, int* offs, int lane) {
+  for (int g = lane; g <= p.num_groups; g += 32) offs[g] = p.m_offsets[g];
+  __syncwarp();
+  if (lane == 0) {
+    int acc = 0;
+    for (int g = 0; g < p.num_groups; ++g) {
+      prefix[g] = acc;
+      acc += (offs[g + 1] - offs[g] + kBwPairM - 1) / kBwPairM;
+    }
+    prefix[p.num_groups] = acc;
+  }
+}
 
 }  // namespace
 
@@ -363,19 +414,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   constexpr bool kWg = (L == kWgrad);
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars);
-  uint64_t* empty = full + kBwStages;
-  uint64_t* pfull = empty + kBwStages;   // [2] partial of a chunk in TMEM buffer b
-  uint64_t* pempty = pfull + 2;          // [2] buffer b drained by every promotion thread
-  uint64_t* sbfull = pempty + 2;
-  uint64_t* sbempty = sbfull + kBwSb;
-  uint64_t* final_bar = sbempty + kBwSb;
+  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars);   // leader: both halves landed
+  uint64_t* empty = full + kBwStages;    // both CTAs: the stage's MMAs are done
+  uint64_t* pfull = empty + kBwStages;   // both CTAs: [2] chunk partial in TMEM buffer b
+  uint64_t* pempty = pfull + 2;          // leader: [2] buffer b drained by both CTAs
+  uint64_t* sfull = pempty + 2;          // local scale ring: slot filled
+  uint64_t* sempty = sfull + kBwSb;      // local scale ring: slot read by every promotion warp
+  uint64_t* final_bar = sempty + kBwSb;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::misc + 4);
   int* prefix = reinterpret_cast<int*>(smem + S::groups);
   int* offs = prefix + kMaxGroups + 1;
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const uint32_t rank = cluster_ctarank();
+  const bool leader = rank == 0;
   const int KB = p.K / kBKB;
 
   if (threadIdx.x == 0) {
@@ -383,71 +436,110 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    // drain barriers take one arrival per promotion warp (lane 0, after __syncwarp), not
-    // one per thread: hundreds of arrivals on one shared word per chunk serialize
     for (int i = 0; i < 2; ++i) {
       mbar_init(&pfull[i], 1);
-      mbar_init(&pempty[i], kBwEpiWarps);
+      mbar_init(&pempty[i], 2 * kBwEpiWarps);  // one arrival per promotion warp of both CTAs
     }
     for (int i = 0; i < kBwSb; ++i) {
-      mbar_init(&sbfull[i], 1);
-      mbar_init(&sbempty[i], kBwEpiWarps);
+      mbar_init(&sfull[i], 33);  // lane 0's expect-tx arrival + 32 cp.async arrivals
+      mbar_init(&sempty[i], kBwEpiWarps);
     }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
   }
-  if (GROUPED && warp == kBwProducerWarp) load_groups(p, prefix, offs, lane);
+  if (GROUPED && warp == kBwProducerWarp) load_pair_groups(p, prefix, offs, lane);
   if (warp == kBwMmaWarp) {
-    tmem_alloc(tmem_slot, 512);
-    tmem_relinquish();
+    tmem_alloc_pair(tmem_slot, 512);
+    tmem_relinquish_pair();
   }
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();
+  cluster_sync();   // barriers and TMEM of both CTAs exist before either CTA uses them
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int row_tiles = GROUPED ? prefix[p.num_groups] : p.tiles_m;
   const int total = row_tiles * p.tiles_n;
+  const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
 
   if (warp == kBwProducerWarp) {
-    // ------------------------------------------------------------------ TMA producer
+    // ------------------------------------------------------------------ producer warp
+    // lane 0: TMA of the A / B halves (completion counted on the leader's barrier);
+    // all lanes: the chunk's scales into the scale ring, so the promotion warps never wait
+    // on global memory.
     if (lane == 0) {
       tma_prefetch_desc(&tma_a);
       tma_prefetch_desc(&tma_b);
       if (kWg) tma_prefetch_desc(&tma_sb);
-      uint32_t it = 0, sbit = 0;
-      bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-        const Tile T = tile_of(t, p, row_tiles, prefix, offs, kBwBN);
-        const int b_row = T.g * p.N + T.n0;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
-          const uint32_t s = it % kBwStages, ph = (it / kBwStages) & 1;
-          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], kAStage + kBwBStage);
-          tma_load_2d(smem + S::a + s * kAStage, &tma_a, &full[s], kb * kBKB, T.m0);
-          tma_load_2d(smem + S::b + s * kBwBStage, &tma_b, &full[s], kb * kBKB, b_row);
-          if (kWg) {
-            const uint32_t ss = sbit % kBwSb, sph = (sbit / kBwSb) & 1;
-            if (!mbar_wait(&sbempty[ss], sph ^ 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
-            mbar_arrive_expect_tx(&sbfull[ss], kBwBN * 4);
-            tma_load_2d(smem + S::sbw + ss * kBwBN * 4, &tma_sb, &sbfull[ss], T.n0, kb);
-            ++sbit;
+    }
+    uint32_t it = 0;
+    bool ok = true;
+    for (int t = cluster; t < total && ok; t += n_clusters) {
+      const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
+      const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
+      const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
+      for (int kb = 0; kb < KB; ++kb, ++it) {
+        const uint32_t s = it % kBwStages, ph = (it / kBwStages) & 1;
+        const uint32_t r = it % kBwSb, rph = (it / kBwSb) & 1;
+        int good = 1;
+        if (lane == 0) {
+          good = mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs) &&
+                 mbar_wait(&sempty[r], rph ^ 1, abort_flag, kWaitLimitNs);
+          if (good) {
+            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kAStage + kBwBStage));
+            const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+            tma_load_2d_pair(smem + S::a + s * kAStage, &tma_a, bar, kb * kBKB, T.m0);
+            tma_load_2d_pair(smem + S::b + s * kBwBStage, &tma_b, bar, kb * kBKB, b_row);
+          } else {
+            raise_timeout(p, abort_flag);
           }
         }
+        if (!__shfl_sync(0xFFFFFFFFu, good, 0)) { ok = false; break; }
+        // scales land through cp.async: the producer does not wait for them, the slot's
+        // barrier completes once all 32 lanes' copies (and the wgrad TMA) have landed
+        uint8_t* slot = smem + S::ring + r * kSlotBytes;
+        float* ssa = reinterpret_cast<float*>(slot + kSlotSa);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {
+          const int m = T.m0 + i * 32 + lane;
+          const bool in = m < p.M;
+          cp_async_4(ssa + i * 32 + lane, p.sa + (in ? (int64_t)kb * p.ld_sa + m : 0), in ? 4u : 0u);
+        }
+        if (!kWg && lane < 3) {
+          const int ncol0 = T.n0 + lane * 64, nblk = ncol0 / kBM;
+          const bool in = ncol0 < p.N;
+          const int64_t off = !in ? 0 : (L == kFprop) ? (int64_t)nblk * p.ld_sb + kb : (int64_t)kb * p.ld_sb + nblk;
+          cp_async_4(reinterpret_cast<float*>(slot + kSlotSb) + lane, sbg + off, in ? 4u : 0u);
+        }
+        if (lane == 0) {
+          mbar_arrive_expect_tx(&sfull[r], kWg ? kBwBN * 4 : 0);
+          if (kWg) tma_load_2d(slot + kSlotSbw, &tma_sb, &sfull[r], T.n0, kb);
+        }
+        cp_async_arrive_noinc(&sfull[r]);
       }
+    }
+    asm volatile("cp.async.wait_all;" ::: "memory");  // no scale copy outlives the CTA
+    if (lane == 0 && leader) {  // the leader's barriers see both halves: wait for the copies in flight
       const uint32_t inflight = it < (uint32_t)kBwStages ? it : (uint32_t)kBwStages;
       for (uint32_t j = 0; j < inflight; ++j) {
         const uint32_t i2 = it - 1 - j;
         mbar_wait_drain(&full[i2 % kBwStages], (i2 / kBwStages) & 1, kWaitLimitNs);
       }
     }
+    if (kWg && lane == 0) {  // the wgrad B-scale TMA of the last slots
+      const uint32_t inflight = it < (uint32_t)kBwSb ? it : (uint32_t)kBwSb;
+      for (uint32_t j = 0; j < inflight; ++j) {
+        const uint32_t i2 = it - 1 - j;
+        mbar_wait_drain(&sfull[i2 % kBwSb], (i2 / kBwSb) & 1, kWaitLimitNs);
+      }
+    }
   } else if (warp == kBwMmaWarp) {
-    // ------------------------------------------------------------------ MMA issuer
-    if (lane == 0) {
-      constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kBwBN >> 3) << 17) | ((uint32_t)(kBM >> 4) << 24);
+    // ------------------------------------------------------------------ MMA issuer (leader)
+    if (lane == 0 && leader) {
+      constexpr uint32_t idesc = (1u << 4) | ((uint32_t)(kBwBN >> 3) << 17) | ((uint32_t)(kBwPairM >> 4) << 24);
       uint32_t it = 0;
       bool ok = true;
-      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+      for (int t = cluster; t < total && ok; t += n_clusters) {
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % kBwStages, ph = (it / kBwStages) & 1, pb = it & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimitNs) ||
@@ -460,12 +552,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           const uint64_t adesc = smem_desc(smem_u32(smem + S::a + s * kAStage), 16, 1024, 2);
           const uint64_t bdesc = smem_desc(smem_u32(smem + S::b + s * kBwBStage), 16, 1024, 2);
 #pragma unroll
-          for (int k = 0; k < 4; ++k) mma_f8f6f4(tmem + pb * kBwBN, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
-          mma_commit(&empty[s]);
-          mma_commit(&pfull[pb]);
+          for (int k = 0; k < 4; ++k) mma_f8f6f4_pair(tmem + pb * kBwBN, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+          mma_commit_pair(&empty[s], 0x3);
+          mma_commit_pair(&pfull[pb], 0x3);
         }
       }
-      mma_commit(final_bar);
+      mma_commit_pair(final_bar, 0x1);
       mbar_wait_drain(final_bar, 0, kWaitLimitNs);
     }
   } else {
@@ -473,39 +565,24 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     const int q = warp & 3, cgp = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cgp * 64);
     const int rloc = q * 32 + lane;
-    uint32_t chunk = 0, sbit = 0;
+    const uint32_t pempty_leader0 = mapa_shared(smem_u32(&pempty[0]), 0);
+    const uint32_t pempty_leader1 = mapa_shared(smem_u32(&pempty[1]), 0);
+    uint32_t chunk = 0;
     bool ok = true;
-    for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
-      const Tile T = tile_of(t, p, row_tiles, prefix, offs, kBwBN);
+    for (int t = cluster; t < total && ok; t += n_clusters) {
+      const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
       const int m = T.m0 + rloc;
       const int ncol0 = T.n0 + cgp * 64;
-      const int nblk = ncol0 / kBM;
-      const bool sa_ok = m < p.M, nb_ok = ncol0 < p.N;
-      const float* sa_row = p.sa + (sa_ok ? m : 0);
-      const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
-      auto b_scale = [&](int kb) -> float {
-        if (L == kFprop) return nb_ok ? __ldg(sbg + (int64_t)nblk * p.ld_sb + kb) : 0.0f;
-        if (L == kDgrad) return nb_ok ? __ldg(sbg + (int64_t)kb * p.ld_sb + nblk) : 0.0f;
-        return 1.0f;
-      };
       float2 acc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
-      float sa_next = sa_ok ? __ldg(sa_row) : 0.0f;
-      float sb_next = b_scale(0);
       for (int kb = 0; kb < KB; ++kb) {
-        const float sa = sa_next, sbv = sb_next;
-        if (kb + 1 < KB) {
-          sa_next = sa_ok ? __ldg(sa_row + (int64_t)(kb + 1) * p.ld_sa) : 0.0f;
-          sb_next = b_scale(kb + 1);
-        }
-        const float* sbw = nullptr;
-        uint32_t ss = 0;
-        if (kWg) {
-          ss = sbit % kBwSb;
-          if (!mbar_wait(&sbfull[ss], (sbit / kBwSb) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
-          sbw = reinterpret_cast<const float*>(smem + S::sbw + ss * kBwBN * 4) + cgp * 64;
-        }
+        const uint32_t rs = chunk % kBwSb;
+        if (!mbar_wait(&sfull[rs], (chunk / kBwSb) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+        const uint8_t* slot = smem + S::ring + rs * kSlotBytes;
+        const float sa = reinterpret_cast<const float*>(slot + kSlotSa)[rloc];
+        const float sbv = kWg ? 1.0f : reinterpret_cast<const float*>(slot + kSlotSb)[cgp];
+        const float* sbw = reinterpret_cast<const float*>(slot + kSlotSbw) + cgp * 64;
         const uint32_t pb = chunk & 1;
         if (!mbar_wait(&pfull[pb], (chunk >> 1) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
         tc_fence_after();
@@ -526,10 +603,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive(&pempty[pb]);
-          if (kWg) mbar_arrive(&sbempty[ss]);
+          mbar_arrive_cluster_relaxed(pb ? pempty_leader1 : pempty_leader0);
+          mbar_arrive_relaxed(&sempty[rs]);
         }
-        if (kWg) ++sbit;
         ++chunk;
       }
       if (!ok) break;
@@ -548,10 +624,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
 
   tc_fence_before();
-  __syncthreads();
+  __syncwarp();     // role loops ran on lane 0 only: reconverge before the aligned barrier
+  cluster_sync();   // the leader's MMAs into both TMEMs are complete before either frees
   if (warp == kBwMmaWarp) {
     tc_fence_after();
-    tmem_dealloc(tmem, 512);
+    tmem_dealloc_pair(tmem, 512);
   }
 }
 
@@ -564,11 +641,29 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   if (e != cudaSuccess) return e;
   GemmParams q = p;
   q.tiles_n = (p.N + kBwBN - 1) / kBwBN;
+  q.tiles_m = G ? (p.M + kBwPairM - 1) / kBwPairM + p.num_groups : (p.M + kBwPairM - 1) / kBwPairM;
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
-  int grid = (int)(tiles < num_sms ? tiles : num_sms);
-  if (grid < 1) grid = 1;
-  kern<<<grid, kBwThreads, smem, s>>>(q, a, b, sb);
-  return cudaGetLastError();
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(num_sms - (num_sms & 1));
+  cfg.blockDim = dim3(kBwThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  // persistent: as many pairs as can be resident at once (never more than the tiles)
+  int resident = 0;
+  e = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg);
+  if (e != cudaSuccess) return e;
+  int clusters = resident < num_sms / 2 ? resident : num_sms / 2;
+  if (clusters > tiles) clusters = (int)tiles;
+  if (clusters < 1) clusters = 1;
+  cfg.gridDim = dim3(2 * clusters);
+  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb);
 }
 
 template <int R>
