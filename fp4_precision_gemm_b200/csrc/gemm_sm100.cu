@@ -94,6 +94,17 @@ __device__ __forceinline__ void store8(const GemmParams& p, int m, int n, const 
   }
 }
 
+// Eight packed BF16 values at (m, n..n+7); scalar stores past column N.
+__device__ __forceinline__ void store8_bf16(const GemmParams& p, int m, int n, uint4 v) {
+  uint16_t* dst = p.c + (int64_t)m * p.ldc + n;
+  if (n + 8 <= p.N) {
+    *reinterpret_cast<uint4*>(dst) = v;
+  } else {
+    const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+    for (int i = 0; i < 8 && n + i < p.N; ++i) dst[i] = (uint16_t)(w[i >> 1] >> (16 * (i & 1)));
+  }
+}
+
 // Expert offsets and the running count of row tiles per expert, into shared memory.
 __device__ __forceinline__ void load_groups(const GemmParams& p, int* prefix, int* offs, int lane) {
   for (int g = lane; g <= p.num_groups; g += 32) offs[g] = p.m_offsets[g];
@@ -330,37 +341,49 @@ __global__ void __launch_bounds__(kThreads, 1)
 // issues for both; the TMA completions of both CTAs are counted on the leader's barrier and
 // the MMA commits arrive on both CTAs' barriers (multicast commit, no multicast loads).
 // In each CTA warps 0-11 promote (warp w: TMEM lanes 32*(w%4).., columns 64*(w/4)..),
-// warp 12 drives TMA, warp 13 owns TMEM (and, in the leader, issues the MMAs).  With at
-// most four warps per SM sub-partition a thread may use 128 registers: its 64 FP32
-// accumulators stay in registers for the whole tile.  Two 192-column TMEM partial buffers
-// alternate per K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted.
+// warp 12 drives the A/B TMA, warp 13 owns TMEM (and, in the leader, issues the MMAs) and
+// warp 14 stages each chunk's scales in a shared-memory ring.  With at most four warps per SM
+// sub-partition a thread may use 128 registers: its 64 FP32 accumulators stay in registers
+// for the whole tile.  Two 192-column TMEM partial buffers alternate per K chunk, so the MMAs
+// of chunk k + 1 run while chunk k is promoted; the stage's single commit tells both the
+// producers (stage free) and the promotion warps (partial complete) of both CTAs.
 namespace {
 
 constexpr int kBwBN = (int)kBlockwiseTileN;     // 192 output columns per pair tile
 constexpr int kBwHalfBN = kBwBN / 2;            // B rows loaded by each CTA
 constexpr int kBwPairM = 2 * kBM;               // 256 output rows per pair tile
 constexpr int kBwEpiWarps = 12;
-constexpr int kBwProducerWarp = 12, kBwMmaWarp = 13;
-constexpr int kBwThreads = 14 * 32;
-constexpr int kBwStages = 7;
+constexpr int kBwProducerWarp = 12, kBwMmaWarp = 13, kBwScaleWarp = 14;
+constexpr int kBwThreads = 15 * 32;
 constexpr int kBwSb = 10;                       // scale ring: chunks of A/B scales staged ahead
-// One scale-ring slot: [wgrad B scales, 192 floats][A scales of the CTA's 128 rows][B scales
-// of the three 64-column groups (fprop/dgrad)], padded to a multiple of 128 bytes.
-constexpr uint32_t kSlotSbw = 0, kSlotSa = kBwBN * 4, kSlotSb = kSlotSa + kBM * 4;
-constexpr uint32_t kSlotBytes = ((kSlotSb + 16 + 127) / 128) * 128;
 constexpr uint32_t kBwBStage = kBwHalfBN * kBKB;  // 12 KB
 
+
+// Shared memory of the blockwise kernel.  A scale-ring slot holds one chunk's scales:
+// wgrad: [B scales of the 192 columns][A scales of the CTA's 128 rows];
+// fprop/dgrad: [A scales][the B scales of the tile's three 64-column groups].
 template <int L>
 struct BwSmem {
+  static constexpr bool wg = (L == kWgrad);
+  static constexpr int stages = 6;
+  static constexpr uint32_t slot_sbw = 0;
+  static constexpr uint32_t slot_sa = wg ? kBwBN * 4 : 0;
+  static constexpr uint32_t slot_sb = slot_sa + kBM * 4;
+  static constexpr uint32_t slot_bytes = ((slot_sb + (wg ? 0 : 16) + 127) / 128) * 128;
   static constexpr uint32_t a = 0;
-  static constexpr uint32_t b = a + kBwStages * kAStage;
-  static constexpr uint32_t ring = b + kBwStages * kBwBStage;
-  static constexpr uint32_t bars = ring + kBwSb * kSlotBytes;
-  static constexpr uint32_t n_bars = 2 * kBwStages + 2 + 2 + 2 * kBwSb + 1;
+  static constexpr uint32_t b = a + stages * kAStage;
+  static constexpr uint32_t ring = b + stages * kBwBStage;
+  // epilogue staging per promotion warp: 32 rows x epi_cols BF16 (wgrad: half the width)
+  static constexpr int epi_cols = wg ? 32 : 64;
+  static constexpr uint32_t stage_c = 32 * epi_cols * 2;
+  static constexpr uint32_t cst = ring + kBwSb * slot_bytes;
+  static constexpr uint32_t bars = cst + kBwEpiWarps * stage_c;
+  static constexpr uint32_t n_bars = 2 * stages + 2 + 2 * kBwSb + 1;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t groups = misc + 16;
   static constexpr uint32_t total = groups + 2 * (kMaxGroups + 1) * 4;
   static constexpr uint32_t alloc = total + 1024;
+  static_assert(alloc <= 227 * 1024, "shared memory");
 };
 
 // Pair tile t: 256 rows x 192 columns, rasterized like tile_of; grouped GEMMs enumerate each
@@ -412,12 +435,12 @@ __global__ void __launch_bounds__(kBwThreads, 1)
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
+  constexpr int kStages = S::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars);   // leader: both halves landed
-  uint64_t* empty = full + kBwStages;    // both CTAs: the stage's MMAs are done
-  uint64_t* pfull = empty + kBwStages;   // both CTAs: [2] chunk partial in TMEM buffer b
-  uint64_t* pempty = pfull + 2;          // leader: [2] buffer b drained by both CTAs
+  uint64_t* empty = full + kStages;    // both CTAs: the stage's MMAs are done (partial ready)
+  uint64_t* pempty = empty + kStages;  // leader: [2] TMEM buffer b drained by both CTAs
   uint64_t* sfull = pempty + 2;          // local scale ring: slot filled
   uint64_t* sempty = sfull + kBwSb;      // local scale ring: slot read by every promotion warp
   uint64_t* final_bar = sempty + kBwSb;
@@ -432,14 +455,11 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const int KB = p.K / kBKB;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kBwStages; ++i) {
+    for (int i = 0; i < kStages; ++i) {
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    for (int i = 0; i < 2; ++i) {
-      mbar_init(&pfull[i], 1);
-      mbar_init(&pempty[i], 2 * kBwEpiWarps);  // one arrival per promotion warp of both CTAs
-    }
+    for (int i = 0; i < 2; ++i) mbar_init(&pempty[i], 2 * kBwEpiWarps);  // per promotion warp, both CTAs
     for (int i = 0; i < kBwSb; ++i) {
       mbar_init(&sfull[i], 33);  // lane 0's expect-tx arrival + 32 cp.async arrivals
       mbar_init(&sempty[i], kBwEpiWarps);
@@ -463,42 +483,59 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
 
   if (warp == kBwProducerWarp) {
-    // ------------------------------------------------------------------ producer warp
-    // lane 0: TMA of the A / B halves (completion counted on the leader's barrier);
-    // all lanes: the chunk's scales into the scale ring, so the promotion warps never wait
-    // on global memory.
+    // ------------------------------------------------------------------ A / B producer
+    // One thread: wait for a free stage, arm the leader's barrier, issue the two TMA loads.
+    // Nothing else runs on this thread, so it stays several chunks ahead of the MMAs.
     if (lane == 0) {
       tma_prefetch_desc(&tma_a);
       tma_prefetch_desc(&tma_b);
-      if (kWg) tma_prefetch_desc(&tma_sb);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = cluster; t < total && ok; t += n_clusters) {
+        const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
+        const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+          if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) {
+            raise_timeout(p, abort_flag);
+            ok = false;
+            break;
+          }
+          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kAStage + kBwBStage));
+          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          tma_load_2d_pair(smem + S::a + s * kAStage, &tma_a, bar, kb * kBKB, T.m0);
+          tma_load_2d_pair(smem + S::b + s * kBwBStage, &tma_b, bar, kb * kBKB, b_row);
+        }
+      }
+      if (leader) {  // the leader's barriers see both halves: wait for the copies in flight
+        const uint32_t inflight = it < (uint32_t)kStages ? it : (uint32_t)kStages;
+        for (uint32_t j = 0; j < inflight; ++j) {
+          const uint32_t i2 = it - 1 - j;
+          mbar_wait_drain(&full[i2 % kStages], (i2 / kStages) & 1, kWaitLimitNs);
+        }
+      }
     }
+  } else if (warp == kBwScaleWarp) {
+    // ------------------------------------------------------------------ scale loader
+    // All 32 lanes copy each chunk's scales into the scale ring with cp.async (the wgrad
+    // B-scale row by TMA); a slot's barrier completes once every lane's copies have landed,
+    // so the promotion warps read scales from shared memory only.
+    if (kWg && lane == 0) tma_prefetch_desc(&tma_sb);
     uint32_t it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
       const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
-      const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
       const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
       for (int kb = 0; kb < KB; ++kb, ++it) {
-        const uint32_t s = it % kBwStages, ph = (it / kBwStages) & 1;
         const uint32_t r = it % kBwSb, rph = (it / kBwSb) & 1;
         int good = 1;
         if (lane == 0) {
-          good = mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs) &&
-                 mbar_wait(&sempty[r], rph ^ 1, abort_flag, kWaitLimitNs);
-          if (good) {
-            if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kAStage + kBwBStage));
-            const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
-            tma_load_2d_pair(smem + S::a + s * kAStage, &tma_a, bar, kb * kBKB, T.m0);
-            tma_load_2d_pair(smem + S::b + s * kBwBStage, &tma_b, bar, kb * kBKB, b_row);
-          } else {
-            raise_timeout(p, abort_flag);
-          }
+          good = mbar_wait(&sempty[r], rph ^ 1, abort_flag, kWaitLimitNs);
+          if (!good) raise_timeout(p, abort_flag);
         }
         if (!__shfl_sync(0xFFFFFFFFu, good, 0)) { ok = false; break; }
-        // scales land through cp.async: the producer does not wait for them, the slot's
-        // barrier completes once all 32 lanes' copies (and the wgrad TMA) have landed
-        uint8_t* slot = smem + S::ring + r * kSlotBytes;
-        float* ssa = reinterpret_cast<float*>(slot + kSlotSa);
+        uint8_t* slot = smem + S::ring + r * S::slot_bytes;
+        float* ssa = reinterpret_cast<float*>(slot + S::slot_sa);
 #pragma unroll
         for (int i = 0; i < 4; ++i) {
           const int m = T.m0 + i * 32 + lane;
@@ -509,23 +546,16 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           const int ncol0 = T.n0 + lane * 64, nblk = ncol0 / kBM;
           const bool in = ncol0 < p.N;
           const int64_t off = !in ? 0 : (L == kFprop) ? (int64_t)nblk * p.ld_sb + kb : (int64_t)kb * p.ld_sb + nblk;
-          cp_async_4(reinterpret_cast<float*>(slot + kSlotSb) + lane, sbg + off, in ? 4u : 0u);
+          cp_async_4(reinterpret_cast<float*>(slot + S::slot_sb) + lane, sbg + off, in ? 4u : 0u);
         }
         if (lane == 0) {
           mbar_arrive_expect_tx(&sfull[r], kWg ? kBwBN * 4 : 0);
-          if (kWg) tma_load_2d(slot + kSlotSbw, &tma_sb, &sfull[r], T.n0, kb);
+          if (kWg) tma_load_2d(slot + S::slot_sbw, &tma_sb, &sfull[r], T.n0, kb);
         }
         cp_async_arrive_noinc(&sfull[r]);
       }
     }
     asm volatile("cp.async.wait_all;" ::: "memory");  // no scale copy outlives the CTA
-    if (lane == 0 && leader) {  // the leader's barriers see both halves: wait for the copies in flight
-      const uint32_t inflight = it < (uint32_t)kBwStages ? it : (uint32_t)kBwStages;
-      for (uint32_t j = 0; j < inflight; ++j) {
-        const uint32_t i2 = it - 1 - j;
-        mbar_wait_drain(&full[i2 % kBwStages], (i2 / kBwStages) & 1, kWaitLimitNs);
-      }
-    }
     if (kWg && lane == 0) {  // the wgrad B-scale TMA of the last slots
       const uint32_t inflight = it < (uint32_t)kBwSb ? it : (uint32_t)kBwSb;
       for (uint32_t j = 0; j < inflight; ++j) {
@@ -541,7 +571,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const uint32_t s = it % kBwStages, ph = (it / kBwStages) & 1, pb = it & 1;
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1, pb = it & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimitNs) ||
               !mbar_wait(&pempty[pb], ((it >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
             raise_timeout(p, abort_flag);
@@ -553,8 +583,9 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           const uint64_t bdesc = smem_desc(smem_u32(smem + S::b + s * kBwBStage), 16, 1024, 2);
 #pragma unroll
           for (int k = 0; k < 4; ++k) mma_f8f6f4_pair(tmem + pb * kBwBN, adesc + 2 * k, bdesc + 2 * k, idesc, k > 0);
+          // one commit per chunk: the stage is free for the producers and the partial is in
+          // TMEM for the promotion warps of both CTAs
           mma_commit_pair(&empty[s], 0x3);
-          mma_commit_pair(&pfull[pb], 0x3);
         }
       }
       mma_commit_pair(final_bar, 0x1);
@@ -579,25 +610,42 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       for (int kb = 0; kb < KB; ++kb) {
         const uint32_t rs = chunk % kBwSb;
         if (!mbar_wait(&sfull[rs], (chunk / kBwSb) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
-        const uint8_t* slot = smem + S::ring + rs * kSlotBytes;
-        const float sa = reinterpret_cast<const float*>(slot + kSlotSa)[rloc];
-        const float sbv = kWg ? 1.0f : reinterpret_cast<const float*>(slot + kSlotSb)[cgp];
-        const float* sbw = reinterpret_cast<const float*>(slot + kSlotSbw) + cgp * 64;
+        const uint8_t* slot = smem + S::ring + rs * S::slot_bytes;
+        const float sa = reinterpret_cast<const float*>(slot + S::slot_sa)[rloc];
+        const float sbv = kWg ? 1.0f : reinterpret_cast<const float*>(slot + S::slot_sb)[cgp];
+        const float* sbw = reinterpret_cast<const float*>(slot + S::slot_sbw) + cgp * 64;
         const uint32_t pb = chunk & 1;
-        if (!mbar_wait(&pfull[pb], (chunk >> 1) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+        // the stage's commit also means: this chunk's partial is complete in TMEM buffer pb
+        if (!mbar_wait(&empty[chunk % kStages], (chunk / kStages) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
         tc_fence_after();
         const float scale = kWg ? sa : __fmul_rn(sa, sbv);
         const float2 s2 = make_float2(scale, scale);
+        if constexpr (!kWg) {
 #pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          uint32_t r[32];
-          tmem_ld_32x32b_x32(t_lane + pb * kBwBN + h * 32, r);
-          tmem_ld_wait(r);
+          for (int h = 0; h < 2; ++h) {
+            uint32_t r[32];
+            tmem_ld_32x32b_x32(t_lane + pb * kBwBN + h * 32, r);
+            tmem_ld_wait(r);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) {
-            float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            if (kWg) pr = __fmul2_rn(pr, *reinterpret_cast<const float2*>(sbw + h * 32 + 2 * i));
-            acc[h * 16 + i] = __ffma2_rn(pr, s2, acc[h * 16 + i]);
+            for (int i = 0; i < 16; ++i) {
+              const float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              acc[h * 16 + i] = __ffma2_rn(pr, s2, acc[h * 16 + i]);
+            }
+          }
+        } else {
+          // wgrad also scales each column: 16 columns per TMEM load keeps the column scales
+          // and the loaded partial sums within the register budget
+#pragma unroll
+          for (int h = 0; h < 4; ++h) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(t_lane + pb * kBwBN + h * 16, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+              pr = __fmul2_rn(pr, *reinterpret_cast<const float2*>(sbw + h * 16 + 2 * i));
+              acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
+            }
           }
         }
         tc_fence_before();
@@ -609,16 +657,30 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         ++chunk;
       }
       if (!ok) break;
-      if (m < T.mend) {
+      // Epilogue through this warp's staging buffer, epi_cols columns at a time: each lane
+      // writes its row's BF16 values as 16-byte chunks XOR-swizzled by row (conflict-free),
+      // then CPR lanes per row store the row's contiguous bytes (128 B for 64 columns),
+      // 32 / CPR rows per instruction.
+      constexpr int EC = S::epi_cols, CPR = EC / 8, RPI = 32 / CPR;
+      auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
+      uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
 #pragma unroll
-        for (int jj = 0; jj < 8; ++jj) {
-          const int n = ncol0 + 8 * jj;
-          if (n < p.N) {
-            const float v[8] = {acc[4 * jj].x,     acc[4 * jj].y,     acc[4 * jj + 1].x, acc[4 * jj + 1].y,
-                                acc[4 * jj + 2].x, acc[4 * jj + 2].y, acc[4 * jj + 3].x, acc[4 * jj + 3].y};
-            store8(p, m, n, v);
-          }
+      for (int h = 0; h < 64 / EC; ++h) {
+#pragma unroll
+        for (int c = 0; c < CPR; ++c) {
+          const float2* a4 = acc + h * (EC / 2) + c * 4;
+          stg[lane * CPR + (c ^ swz(lane))] = make_uint4(pack_bf16(a4[0].x, a4[0].y), pack_bf16(a4[1].x, a4[1].y),
+                                                         pack_bf16(a4[2].x, a4[2].y), pack_bf16(a4[3].x, a4[3].y));
         }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < CPR; ++i) {
+          const int r = i * RPI + lane / CPR, c = lane % CPR;
+          const uint4 v = stg[r * CPR + (c ^ swz(r))];
+          const int mr = T.m0 + q * 32 + r, n = ncol0 + h * EC + c * 8;
+          if (mr < T.mend && n < p.N) store8_bf16(p, mr, n, v);
+        }
+        __syncwarp();
       }
     }
   }
