@@ -83,46 +83,31 @@ __device__ __forceinline__ float pow2_neg(int e) {
 }
 
 // ------------------------------------------------------------------ E2M1
-// Magnitude grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}; code index = grid index.
-__device__ __forceinline__ int e2m1_floor_index(float a) {   // largest i with grid[i] <= a (a < 6)
-  return (a >= 0.5f) + (a >= 1.0f) + (a >= 1.5f) + (a >= 2.0f) + (a >= 3.0f) + (a >= 4.0f);
-}
-__device__ __forceinline__ float e2m1_grid(int i) {
-  // 0, .5, 1, 1.5, 2, 3, 4, 6
-  return (i < 4) ? 0.5f * (float)i : (i == 4 ? 2.0f : (i == 5 ? 3.0f : (i == 6 ? 4.0f : 6.0f)));
-}
-
-// Round to nearest, ties to the even code, saturating at 6.  Returns the 4-bit code.
-__device__ __forceinline__ uint32_t e2m1_rne(float y) {
-  float a = fabsf(y);
-  uint32_t code;
-  if (a >= 6.0f) {
-    code = 7;
-  } else {
-    int i = e2m1_floor_index(a);
-    float mid = 0.5f * (e2m1_grid(i) + e2m1_grid(i + 1));       // exact grid midpoint
-    bool up = (a > mid) || (a == mid && (i & 1));
-    code = (uint32_t)(i + (up ? 1 : 0));
-  }
-  return code | ((__float_as_uint(y) >> 28) & 8u);
-}
-
+// Magnitude grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}; code index = grid index, bit 3 = sign.
 // Stochastic rounding with one 32-bit random word: up iff (word >> 8) * 2^-24 < p,
-// p = (|y| - lo) / (hi - lo) (exact: the gaps are powers of two).
+// p = (|y| - lo) / (hi - lo).  The gaps of the E2M1 grid are powers of two, so p is a
+// fixed-point fraction of |y|'s own mantissa bits and the decision is an exact integer
+// compare against the 24-bit random value u24 = word >> 8:
+//   |y| in [1, 6):   lo has |y|'s exponent and top mantissa bit, p = (low 22 bits) / 2^22,
+//                    floor code = 2 + 2*(exponent) + top bit = (bits >> 22) - 252;
+//   |y| in [0.5, 1): lo = 0.5, gap 0.5, p = (23 mantissa bits) / 2^23, floor code 1;
+//   |y| < 0.5:       lo = 0, gap 0.5, p = 2|y| (compared in FP32, exact), floor code 0;
+//   |y| >= 6:        code 7 (saturation, no rounding).
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t word) {
-  float a = fabsf(y);
-  uint32_t code;
-  if (a >= 6.0f) {
-    code = 7;
-  } else {
-    int i = e2m1_floor_index(a);
-    float lo = e2m1_grid(i);
-    float inv_gap = (i < 4) ? 2.0f : (i < 6 ? 1.0f : 0.5f);
-    float p = (a - lo) * inv_gap;
-    float u = (float)(word >> 8) * 5.9604644775390625e-08f;   // 2^-24
-    code = (uint32_t)(i + (u < p ? 1 : 0));
-  }
-  return code | ((__float_as_uint(y) >> 28) & 8u);
+  const uint32_t b = __float_as_uint(y), ab = b & 0x7FFFFFFFu, u24 = word >> 8;
+  const uint32_t c_hi = (ab >> 22) - 252u + (u24 < ((ab & 0x3FFFFFu) << 2) ? 1u : 0u);
+  const uint32_t c_mid = 1u + (u24 < ((ab & 0x7FFFFFu) << 1) ? 1u : 0u);
+  const uint32_t c_lo = (__fmul_rn((float)u24, 5.9604644775390625e-08f) < __fmul_rn(__uint_as_float(ab), 2.0f)) ? 1u : 0u;
+  const uint32_t code = ab >= 0x40C00000u ? 7u : ab >= 0x3F800000u ? c_hi : ab >= 0x3F000000u ? c_mid : c_lo;
+  return code | ((b >> 28) & 8u);
+}
+
+// Two values to E2M1 by round-to-nearest-even with saturation at 6 (hardware conversion):
+// returns (code(hi) << 4) | code(lo).
+__device__ __forceinline__ uint32_t e2m1x2_rne(float hi, float lo) {
+  uint32_t r;
+  asm("{\n\t.reg .b8 t;\n\tcvt.rn.satfinite.e2m1x2.f32 t, %1, %2;\n\tcvt.u32.u8 %0, t;\n\t}" : "=r"(r) : "f"(hi), "f"(lo));
+  return r & 0xFFu;
 }
 
 // ------------------------------------------------------------------ Philox4x32-10

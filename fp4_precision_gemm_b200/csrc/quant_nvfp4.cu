@@ -93,11 +93,18 @@ __device__ __forceinline__ float global_scale(uint32_t amax_bits) {
   return (s > FLT_MAX) ? FLT_MAX : s;
 }
 
-// E4M3 block scale and the matching encode scale for block amax `m`.
-__device__ __forceinline__ void block_scale(float m, float S_g, uint32_t& sb, float& enc) {
+// E4M3 block scale and the matching encode scale S_g / decode(sb) for block amax `m`; the
+// encode scales of all 128 non-negative codes are tabulated once per CTA (enc_tab).
+__device__ __forceinline__ void block_scale(float m, float S_g, const float* enc_tab, uint32_t& sb, float& enc) {
   const float t = __fmul_rn(__fdiv_rn(m, 6.0f), S_g);
   sb = cvt_e4m3x2(t, 0.0f) & 0xFFu;
-  enc = (sb == 0) ? 0.0f : __fdiv_rn(S_g, e4m3_to_float(sb));
+  enc = enc_tab[sb & 0x7Fu];
+}
+
+// enc_tab[c] = S_g / decode(c) for codes 1..126 (code 0: 0, no value is encoded).
+__device__ __forceinline__ void fill_enc_tab(float* enc_tab, float S_g) {
+  const int c = threadIdx.x & 127;
+  enc_tab[c] = (c == 0 || c == 0x7F) ? 0.0f : __fdiv_rn(S_g, e4m3_to_float((uint32_t)c));
 }
 
 __device__ __forceinline__ uint32_t rht_signs(const Fp4QuantParams& P) {
@@ -151,7 +158,7 @@ __device__ __forceinline__ void block_max_atomic(float m, uint32_t* dst) {
 }  // namespace
 
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256) fp4_amax_kernel(const __grid_constant__ Fp4QuantParams P) {
+__global__ void __launch_bounds__(256, 3) fp4_amax_kernel(const __grid_constant__ Fp4QuantParams P) {
   const Tile T = tile_coords(P);
   float x[16][4];
   load16x4(P, T, x);
@@ -194,12 +201,16 @@ __global__ void __launch_bounds__(256) fp4_amax_kernel(const __grid_constant__ F
 }
 
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
+__global__ void __launch_bounds__(256, (ROW && COL) ? 2 : 3) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
   __shared__ __align__(16) uint8_t tq[COL ? 128 * 64 : 16];
+  __shared__ float enc_tab[2][128];
   const Tile T = tile_coords(P);
   float x[16][4];
   load16x4(P, T, x);
   const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
+  if (ROW && threadIdx.x < 128) fill_enc_tab(enc_tab[0], global_scale(P.amax_bits[0]));
+  if (COL && threadIdx.x >= 128) fill_enc_tab(enc_tab[1], global_scale(P.amax_bits[1]));
+  __syncthreads();
 
   if (ROW) {
     const float S_g = global_scale(P.amax_bits[0]);
@@ -215,7 +226,7 @@ __global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ 
       m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       uint32_t sb;
       float enc;
-      block_scale(m, S_g, sb, enc);
+      block_scale(m, S_g, enc_tab[0], sb, enc);
       uint32_t codes = 0;
       if (P.sr_row) {
         const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
@@ -224,8 +235,8 @@ __global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ 
         codes = e2m1_sr(__fmul_rn(e[0], enc), r.x) | (e2m1_sr(__fmul_rn(e[1], enc), r.y) << 4) |
                 (e2m1_sr(__fmul_rn(e[2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[3], enc), r.w) << 12);
       } else {
-        codes = e2m1_rne(__fmul_rn(e[0], enc)) | (e2m1_rne(__fmul_rn(e[1], enc)) << 4) |
-                (e2m1_rne(__fmul_rn(e[2], enc)) << 8) | (e2m1_rne(__fmul_rn(e[3], enc)) << 12);
+        codes = e2m1x2_rne(__fmul_rn(e[1], enc), __fmul_rn(e[0], enc)) |
+                (e2m1x2_rne(__fmul_rn(e[3], enc), __fmul_rn(e[2], enc)) << 8);
       }
       if (row < P.rows && T.cok) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)codes;
       if ((T.lane & 3) == 0) {
@@ -256,7 +267,7 @@ __global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ 
       for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
       uint32_t sb;
       float enc;
-      block_scale(m, S_g, sb, enc);
+      block_scale(m, S_g, enc_tab[1], sb, enc);
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -269,8 +280,8 @@ __global__ void __launch_bounds__(256) fp4_quant_kernel(const __grid_constant__ 
                (e2m1_sr(__fmul_rn(e[4 * q + 2], enc), r.z) << 8) |
                (e2m1_sr(__fmul_rn(e[4 * q + 3], enc), r.w) << 12);
         } else {
-          c4 = e2m1_rne(__fmul_rn(e[4 * q], enc)) | (e2m1_rne(__fmul_rn(e[4 * q + 1], enc)) << 4) |
-               (e2m1_rne(__fmul_rn(e[4 * q + 2], enc)) << 8) | (e2m1_rne(__fmul_rn(e[4 * q + 3], enc)) << 12);
+          c4 = e2m1x2_rne(__fmul_rn(e[4 * q + 1], enc), __fmul_rn(e[4 * q], enc)) |
+               (e2m1x2_rne(__fmul_rn(e[4 * q + 3], enc), __fmul_rn(e[4 * q + 2], enc)) << 8);
         }
         if (q < 2) lo |= c4 << (16 * q);
         else hi |= c4 << (16 * (q - 2));

@@ -42,8 +42,13 @@ __device__ __forceinline__ int tq_chunk(int c, int k) { return k ^ ((c >> 3) ^ (
 
 }  // namespace
 
+// Resident CTAs per SM: the kernel is latency bound on its loads, so the register budget is
+// set for 4 CTAs (64 registers); the rowwise-only variants need a few more and get 3.
+template <bool ROW, bool COL>
+constexpr int kTileQuantCtas = (ROW && !COL) ? 3 : 4;
+
 template <int MODE, bool ROW, bool COL>
-__global__ void __launch_bounds__(256, 2) tile_quant_kernel(const __grid_constant__ TileQuantParams P) {
+__global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kernel(const __grid_constant__ TileQuantParams P) {
   __shared__ uint32_t red[8][64];
   __shared__ float colsf[128];
   __shared__ uint8_t colexp[128 * 4];
