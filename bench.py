@@ -78,12 +78,11 @@ class LlamaStep:
 
     def __init__(self, fq, rank, M=8192, K=4096, N=14336):
         self.fq, self.M, self.K, self.N = fq, M, K, N
+        self.workload = f"llama3-8b up-proj blockwise fwd+bwd: X {M}x{K}, W {K}x{N}, dY {M}x{N}"
         d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
         if rank:   # other ranks: their own tokens, the same weights
-            g = workloads.llama8b(device="cuda", M=M, K=K, N=N)
             d["X"] = workloads.normal_bf16((M, K), 1.0, 10_000 + rank, 1e-3, 50.0, "cuda")
             d["dY"] = workloads.normal_bf16((M, N), 1e-3, 20_000 + rank, device="cuda")
-            del g
         self.X, self.W, self.dY = d["X"], d["W"], d["dY"]
         dev = self.X.device
         u8, f32 = torch.uint8, torch.float32
@@ -499,7 +498,7 @@ def run_ours(args, rank, world, local_rank):
     import fp4_precision_gemm_b200 as fq
     torch.cuda.set_device(local_rank)
     fq.lib()
-    step = STEPS[args.workload](fq, rank)
+    step = STEPS[args.workload](fq, rank, **({"M": args.tokens} if args.tokens else {}))
     launches = step.launches()
     n_launch = getattr(step, "launch_count", lambda: len(launches))()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -577,7 +576,7 @@ def run_ours(args, rank, world, local_rank):
         ach = f["bytes"] / (f["ms"] * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 3), "traffic": None, "peak_source": f"{src}: hbm_gbs"}
-    roof["traffic"] = traffic_for(dom, args.workload)
+    roof["traffic"] = traffic_for(dom, args.workload) if not args.tokens else None
 
     e2e = measure_e2e(step, launches, stream, args) if (not args.no_e2e) else None
     value = world * step.gemm_flop / (ms * 1e-3) / 1e12
@@ -689,8 +688,12 @@ def main():
     ap.add_argument("--workload", choices=sorted(STEPS) + ["all"], default="llama8b")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--tokens", type=int, default=None,
+                    help="llama8b only: token count M (default 8192); smaller cases for profiler captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
+    if args.tokens and args.workload != "llama8b":
+        ap.error("--tokens applies to the llama8b workload only")
 
     world = int(os.environ.get("WORLD_SIZE", "1"))
     rank = int(os.environ.get("RANK", "0"))

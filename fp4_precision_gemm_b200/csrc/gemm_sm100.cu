@@ -33,7 +33,7 @@ using namespace sm100;
 namespace {
 
 constexpr int kBM = 128, kBKB = 128;  // tile rows, K bytes per stage
-constexpr int kGroupM = 16;           // rasterization: 16 row tiles share each column sweep
+constexpr int kGroupM = 16;           // rasterization of grouped (expert) GEMMs
 constexpr int kMaxGroups = 256;
 constexpr uint64_t kWaitLimitNs = 4000000000ull;
 constexpr uint32_t kAStage = kBM * kBKB;  // 16 KB
@@ -45,13 +45,13 @@ struct Tile {
   int m0, mend, n0, g;
 };
 
-// Tile t of the rasterized order (groups of kGroupM row tiles, column-major inside a group)
+// Tile t of the rasterized order (groups of p.group_m row tiles, column-major inside a group)
 // for output tiles `bn` columns wide.  Grouped GEMMs enumerate each expert's row tiles.
 __device__ __forceinline__ Tile tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
                                         const int* offs, int bn) {
-  const int per = kGroupM * p.tiles_n;
-  const int grp = t / per, first = grp * kGroupM;
-  const int gsz = min(row_tiles - first, kGroupM);
+  const int per = p.group_m * p.tiles_n;
+  const int grp = t / per, first = grp * p.group_m;
+  const int gsz = min(row_tiles - first, p.group_m);
   const int local = t - grp * per;
   const int rt = first + local % gsz, nt = local / gsz;
   Tile T;
@@ -390,9 +390,9 @@ struct BwSmem {
 // expert's 256-row tiles.  Returns this CTA's 128-row half.
 __device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
                                              const int* offs, uint32_t rank) {
-  const int per = kGroupM * p.tiles_n;
-  const int grp = t / per, first = grp * kGroupM;
-  const int gsz = min(row_tiles - first, kGroupM);
+  const int per = p.group_m * p.tiles_n;
+  const int grp = t / per, first = grp * p.group_m;
+  const int gsz = min(row_tiles - first, p.group_m);
   const int local = t - grp * per;
   const int rt = first + local % gsz, nt = local / gsz;
   Tile T;
@@ -694,6 +694,21 @@ __global__ void __launch_bounds__(kBwThreads, 1)
   }
 }
 
+// Raster group (row tiles per column sweep).  Concurrent tiles should share operands in L2
+// and the operand that is re-read across sweeps should stay resident: when A is the
+// smaller operand (M <= N) a group spans all row tiles (A stays resident, B streams through
+// once), capped at about 40 MB of A; otherwise tiles go row-major (group of one row tile),
+// so each row band of A streams through once against a resident B.  Grouped (expert)
+// GEMMs keep groups of kGroupM row tiles.
+static int raster_group(const GemmParams& p, int row_tiles, int tile_m) {
+  if (p.num_groups > 0) return kGroupM;
+  if (p.M > p.N) return 1;
+  const int64_t slab = (int64_t)tile_m * (p.recipe == kNvfp4 ? p.K / 2 : p.K);   // bytes of A per row tile
+  int64_t g = (40ll << 20) / (slab > 0 ? slab : 1);
+  if (g < 1) g = 1;
+  return (int)(g < row_tiles ? g : row_tiles);
+}
+
 template <int L, bool G>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
@@ -704,6 +719,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   GemmParams q = p;
   q.tiles_n = (p.N + kBwBN - 1) / kBwBN;
   q.tiles_m = G ? (p.M + kBwPairM - 1) / kBwPairM + p.num_groups : (p.M + kBwPairM - 1) / kBwPairM;
+  q.group_m = raster_group(q, q.tiles_m, kBwPairM);
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
@@ -737,6 +753,7 @@ static cudaError_t launch_scaled(const GemmParams& p, const CUtensorMap& a, cons
   if (e != cudaSuccess) return e;
   GemmParams q = p;
   q.tiles_n = (p.N + kBN - 1) / kBN;
+  q.group_m = raster_group(q, q.tiles_m, kBM);
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   int grid = (int)(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;

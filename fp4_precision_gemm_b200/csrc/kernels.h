@@ -73,6 +73,7 @@ struct GemmParams {
   const int32_t* m_offsets;
   int num_groups;
   int tiles_m, tiles_n;    // output tile grid (non-grouped)
+  int group_m;             // raster: row tiles per column sweep (set by the launcher)
   uint32_t* status;        // device status word
 };
 
