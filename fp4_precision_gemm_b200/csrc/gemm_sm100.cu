@@ -81,19 +81,6 @@ __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
 }
 
 // Stores 8 consecutive results of row m starting at column n (masking the N tail).
-__device__ __forceinline__ void store8(const GemmParams& p, int m, int n, const float* v) {
-  uint16_t* dst = p.c + (int64_t)m * p.ldc + n;
-  if (n + 8 <= p.N) {
-    *reinterpret_cast<uint4*>(dst) = make_uint4(pack_bf16(v[0], v[1]), pack_bf16(v[2], v[3]),
-                                                pack_bf16(v[4], v[5]), pack_bf16(v[6], v[7]));
-  } else {
-    for (int i = 0; i < 8 && n + i < p.N; ++i) {
-      __nv_bfloat16 h = __float2bfloat16_rn(v[i]);
-      dst[i] = *reinterpret_cast<uint16_t*>(&h);
-    }
-  }
-}
-
 // Eight packed BF16 values at (m, n..n+7); scalar stores past column N.
 __device__ __forceinline__ void store8_bf16(const GemmParams& p, int m, int n, uint4 v) {
   uint16_t* dst = p.c + (int64_t)m * p.ldc + n;
@@ -105,24 +92,15 @@ __device__ __forceinline__ void store8_bf16(const GemmParams& p, int m, int n, u
   }
 }
 
-// Expert offsets and the running count of row tiles per expert, into shared memory.
-__device__ __forceinline__ void load_groups(const GemmParams& p, int* prefix, int* offs, int lane) {
-  for (int g = lane; g <= p.num_groups; g += 32) offs[g] = p.m_offsets[g];
-  __syncwarp();
-  if (lane == 0) {
-    int acc = 0;
-    for (int g = 0; g < p.num_groups; ++g) {
-      prefix[g] = acc;
-      acc += (offs[g + 1] - offs[g] + kBM - 1) / kBM;
-    }
-    prefix[p.num_groups] = acc;
-  }
-}
 
 // ------------------------------------------------------------------ hardware-scaled kernel
-// MXFP8, NVFP4 and per-tensor: 128 x 256 output tiles accumulated across all of K in one
-// TMEM buffer (256 columns); the scale factors of MX / NVFP4 stages are copied from shared
-// memory into TMEM with tcgen05.cp and consumed by the block-scaled MMA.
+// MXFP8, NVFP4 and per-tensor: 128 x 256 output tiles accumulated across all of K in TMEM
+// (256 columns per accumulator); the scale factors of MX / NVFP4 stages are copied from
+// shared memory into TMEM with tcgen05.cp and consumed by the block-scaled MMA.  Per-tensor
+// has no scale columns, so it keeps two accumulators and the epilogue of one tile overlaps
+// the MMAs of the next; MX / NVFP4 drain their single accumulator before the next tile.
+// The epilogue stages BF16 rows through shared memory (width per recipe, as shared memory
+// allows) so global stores are contiguous row segments.
 constexpr int kBN = 256;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
@@ -131,9 +109,15 @@ constexpr int kThreads = 320;
 constexpr uint32_t kBStage = kBN * kBKB;  // 32 KB
 
 template <int R> struct Cfg;
-template <> struct Cfg<kPerTensor> { static constexpr uint32_t sfa = 0, sfb = 0, tmem_cols = 256; };
-template <> struct Cfg<kMx> { static constexpr uint32_t sfa = 512, sfb = 1024, tmem_cols = 512, sf_cols = 16; };
-template <> struct Cfg<kNvfp4> { static constexpr uint32_t sfa = 2048, sfb = 4096, tmem_cols = 512, sf_cols = 64; };
+template <> struct Cfg<kPerTensor> {
+  static constexpr uint32_t sfa = 0, sfb = 0, tmem_cols = 512, acc_bufs = 2, epi_cols = 64;
+};
+template <> struct Cfg<kMx> {
+  static constexpr uint32_t sfa = 512, sfb = 1024, tmem_cols = 512, sf_cols = 16, acc_bufs = 1, epi_cols = 32;
+};
+template <> struct Cfg<kNvfp4> {
+  static constexpr uint32_t sfa = 2048, sfb = 4096, tmem_cols = 512, sf_cols = 64, acc_bufs = 1, epi_cols = 16;
+};
 
 template <int R>
 struct Smem {
@@ -141,11 +125,38 @@ struct Smem {
   static constexpr uint32_t b = a + kStages * kAStage;
   static constexpr uint32_t sf = b + kStages * kBStage;
   static constexpr uint32_t sf_stage = Cfg<R>::sfa + Cfg<R>::sfb;
-  static constexpr uint32_t bars = sf + kStages * sf_stage;
-  static constexpr uint32_t n_bars = 2 * kStages + 3;
+  static constexpr uint32_t stage_c = 32 * Cfg<R>::epi_cols * 2;   // per epilogue warp
+  static constexpr uint32_t cst = sf + kStages * sf_stage;
+  static constexpr uint32_t bars = cst + kEpiWarps * stage_c;
+  static constexpr uint32_t n_bars = 2 * kStages + 2 * Cfg<R>::acc_bufs + 1;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t alloc = misc + 16 + 1024;  // + room to align the base to 1024 bytes
+  static_assert(alloc <= 227 * 1024, "shared memory");
 };
+
+// Epilogue store of one warp's 32 rows x EC columns (values already scaled, FP32 in `v`,
+// lane = row): BF16 rows into the warp's staging buffer (16-byte chunks XOR-swizzled by row,
+// bank-conflict free), then CPR = EC / 8 lanes per row store contiguous 16-byte chunks.
+template <int EC>
+__device__ __forceinline__ void stage_store_rows(uint4* stg, const float* v, const GemmParams& p, int row0,
+                                                 int mend, int n0, int lane) {
+  constexpr int CPR = EC / 8, RPI = 32 / CPR, SH = CPR == 8 ? 0 : (CPR == 4 ? 1 : 2);
+#pragma unroll
+  for (int c = 0; c < CPR; ++c) {
+    const float* a = v + 8 * c;
+    stg[lane * CPR + (c ^ ((lane >> SH) & (CPR - 1)))] =
+        make_uint4(pack_bf16(a[0], a[1]), pack_bf16(a[2], a[3]), pack_bf16(a[4], a[5]), pack_bf16(a[6], a[7]));
+  }
+  __syncwarp();
+#pragma unroll
+  for (int i = 0; i < CPR; ++i) {
+    const int r = i * RPI + lane / CPR, c = lane % CPR;
+    const uint4 w = stg[r * CPR + (c ^ ((r >> SH) & (CPR - 1)))];
+    const int m = row0 + r, n = n0 + c * 8;
+    if (m < mend && n < p.N) store8_bf16(p, m, n, w);
+  }
+  __syncwarp();
+}
 
 }  // namespace
 
@@ -158,9 +169,10 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars);
   uint64_t* empty = full + kStages;
-  uint64_t* accfull = empty + kStages;   // the tile's accumulator is complete
-  uint64_t* accempty = accfull + 1;      // the epilogue has drained it
-  uint64_t* final_bar = accempty + 1;    // MMA wind-down
+  constexpr uint32_t kAcc = Cfg<R>::acc_bufs;
+  uint64_t* accfull = empty + kStages;   // [kAcc] the tile's accumulator is complete
+  uint64_t* accempty = accfull + kAcc;   // [kAcc] the epilogue has drained it
+  uint64_t* final_bar = accempty + kAcc; // MMA wind-down
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::misc + 4);
 
@@ -172,8 +184,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[i], 1);
       mbar_init(&empty[i], 1);
     }
-    mbar_init(accfull, 1);
-    mbar_init(accempty, kEpiWarps);  // one arrival per epilogue warp
+    for (uint32_t b = 0; b < kAcc; ++b) {
+      mbar_init(&accfull[b], 1);
+      mbar_init(&accempty[b], kEpiWarps);  // one arrival per epilogue warp
+    }
     mbar_init(final_bar, 1);
     *abort_flag = 0;
     fence_barrier_init();
@@ -238,7 +252,8 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t it = 0, tiles_done = 0;
       bool ok = true;
       for (int t = blockIdx.x; t < total && ok; t += gridDim.x, ++tiles_done) {
-        if (!mbar_wait(accempty, (tiles_done & 1) ^ 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); break; }
+        const uint32_t ab = tiles_done % kAcc, acc_t = tmem + ab * (uint32_t)kBN;
+        if (!mbar_wait(&accempty[ab], ((tiles_done / kAcc) & 1) ^ 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); break; }
         tc_fence_after();
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
@@ -248,7 +263,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           const uint64_t bdesc = smem_desc(smem_u32(smem + S::b + s * kBStage), 16, 1024, 2);
           if constexpr (R == kPerTensor) {
 #pragma unroll
-            for (int k = 0; k < 4; ++k) mma_f8f6f4(tmem, adesc + 2 * k, bdesc + 2 * k, idesc_dense, kb > 0 || k > 0);
+            for (int k = 0; k < 4; ++k) mma_f8f6f4(acc_t, adesc + 2 * k, bdesc + 2 * k, idesc_dense, kb > 0 || k > 0);
           } else {
             const uint32_t sf_col = kBN + s * Cfg<R>::sf_cols;  // this stage's scale columns
             const uint32_t sfa_t = tmem + sf_col;
@@ -280,7 +295,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&empty[s]);
         }
         if (!ok) break;
-        mma_commit(accfull);
+        mma_commit(&accfull[ab]);
       }
       // wind down: all MMAs this thread issued complete before TMEM is released
       mma_commit(final_bar);
@@ -288,40 +303,35 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps 0-7
+    constexpr int EC = (int)Cfg<R>::epi_cols;
     const int q = warp & 3, wg = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(wg * 128);
-    const int rloc = q * 32 + lane;
+    uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
     uint32_t tiles_done = 0;
     float alpha = 1.0f;
     if (R == kPerTensor || R == kNvfp4) alpha = __fmul_rn(*p.a_global, *p.b_global);
     for (int t = blockIdx.x; t < total; t += gridDim.x, ++tiles_done) {
       const Tile T = tile_of(t, p, p.tiles_m, nullptr, nullptr, kBN);
-      const int m = T.m0 + rloc;
-      const bool row_ok = m < T.mend;
+      const uint32_t ab = tiles_done % kAcc;
       const int ncol0 = T.n0 + wg * 128;
-      if (!mbar_wait(accfull, tiles_done & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); break; }
+      if (!mbar_wait(&accfull[ab], (tiles_done / kAcc) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); break; }
       tc_fence_after();
 #pragma unroll 1
-      for (int c = 0; c < 4; ++c) {
-        uint32_t r[32];
-        tmem_ld_32x32b_x32(t_lane + c * 32, r);
-        tmem_ld_wait(r);
-        if (row_ok) {
+      for (int c = 0; c < 128 / EC; ++c) {
+        float v[EC];
 #pragma unroll
-          for (int j = 0; j < 4; ++j) {
-            const int n = ncol0 + c * 32 + 8 * j;
-            if (n < p.N) {
-              float v[8];
+        for (int h = 0; h < EC / 16; ++h) {
+          uint32_t r[16];
+          tmem_ld_32x32b_x16(t_lane + ab * (uint32_t)kBN + c * EC + h * 16, r);
+          tmem_ld_wait(r);
 #pragma unroll
-              for (int i = 0; i < 8; ++i) v[i] = __fmul_rn(__uint_as_float(r[8 * j + i]), alpha);
-              store8(p, m, n, v);
-            }
-          }
+          for (int i = 0; i < 16; ++i) v[h * 16 + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
         }
+        stage_store_rows<EC>(stg, v, p, T.m0 + q * 32, T.mend, ncol0 + c * EC, lane);
       }
       tc_fence_before();
       __syncwarp();
-      if (lane == 0) mbar_arrive_relaxed(accempty);
+      if (lane == 0) mbar_arrive_relaxed(&accempty[ab]);
     }
   }
 
@@ -602,7 +612,6 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
       const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
-      const int m = T.m0 + rloc;
       const int ncol0 = T.n0 + cgp * 64;
       float2 acc[32];
 #pragma unroll
