@@ -201,7 +201,7 @@ __global__ void __launch_bounds__(256, 3) fp4_amax_kernel(const __grid_constant_
 }
 
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256, (ROW && COL) ? 2 : 3) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
+__global__ void __launch_bounds__(256, 3) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
   __shared__ __align__(16) uint8_t tq[COL ? 128 * 64 : 16];
   __shared__ float enc_tab[2][128];
   const Tile T = tile_coords(P);
