@@ -319,19 +319,115 @@ __global__ void __launch_bounds__(256, 3) fp4_quant_kernel(const __grid_constant
   }
 }
 
+// ------------------------------------------------------------------ rowwise-only path
+// When only the rowwise output is requested, one thread owns one 16-element group of a row
+// (two 16-byte loads): the group's transform, amax, scale and codes stay in-thread and a warp
+// reads 1 KB of a row per instruction pair.  The butterflies run in the same stage order as
+// the tiled kernels, so every value is identical.  With the MMA-tiled scale layout the
+// threads also cover the image's padding (rows up to a multiple of 128, scale columns up to
+// a multiple of 4), writing scale code 0 there.
+__device__ __forceinline__ void load_group16(const Fp4QuantParams& P, int64_t row, int64_t c, float (&e)[16]) {
+  const uint16_t* src = P.x + row * P.ld_x + c;
+  const uint4 a = ldg_nc_v4(src), b = ldg_nc_v4(src + 8);
+  const uint32_t w[8] = {a.x, a.y, a.z, a.w, b.x, b.y, b.z, b.w};
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    e[2 * i] = bf16_lo(w[i]);
+    e[2 * i + 1] = bf16_hi(w[i]);
+  }
+}
+
+__device__ __forceinline__ void rht16_inthread(float (&e)[16], uint32_t signs) {
+#pragma unroll
+  for (int i = 0; i < 16; ++i) e[i] = flip(e[i], signs, i);
+  fwht16(e);
+}
+
+__global__ void __launch_bounds__(256) fp4_amax_row_kernel(const __grid_constant__ Fp4QuantParams P) {
+  const int64_t ng = P.cols >> 4;
+  const int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  float m = 0.0f;
+  if (g < P.rows * ng) {
+    float e[16];
+    load_group16(P, g / ng, (g % ng) * 16, e);
+    if (P.rht_row) rht16_inthread(e, rht_signs(P));
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+  }
+  block_max_atomic(m, P.amax_bits);
+}
+
+__global__ void __launch_bounds__(256) fp4_quant_row_kernel(const __grid_constant__ Fp4QuantParams P) {
+  __shared__ float enc_tab[128];
+  const float S_g = global_scale(P.amax_bits[0]);
+  if (threadIdx.x < 128) fill_enc_tab(enc_tab, S_g);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_row = __frcp_rn(S_g);
+  __syncthreads();
+  const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
+  const int64_t kdom = P.sf_tiled ? s4 * 4 : nsf;
+  const int64_t rdom = P.sf_tiled ? (P.rows + 127) / 128 * 128 : P.rows;
+  const int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  if (g >= rdom * kdom) return;
+  const int64_t row = g / kdom, kc = g % kdom;
+  uint32_t sb = 0;
+  if (row < P.rows && kc < nsf) {
+    const int64_t c = kc * 16;
+    float e[16];
+    load_group16(P, row, c, e);
+    if (P.rht_row) rht16_inthread(e, rht_signs(P));
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+    float enc;
+    block_scale(m, S_g, enc_tab, sb, enc);
+    uint32_t w[2];
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      uint32_t codes = 0;
+#pragma unroll
+      for (int q = 0; q < 2; ++q) {
+        const int j = 8 * h + 4 * q;
+        uint32_t c4;
+        if (P.sr_row) {
+          const uint64_t blk = (uint64_t)(row * P.cols + c + j) >> 2;
+          const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
+          c4 = e2m1_sr(__fmul_rn(e[j], enc), r.x) | (e2m1_sr(__fmul_rn(e[j + 1], enc), r.y) << 4) |
+               (e2m1_sr(__fmul_rn(e[j + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[j + 3], enc), r.w) << 12);
+        } else {
+          c4 = e2m1x2_rne(__fmul_rn(e[j + 1], enc), __fmul_rn(e[j], enc)) |
+               (e2m1x2_rne(__fmul_rn(e[j + 3], enc), __fmul_rn(e[j + 2], enc)) << 8);
+        }
+        codes |= c4 << (16 * q);
+      }
+      w[h] = codes;
+    }
+    *(uint2*)(P.q_row + row * (P.cols >> 1) + (c >> 1)) = make_uint2(w[0], w[1]);
+  }
+  if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+  else P.sf_row[row * nsf + kc] = (uint8_t)sb;
+}
+
+static unsigned blocks_for(int64_t threads) { return (unsigned)((threads + 255) / 256); }
+
 cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
   const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
   if (row && col) fp4_amax_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
-  else if (row) fp4_amax_kernel<true, false><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else if (row) fp4_amax_row_kernel<<<blocks_for(p.rows * (p.cols >> 4)), 256, 0, s>>>(p);
   else fp4_amax_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
   const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
-  if (row && col) fp4_quant_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
-  else if (row) fp4_quant_kernel<true, false><<<(unsigned)tiles, 256, 0, s>>>(p);
-  else fp4_quant_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  if (row && col) {
+    fp4_quant_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  } else if (row) {
+    const int64_t nsf = p.cols >> 4, kdom = p.sf_tiled ? (nsf + 3) / 4 * 4 : nsf;
+    const int64_t rdom = p.sf_tiled ? (p.rows + 127) / 128 * 128 : p.rows;
+    fp4_quant_row_kernel<<<blocks_for(rdom * kdom), 256, 0, s>>>(p);
+  } else {
+    fp4_quant_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -50,6 +50,28 @@ def test_blockwise_fprop(cuda_lib, M, K, N):
     check(c, ref, t, "fprop")
 
 
+def test_tiny_config_end_to_end(cuda_lib):
+    """The tiny blockwise configuration exactly as specified (A 256x512 N(0,1) with 0.1% x100
+    outliers, B 512x256 N(0,0.02), seed 0): quantized codes and scales bit-exact, and every
+    element of C = A.B within the tolerance."""
+    fq = cuda_lib
+    d = workloads.tiny()
+    A, B = d["A"], d["B"]
+    qa = fq.quantize_1x128(A.cuda())
+    qb = fq.quantize_128x128(B.cuda())
+    c = fq.gemm(qa["q_row"], qb["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qa["s_row"], b_scale=qb["s"])
+    assert fq.device_status() == 0
+    oa, osa = Q.quantize_1x128_rowwise(workloads.bf16_bits(A))
+    _, obt, osb = Q.quantize_128x128(workloads.bf16_bits(B))
+    assert np.array_equal(host(qa["q_row"]), oa)
+    assert np.array_equal(host(qa["s_row"]).view(np.uint32), osa.astype(np.float32).view(np.uint32))
+    assert np.array_equal(host(qb["q_t"]), obt)
+    assert np.array_equal(host(qb["s"]).view(np.uint32), osb.astype(np.float32).view(np.uint32))
+    ref, t = G.reference(G.dequant_a_1x128(oa, osa), G.dequant_b_blockwise(obt, osb, G.FPROP))
+    assert c.shape == (256, 256)
+    check(c, ref, t, "tiny fprop")
+
+
 @pytest.mark.parametrize("M,Kw,Nw", [(300, 384, 512), (256, 256, 1024)])
 def test_blockwise_dgrad(cuda_lib, M, Kw, Nw):
     """dX = dY . W^T with W (Kw x Nw): GEMM N = Kw, K = Nw, B = W's K x N codes."""
