@@ -11,15 +11,17 @@
 // transform, per-16 block amax, E4M3 block scale, encode scale, and E2M1 codes by
 // round-to-nearest-even or by Philox4x32-10 stochastic rounding.
 //
-// One CTA (256 threads) handles a 128x128 tile.  Warp w owns rows 16w..16w+15, lane l
-// owns columns 4l..4l+3, so a thread holds a 16x4 sub-block:
+// Rowwise output: one thread per 16-element group of a row (two 16-byte loads); the group's
+// transform, amax and codes stay in-thread.
+// Colwise output and the two-output amax pass: one CTA (256 threads) per 128x128 tile, warp w
+// owns rows 16w..16w+15, lane l owns columns 4l..4l+3, so a thread holds a 16x4 sub-block:
 //   * colwise (along rows) 16-element groups and blocks are entirely in-thread, so the
 //     transform's butterflies and the block amax need no shuffles;
 //   * rowwise 16-element groups span 4 lanes (2 xor-shuffles for the amax, and for the
 //     two upper butterfly stages when the rowwise transform is on);
-//   * one Philox call yields the 4 words of 4 consecutive output elements in either
-//     direction.
+//   * one Philox call yields the 4 words of 4 consecutive output elements.
 // The transposed colwise codes are staged in shared memory and stored as 64-byte rows.
+// With both outputs requested the rowwise and colwise quantization run as separate kernels.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -117,12 +119,12 @@ struct Tile {
   int lane, w;
 };
 
-__device__ __forceinline__ Tile tile_coords(const Fp4QuantParams& P) {
+__device__ __forceinline__ Tile tile_coords(const Fp4QuantParams& P, int64_t tile) {
   Tile T;
   T.lane = threadIdx.x & 31;
   T.w = threadIdx.x >> 5;
-  T.r0 = (int64_t)(blockIdx.x / P.tiles_c) * 128;
-  T.c0 = (int64_t)(blockIdx.x % P.tiles_c) * 128;
+  T.r0 = (tile / P.tiles_c) * 128;
+  T.c0 = (tile % P.tiles_c) * 128;
   T.col = T.c0 + T.lane * 4;
   T.cok = T.col < P.cols;
   return T;
@@ -157,100 +159,68 @@ __device__ __forceinline__ void block_max_atomic(float m, uint32_t* dst) {
 
 }  // namespace
 
+// Grid-stride over 128x128 tiles with a bounded grid: one atomicMax per output per CTA.
 template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256, 3) fp4_amax_kernel(const __grid_constant__ Fp4QuantParams P) {
-  const Tile T = tile_coords(P);
-  float x[16][4];
-  load16x4(P, T, x);
+__global__ void __launch_bounds__(256, 3) fp4_amax_kernel(const __grid_constant__ Fp4QuantParams P, int64_t tiles) {
   const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
-  float m_plain = 0.0f;
+  float m_row = 0.0f, m_col = 0.0f;
+  for (int64_t tile = blockIdx.x; tile < tiles; tile += gridDim.x) {
+    const Tile T = tile_coords(P, tile);
+    float x[16][4];
+    load16x4(P, T, x);
+    float m_plain = 0.0f;
 #pragma unroll
-  for (int i = 0; i < 16; ++i)
+    for (int i = 0; i < 16; ++i)
 #pragma unroll
-    for (int j = 0; j < 4; ++j) m_plain = fmaxf(m_plain, fabsf(x[i][j]));
-  if (ROW) {
-    float m = m_plain;
-    if (P.rht_row) {
-      m = 0.0f;
+      for (int j = 0; j < 4; ++j) m_plain = fmaxf(m_plain, fabsf(x[i][j]));
+    if (ROW) {
+      float m = m_plain;
+      if (P.rht_row) {
+        m = 0.0f;
 #pragma unroll
-      for (int i = 0; i < 16; ++i) {
-        float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
-        rht_row4(e, signs, T.lane);
+        for (int i = 0; i < 16; ++i) {
+          float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
+          rht_row4(e, signs, T.lane);
 #pragma unroll
-        for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(e[j]));
-      }
-    }
-    block_max_atomic(m, P.amax_bits);
-  }
-  if (COL) {
-    float m = m_plain;
-    if (P.rht_col) {
-      m = 0.0f;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) {
-        float e[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) e[i] = flip(x[i][j], signs, i);
-        fwht16(e);
-#pragma unroll
-        for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
-      }
-    }
-    block_max_atomic(m, P.amax_bits + 1);
-  }
-}
-
-template <bool ROW, bool COL>
-__global__ void __launch_bounds__(256, 3) fp4_quant_kernel(const __grid_constant__ Fp4QuantParams P) {
-  __shared__ __align__(16) uint8_t tq[COL ? 128 * 64 : 16];
-  __shared__ float enc_tab[2][128];
-  const Tile T = tile_coords(P);
-  float x[16][4];
-  load16x4(P, T, x);
-  const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
-  if (ROW && threadIdx.x < 128) fill_enc_tab(enc_tab[0], global_scale(P.amax_bits[0]));
-  if (COL && threadIdx.x >= 128) fill_enc_tab(enc_tab[1], global_scale(P.amax_bits[1]));
-  __syncthreads();
-
-  if (ROW) {
-    const float S_g = global_scale(P.amax_bits[0]);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_row = __frcp_rn(S_g);
-    const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
-#pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int64_t row = T.r0 + T.w * 16 + i;
-      float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
-      if (P.rht_row) rht_row4(e, signs, T.lane);
-      float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      uint32_t sb;
-      float enc;
-      block_scale(m, S_g, enc_tab[0], sb, enc);
-      uint32_t codes = 0;
-      if (P.sr_row) {
-        const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u),
-                                      P.sr_k0, P.sr_k1);
-        codes = e2m1_sr(__fmul_rn(e[0], enc), r.x) | (e2m1_sr(__fmul_rn(e[1], enc), r.y) << 4) |
-                (e2m1_sr(__fmul_rn(e[2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[3], enc), r.w) << 12);
-      } else {
-        codes = e2m1x2_rne(__fmul_rn(e[1], enc), __fmul_rn(e[0], enc)) |
-                (e2m1x2_rne(__fmul_rn(e[3], enc), __fmul_rn(e[2], enc)) << 8);
-      }
-      if (row < P.rows && T.cok) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)codes;
-      if ((T.lane & 3) == 0) {
-        const int64_t kc = T.col >> 4;
-        if (P.sf_tiled) {
-          if (kc < s4 * 4) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
-        } else if (row < P.rows && kc < nsf) {
-          P.sf_row[row * nsf + kc] = (uint8_t)sb;
+          for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(e[j]));
         }
       }
+      m_row = fmaxf(m_row, m);
+    }
+    if (COL) {
+      float m = m_plain;
+      if (P.rht_col) {
+        m = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 4; ++j) {
+          float e[16];
+#pragma unroll
+          for (int i = 0; i < 16; ++i) e[i] = flip(x[i][j], signs, i);
+          fwht16(e);
+#pragma unroll
+          for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+        }
+      }
+      m_col = fmaxf(m_col, m);
     }
   }
+  if (ROW) block_max_atomic(m_row, P.amax_bits);
+  if (COL) block_max_atomic(m_col, P.amax_bits + 1);
+}
 
-  if (COL) {
+// Colwise output (16-element groups along rows): the 16x4-per-thread tile mapping keeps each
+// group, its transform and its block amax in-thread.
+__global__ void __launch_bounds__(256, 3) fp4_quant_col_kernel(const __grid_constant__ Fp4QuantParams P) {
+  __shared__ __align__(16) uint8_t tq[128 * 64];
+  __shared__ float enc_tab[128];
+  const Tile T = tile_coords(P, blockIdx.x);
+  float x[16][4];
+  load16x4(P, T, x);
+  const uint32_t signs = P.rht_col ? rht_signs(P) : 0u;
+  if (threadIdx.x < 128) fill_enc_tab(enc_tab, global_scale(P.amax_bits[1]));
+  __syncthreads();
+
+  {
     const float S_g = global_scale(P.amax_bits[1]);
     if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_col = __frcp_rn(S_g);
     const int64_t nsf = P.rows >> 4, s4 = (nsf + 3) >> 2;
@@ -267,7 +237,7 @@ __global__ void __launch_bounds__(256, 3) fp4_quant_kernel(const __grid_constant
       for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
       uint32_t sb;
       float enc;
-      block_scale(m, S_g, enc_tab[1], sb, enc);
+      block_scale(m, S_g, enc_tab, sb, enc);
       uint32_t lo = 0, hi = 0;
 #pragma unroll
       for (int q = 0; q < 4; ++q) {
@@ -343,14 +313,16 @@ __device__ __forceinline__ void rht16_inthread(float (&e)[16], uint32_t signs) {
   fwht16(e);
 }
 
+// Grid-stride over the groups with a bounded grid, so the per-CTA atomicMax on the single
+// amax word stays rare (one launch per group of 256 would serialize on it).
 __global__ void __launch_bounds__(256) fp4_amax_row_kernel(const __grid_constant__ Fp4QuantParams P) {
-  const int64_t ng = P.cols >> 4;
-  const int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x;
+  const int64_t ng = P.cols >> 4, total = P.rows * ng;
+  const uint32_t signs = P.rht_row ? rht_signs(P) : 0u;
   float m = 0.0f;
-  if (g < P.rows * ng) {
+  for (int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x; g < total; g += (int64_t)gridDim.x * 256) {
     float e[16];
     load_group16(P, g / ng, (g % ng) * 16, e);
-    if (P.rht_row) rht16_inthread(e, rht_signs(P));
+    if (P.rht_row) rht16_inthread(e, signs);
 #pragma unroll
     for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
   }
@@ -366,68 +338,74 @@ __global__ void __launch_bounds__(256) fp4_quant_row_kernel(const __grid_constan
   const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
   const int64_t kdom = P.sf_tiled ? s4 * 4 : nsf;
   const int64_t rdom = P.sf_tiled ? (P.rows + 127) / 128 * 128 : P.rows;
-  const int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x;
-  if (g >= rdom * kdom) return;
-  const int64_t row = g / kdom, kc = g % kdom;
-  uint32_t sb = 0;
-  if (row < P.rows && kc < nsf) {
-    const int64_t c = kc * 16;
-    float e[16];
-    load_group16(P, row, c, e);
-    if (P.rht_row) rht16_inthread(e, rht_signs(P));
-    float m = 0.0f;
+  const uint32_t signs = P.rht_row ? rht_signs(P) : 0u;
+  for (int64_t g = (int64_t)blockIdx.x * 256 + threadIdx.x; g < rdom * kdom; g += (int64_t)gridDim.x * 256) {
+    const int64_t row = g / kdom, kc = g % kdom;
+    uint32_t sb = 0;
+    if (row < P.rows && kc < nsf) {
+      const int64_t c = kc * 16;
+      float e[16];
+      load_group16(P, row, c, e);
+      if (P.rht_row) rht16_inthread(e, signs);
+      float m = 0.0f;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
-    float enc;
-    block_scale(m, S_g, enc_tab, sb, enc);
-    uint32_t w[2];
+      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+      float enc;
+      block_scale(m, S_g, enc_tab, sb, enc);
+      uint32_t w[2];
 #pragma unroll
-    for (int h = 0; h < 2; ++h) {
-      uint32_t codes = 0;
+      for (int h = 0; h < 2; ++h) {
+        uint32_t codes = 0;
 #pragma unroll
-      for (int q = 0; q < 2; ++q) {
-        const int j = 8 * h + 4 * q;
-        uint32_t c4;
-        if (P.sr_row) {
-          const uint64_t blk = (uint64_t)(row * P.cols + c + j) >> 2;
-          const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
-          c4 = e2m1_sr(__fmul_rn(e[j], enc), r.x) | (e2m1_sr(__fmul_rn(e[j + 1], enc), r.y) << 4) |
-               (e2m1_sr(__fmul_rn(e[j + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[j + 3], enc), r.w) << 12);
-        } else {
-          c4 = e2m1x2_rne(__fmul_rn(e[j + 1], enc), __fmul_rn(e[j], enc)) |
-               (e2m1x2_rne(__fmul_rn(e[j + 3], enc), __fmul_rn(e[j + 2], enc)) << 8);
+        for (int q = 0; q < 2; ++q) {
+          const int j = 8 * h + 4 * q;
+          uint32_t c4;
+          if (P.sr_row) {
+            const uint64_t blk = (uint64_t)(row * P.cols + c + j) >> 2;
+            const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
+            c4 = e2m1_sr(__fmul_rn(e[j], enc), r.x) | (e2m1_sr(__fmul_rn(e[j + 1], enc), r.y) << 4) |
+                 (e2m1_sr(__fmul_rn(e[j + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[j + 3], enc), r.w) << 12);
+          } else {
+            c4 = e2m1x2_rne(__fmul_rn(e[j + 1], enc), __fmul_rn(e[j], enc)) |
+                 (e2m1x2_rne(__fmul_rn(e[j + 3], enc), __fmul_rn(e[j + 2], enc)) << 8);
+          }
+          codes |= c4 << (16 * q);
         }
-        codes |= c4 << (16 * q);
+        w[h] = codes;
       }
-      w[h] = codes;
+      *(uint2*)(P.q_row + row * (P.cols >> 1) + (c >> 1)) = make_uint2(w[0], w[1]);
     }
-    *(uint2*)(P.q_row + row * (P.cols >> 1) + (c >> 1)) = make_uint2(w[0], w[1]);
+    if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+    else P.sf_row[row * nsf + kc] = (uint8_t)sb;
   }
-  if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
-  else P.sf_row[row * nsf + kc] = (uint8_t)sb;
 }
 
-static unsigned blocks_for(int64_t threads) { return (unsigned)((threads + 255) / 256); }
+// Grid of the group-per-thread kernels: enough CTAs to fill the GPU, at most 8192.
+static unsigned blocks_for(int64_t threads) {
+  const int64_t b = (threads + 255) / 256;
+  return (unsigned)(b < 8192 ? b : 8192);
+}
 
 cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
   const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
-  if (row && col) fp4_amax_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  const unsigned tile_grid = (unsigned)(tiles < 2048 ? tiles : 2048);
+  if (row && col) fp4_amax_kernel<true, true><<<tile_grid, 256, 0, s>>>(p, tiles);
   else if (row) fp4_amax_row_kernel<<<blocks_for(p.rows * (p.cols >> 4)), 256, 0, s>>>(p);
-  else fp4_amax_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
+  else fp4_amax_kernel<false, true><<<tile_grid, 256, 0, s>>>(p, tiles);
   return cudaGetLastError();
 }
 
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
   const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
-  if (row && col) {
-    fp4_quant_kernel<true, true><<<(unsigned)tiles, 256, 0, s>>>(p);
-  } else if (row) {
+  // Both outputs: the rowwise pass and the colwise pass run as separate kernels (one extra
+  // read of the input); each is ALU-bound with stochastic rounding, and apart they keep far
+  // more threads resident than the combined 16x4 kernel.
+  if (row) {
     const int64_t nsf = p.cols >> 4, kdom = p.sf_tiled ? (nsf + 3) / 4 * 4 : nsf;
     const int64_t rdom = p.sf_tiled ? (p.rows + 127) / 128 * 128 : p.rows;
     fp4_quant_row_kernel<<<blocks_for(rdom * kdom), 256, 0, s>>>(p);
-  } else {
-    fp4_quant_kernel<false, true><<<(unsigned)tiles, 256, 0, s>>>(p);
   }
+  if (col) fp4_quant_col_kernel<<<(unsigned)tiles, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 
