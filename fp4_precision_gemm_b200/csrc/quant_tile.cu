@@ -157,6 +157,14 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
 
   // ---------------------------------------------------------------- rowwise output
   if (ROW) {
+    // 1x128: the 16 lanes of a row group hold the same 8 row maxima; lane cs divides for row
+    // cs % 8 and the scales are shuffled out (one IEEE division per thread instead of 8)
+    float sf_own = 1.0f;
+    if (MODE == kTile1x128) {
+      const int pr = cs & 7;
+      const uint32_t w = pr < 2 ? rp[0] : pr < 4 ? rp[1] : pr < 6 ? rp[2] : rp[3];
+      sf_own = e4m3_sf(bf16_bits_to_float((pr & 1) ? (w >> 16) : (w & 0xFFFFu)));
+    }
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
       const int64_t row = r0 + rb * 8 + p;
@@ -166,18 +174,20 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
       if (MODE == kTile128) {
         sf = blk_sf;
       } else if (MODE == kTile1x128) {
-        sf = e4m3_sf(bf16_bits_to_float(abits));
+        sf = __shfl_sync(0xFFFFFFFFu, sf_own, (t & 16) | p);
       } else {
         e = mx_exponent(bf16_bits_to_float(abits));
         sf = pow2_neg(e);
       }
       if (row < P.rows && cok) {
-        uint2 o;
-        o.x = cvt_e4m3x2(__fmul_rn(elem(v[p], 0), sf), __fmul_rn(elem(v[p], 1), sf)) |
-              (cvt_e4m3x2(__fmul_rn(elem(v[p], 2), sf), __fmul_rn(elem(v[p], 3), sf)) << 16);
-        o.y = cvt_e4m3x2(__fmul_rn(elem(v[p], 4), sf), __fmul_rn(elem(v[p], 5), sf)) |
-              (cvt_e4m3x2(__fmul_rn(elem(v[p], 6), sf), __fmul_rn(elem(v[p], 7), sf)) << 16);
-        *(uint2*)(P.q_row + row * P.cols + col) = o;
+        const float2 s2 = make_float2(sf, sf);
+        uint32_t c[4];
+#pragma unroll
+        for (int q = 0; q < 4; ++q) {
+          const float2 y = __fmul2_rn(make_float2(elem(v[p], 2 * q), elem(v[p], 2 * q + 1)), s2);
+          c[q] = cvt_e4m3x2(y.x, y.y);
+        }
+        *(uint2*)(P.q_row + row * P.cols + col) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
       }
       if (MODE == kTile1x128 && cs == 0 && row < P.rows)
         ((float*)P.s_row)[(c0 >> 7) * P.ld_s_row + row] = __frcp_rn(sf);
@@ -203,13 +213,15 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
       if (MODE == kTile128) sf = blk_sf;
       else if (MODE == kTile1x128) sf = colsf[cs * 8 + j];
       else sf = pow2_neg(ecol[j]);
+      const float2 s2 = make_float2(sf, sf);
       uint32_t lo = 0, hi = 0;
 #pragma unroll
-      for (int p = 0; p < 4; p += 2)
-        lo |= cvt_e4m3x2(__fmul_rn(elem(v[p], j), sf), __fmul_rn(elem(v[p + 1], j), sf)) << (8 * p);
-#pragma unroll
-      for (int p = 4; p < 8; p += 2)
-        hi |= cvt_e4m3x2(__fmul_rn(elem(v[p], j), sf), __fmul_rn(elem(v[p + 1], j), sf)) << (8 * (p - 4));
+      for (int p = 0; p < 8; p += 2) {
+        const float2 y = __fmul2_rn(make_float2(elem(v[p], j), elem(v[p + 1], j)), s2);
+        const uint32_t c = cvt_e4m3x2(y.x, y.y);
+        if (p < 4) lo |= c << (8 * p);
+        else hi |= c << (8 * (p - 4));
+      }
       const int c = cs * 8 + j;
       *(uint2*)&tq[c * 128 + tq_chunk(c, rb) * 8] = make_uint2(lo, hi);
     }
