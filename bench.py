@@ -652,14 +652,18 @@ def measure_e2e(step, launches, stream, args):
             "ms_per_step": round(ms, 3), "h2d_bytes_per_step": bi, "d2h_bytes_per_step": bo}
 
 
-def cpu_baseline(step):
-    threads = torch.get_num_threads()
+def cpu_cores():
+    """Threads the oracle's NumPy/BLAS calls use on this host."""
     try:
         import numpy as np  # noqa: F401
         from threadpoolctl import threadpool_info
-        blas = max([i.get("num_threads", 1) for i in threadpool_info()] or [1])
+        return int(max([i.get("num_threads", 1) for i in threadpool_info()] or [1]))
     except Exception:  # noqa: BLE001
-        blas = threads
+        return int(torch.get_num_threads())
+
+
+def cpu_baseline(step):
+    blas = cpu_cores()
     # a bounded sample of about 12 s of CPU work: time one sampled tile per GEMM, then size
     # the measured sample (more sampled tiles of the same workload) from it
     _, dt1, _ = step.cpu_sample(tiles=1)
@@ -687,7 +691,7 @@ def run_reference(args, rank, world):
         flops += f
         secs += dt
     value = flops / secs / 1e12
-    cb = cpu_baseline(step)
+    cb = {"cores": cpu_cores()}
     return {"impl": "reference", "metric": METRIC, "value": round(value, 6), "unit": "TFLOP/s", "n_gpus": world,
             "steps": args.steps, "warmup": args.warmup, "ms_per_step": round(secs / args.steps * 1e3, 2),
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64",
