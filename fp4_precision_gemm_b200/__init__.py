@@ -21,13 +21,13 @@ __all__ = [
     "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp8q_quantize_tensor_noalloc", "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
-    "fp8q_get_device_status", "fp8q_status_string", "fp8q_version", "GemmArgs",
+    "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
     "quantize_1x128", "quantize_128x128", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
     "gemm", "device_status", "EXPORTED_SYMBOLS",
 ]
 
 FP8Q_OK = 0
-FP8Q_ERR_TIMEOUT = 6
+FP8Q_ERR_NULL, FP8Q_ERR_SHAPE, FP8Q_ERR_ALIGN, FP8Q_ERR_UNSUPPORTED, FP8Q_ERR_CUDA, FP8Q_ERR_TIMEOUT = 1, 2, 3, 4, 5, 6
 FP8Q_BLOCKWISE, FP8Q_MXFP8, FP8Q_PERTENSOR, FP8Q_NVFP4 = 0, 1, 2, 3
 FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD = 0, 1, 2
 FP8Q_SF_ROWMAJOR, FP8Q_SF_MMA_TILED = 0, 1
@@ -37,6 +37,7 @@ EXPORTED_SYMBOLS = [
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
+    "fp8q_selftest_bounded_wait",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -84,6 +85,7 @@ def lib():
         L.fp8q_sf_bytes.argtypes = [_int, _i64, _i64, _int]
         L.fp8q_sf_bytes.restype = ctypes.c_size_t
         L.fp8q_get_device_status.argtypes = [_vp]
+        L.fp8q_selftest_bounded_wait.argtypes = [_u64, _vp]
         L.fp8q_release_scratch.argtypes = []
         L.fp8q_status_string.argtypes = [_int]
         L.fp8q_status_string.restype = ctypes.c_char_p
@@ -94,7 +96,8 @@ def lib():
             if f.restype is ctypes.c_int or name in ("fp8q_quantize_1x128", "fp8q_quantize_128x128",
                                                      "fp8q_quantize_mx32", "fp8q_quantize_tensor",
                                                      "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
-                                                     "fp8q_get_device_status", "fp8q_release_scratch"):
+                                                     "fp8q_get_device_status", "fp8q_release_scratch",
+                                                     "fp8q_selftest_bounded_wait"):
                 f.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -161,6 +164,10 @@ def fp8q_sf_bytes(recipe, outer, inner, layout):
 
 def fp8q_get_device_status(stream):
     return lib().fp8q_get_device_status(stream)
+
+
+def fp8q_selftest_bounded_wait(limit_ns, stream):
+    return lib().fp8q_selftest_bounded_wait(limit_ns, stream)
 
 
 def fp8q_status_string(st):

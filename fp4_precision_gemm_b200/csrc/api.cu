@@ -131,6 +131,14 @@ fp8q_status fp8q_get_device_status(void* stream) {
   return word == 0 ? FP8Q_OK : static_cast<fp8q_status>(word);
 }
 
+fp8q_status fp8q_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
+  if (limit_ns < 1000ull || limit_ns > 1000000000ull) return FP8Q_ERR_SHAPE;
+  DeviceScratch* d = nullptr;
+  fp8q_status st = scratch(&d);
+  if (st != FP8Q_OK) return st;
+  return from_cuda(launch_selftest_wait(d->base, limit_ns, static_cast<cudaStream_t>(stream)));
+}
+
 fp8q_status fp8q_release_scratch(void) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;

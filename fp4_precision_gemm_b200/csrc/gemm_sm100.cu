@@ -770,6 +770,25 @@ static cudaError_t launch_scaled(const GemmParams& p, const CUtensorMap& a, cons
   return cudaGetLastError();
 }
 
+// Failure-detection self test: one thread waits on a barrier nothing arrives on; the bounded
+// wait gives up after limit_ns and records the timeout like a GEMM role would.
+__global__ void __launch_bounds__(32) selftest_wait_kernel(uint32_t* status, uint64_t limit_ns) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(&bar, 1);
+    abort_flag = 0;
+    fence_barrier_init();
+  }
+  __syncwarp();
+  if (threadIdx.x == 0 && !mbar_wait(&bar, 0, &abort_flag, limit_ns)) atomicExch(status, kDevTimeout);
+}
+
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s) {
+  selftest_wait_kernel<<<1, 32, 0, s>>>(status, limit_ns);
+  return cudaGetLastError();
+}
+
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, int num_sms, cudaStream_t s) {
   if (p.recipe == kBlockwise) {

@@ -77,6 +77,8 @@ struct GemmParams {
   uint32_t* status;        // device status word
 };
 
+cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
+
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, int num_sms, cudaStream_t s);
 

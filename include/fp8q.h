@@ -224,6 +224,16 @@ size_t fp8q_sf_bytes(fp8q_recipe recipe, int64_t outer, int64_t inner, fp8q_sf_l
  * (FP8Q_OK, or FP8Q_ERR_TIMEOUT if a kernel's bounded wait ran out since the last call). */
 fp8q_status fp8q_get_device_status(void* stream);
 
+/* Failure-detection self test (not part of the pages' method).  Launches one warp whose
+ * first thread waits, with the same bounded mbarrier wait the GEMM kernels use, on a
+ * shared-memory barrier that nothing ever arrives on.  After `limit_ns` nanoseconds of
+ * wall time (1e3 .. 1e9) the wait gives up and records FP8Q_ERR_TIMEOUT in the device
+ * status word, exactly as a GEMM role does before it winds down; the kernel then exits
+ * with no copy or MMA in flight and the context stays usable.  Returns the launch status
+ * (FP8Q_ERR_SHAPE for a limit out of range); read the outcome with
+ * fp8q_get_device_status(). */
+fp8q_status fp8q_selftest_bounded_wait(uint64_t limit_ns, void* stream);
+
 /* Frees the current device's scratch pool (after a device sync).  Optional. */
 fp8q_status fp8q_release_scratch(void);
 

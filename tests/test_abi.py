@@ -145,3 +145,8 @@ def test_product_path_has_no_cpu_fallback():
             mod.lib()
     finally:
         mod.library_path, mod._LIB = saved_path, saved_lib
+
+
+def test_selftest_rejects_limits_out_of_range(L):
+    assert L.fp8q_selftest_bounded_wait(10, None) == fq.FP8Q_ERR_SHAPE          # below 1 us
+    assert L.fp8q_selftest_bounded_wait(5_000_000_000, None) == fq.FP8Q_ERR_SHAPE   # above 1 s
