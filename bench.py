@@ -337,23 +337,22 @@ class MoeStep:
                 assert fq.fp8q_quantize_1x128(P(p["A"]), M, K, K, P(p["qa"]), P(p["sa"]), M, None, None, 0,
                                               fq._stream()) == 0
 
-            def qw(p=p, K=K, N=N, Gn=Gn):
-                for g in range(Gn):
-                    assert fq.fp8q_quantize_128x128(P(p["W"][g]), K, N, N, P(p["B"][g]), None, P(p["SB"][g]),
-                                                    fq._stream()) == 0
+            def qw(p=p, K=K, N=N, Gn=Gn):   # all experts' weights in one grouped call
+                assert fq.fp8q_quantize_128x128_grouped(P(p["W"]), Gn, K, N, N, P(p["B"]), None, P(p["SB"]),
+                                                        fq._stream()) == 0
 
             def g_(p=p, K=K):
                 fq.gemm(p["qa"], p["B"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=p["sa"], b_scale=p["SB"],
                         ld_sb=K // 128, m_offsets=p["offs"], out=p["C"])
 
             out += [Launch(f"quantize_1x128 A_{p['proj']}", qa, "quantize", bytes_=b_1x128_row(M, K)),
-                    Launch(f"quantize_128x128 W_{p['proj']} x{Gn}", qw, "quantize",
+                    Launch(f"quantize_128x128 grouped W_{p['proj']} ({Gn} experts)", qw, "quantize",
                            bytes_=Gn * (K * N * 3.0 + (K // 128) * (N // 128) * 4)),
                     Launch(f"gemm grouped blockwise {p['proj']}", g_, "gemm_grouped", flop=2.0 * M * N * K)]
         return out
 
     def launch_count(self):
-        return sum(2 + p["G"] for p in self.parts)
+        return 3 * len(self.parts)
 
     def cpu_sample(self, tiles=1):
         from oracle import gemm as G

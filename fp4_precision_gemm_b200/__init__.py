@@ -20,9 +20,9 @@ __all__ = [
     "FP8Q_FPROP", "FP8Q_DGRAD", "FP8Q_WGRAD", "FP8Q_SF_ROWMAJOR", "FP8Q_SF_MMA_TILED",
     "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
-    "fp8q_quantize_tensor_noalloc", "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
+    "fp8q_quantize_tensor_noalloc", "fp8q_quantize_128x128_grouped", "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
     "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
-    "quantize_1x128", "quantize_128x128", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
+    "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
     "gemm", "device_status", "EXPORTED_SYMBOLS",
 ]
 
@@ -37,7 +37,7 @@ EXPORTED_SYMBOLS = [
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
-    "fp8q_selftest_bounded_wait",
+    "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -76,6 +76,7 @@ def lib():
         L = ctypes.CDLL(library_path)
         L.fp8q_quantize_1x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _i64, _vp, _vp, _i64, _vp]
         L.fp8q_quantize_128x128.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
+        L.fp8q_quantize_128x128_grouped.argtypes = [_vp, _i64, _i64, _i64, _i64, _vp, _vp, _vp, _vp]
         L.fp8q_quantize_mx32.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_quantize_tensor.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
         L.fp8q_quantize_tensor_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
@@ -97,7 +98,7 @@ def lib():
                                                      "fp8q_quantize_mx32", "fp8q_quantize_tensor",
                                                      "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
                                                      "fp8q_get_device_status", "fp8q_release_scratch",
-                                                     "fp8q_selftest_bounded_wait"):
+                                                     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped"):
                 f.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -132,6 +133,10 @@ def fp8q_quantize_1x128(x, rows, cols, ld_x, q_row, s_row, ld_s_row, q_col, s_co
 
 def fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream):
     return lib().fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream)
+
+
+def fp8q_quantize_128x128_grouped(w, groups, K, N, ld_w, q_t, q, s, stream):
+    return lib().fp8q_quantize_128x128_grouped(w, groups, K, N, ld_w, q_t, q, s, stream)
 
 
 def fp8q_quantize_mx32(x, rows, cols, ld_x, q_row, e_row, q_col, e_col, sf_layout, stream):
@@ -217,6 +222,26 @@ def quantize_128x128(w, transposed=True, plain=True, stream=None):
     st = fp8q_quantize_128x128(_ptr(w), K, N, w.stride(0), _ptr(out.get("q_t")), _ptr(out.get("q")),
                                _ptr(out["s"]), _stream(stream))
     _check(st, "fp8q_quantize_128x128")
+    return out
+
+
+def quantize_128x128_grouped(w, transposed=True, plain=True, stream=None):
+    """128x128 blocks of every matrix of a stack W (G x K x N, contiguous matrices) in one
+    call.  Returns q_t (G, N, K), q (G, K, N), s (G, N/128, K/128)."""
+    if w.dim() != 3 or w.dtype != torch.bfloat16 or not w.is_cuda:
+        raise ValueError("w must be a CUDA bfloat16 tensor of shape (G, K, N)")
+    if w.stride(2) != 1 or w.stride(0) != w.shape[1] * w.stride(1):
+        raise ValueError("w must hold contiguous row-major matrices (row stride may be padded)")
+    G, K, N = w.shape
+    dev = w.device
+    out = {"s": torch.empty((G, N // 128, K // 128), dtype=torch.float32, device=dev)}
+    if transposed:
+        out["q_t"] = torch.empty((G, N, K), dtype=torch.uint8, device=dev)
+    if plain:
+        out["q"] = torch.empty((G, K, N), dtype=torch.uint8, device=dev)
+    st = fp8q_quantize_128x128_grouped(_ptr(w), G, K, N, w.stride(1), _ptr(out.get("q_t")), _ptr(out.get("q")),
+                                       _ptr(out["s"]), _stream(stream))
+    _check(st, "fp8q_quantize_128x128_grouped")
     return out
 
 

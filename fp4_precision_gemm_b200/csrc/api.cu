@@ -197,6 +197,28 @@ fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t l
                                      static_cast<cudaStream_t>(stream)));
 }
 
+fp8q_status fp8q_quantize_128x128_grouped(const void* w, int64_t groups, int64_t K, int64_t N, int64_t ld_w,
+                                          uint8_t* q_t, uint8_t* q, float* s, void* stream) {
+  if (groups < 0) return FP8Q_ERR_SHAPE;
+  fp8q_status st = check_input(w, K, N, ld_w);
+  if (st != FP8Q_OK) return st;
+  if (!s) return FP8Q_ERR_NULL;
+  if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
+  if ((q && !aligned16(q)) || (q_t && !aligned16(q_t))) return FP8Q_ERR_ALIGN;
+  if (groups == 0 || K == 0 || N == 0) return FP8Q_OK;
+  const int64_t per = tiles_of(K, N);
+  if (groups * per >= (1ll << 31)) return FP8Q_ERR_SHAPE;
+  TileQuantParams p{static_cast<const uint16_t*>(w), K, N, ld_w, q, s, K / 128, q_t, nullptr, 0,
+                    (int)(N / 128), 0};
+  p.batch_tiles = per;
+  p.x_bstride = K * ld_w;
+  p.q_row_bstride = K * N;
+  p.q_col_bstride = N * K;
+  p.s_row_bstride = (N / 128) * (K / 128) * (int64_t)sizeof(float);
+  return from_cuda(launch_tile_quant(kTile128, q != nullptr, q_t != nullptr, p, groups * per,
+                                     static_cast<cudaStream_t>(stream)));
+}
+
 fp8q_status fp8q_quantize_mx32(const void* x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t* q_row,
                                uint8_t* e8m0_row, uint8_t* q_col, uint8_t* e8m0_col, fp8q_sf_layout sf_layout,
                                void* stream) {

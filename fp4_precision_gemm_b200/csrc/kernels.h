@@ -19,6 +19,10 @@ struct TileQuantParams {
   int64_t ld_s_col;
   int tiles_c;      // 128-column tiles per 128-row band
   int sf_tiled;     // MX scale bytes in the MMA-tiled layout
+  // grouped calls (0 = one matrix): tiles per matrix, and each operand's stride between
+  // consecutive matrices (x in elements, outputs and scales in bytes)
+  int64_t batch_tiles;
+  int64_t x_bstride, q_row_bstride, q_col_bstride, s_row_bstride, s_col_bstride;
 };
 
 cudaError_t launch_tile_quant(int mode, bool row, bool col, const TileQuantParams& p,

@@ -56,8 +56,17 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
 
   const int t = threadIdx.x, warp = t >> 5;
   const int cs = t & 15, rb = t >> 4;
-  const int64_t r0 = (int64_t)(blockIdx.x / P.tiles_c) * 128;
-  const int64_t c0 = (int64_t)(blockIdx.x % P.tiles_c) * 128;
+  // grouped calls: CTA -> (matrix b, tile within it); every operand pointer moves by b strides
+  int64_t tile = blockIdx.x;
+  const int64_t bidx = P.batch_tiles ? tile / P.batch_tiles : 0;
+  tile -= bidx * P.batch_tiles;
+  const uint16_t* X = P.x + bidx * P.x_bstride;
+  uint8_t* QR = P.q_row ? P.q_row + bidx * P.q_row_bstride : nullptr;
+  uint8_t* QC = P.q_col ? P.q_col + bidx * P.q_col_bstride : nullptr;
+  uint8_t* SR = P.s_row ? (uint8_t*)P.s_row + bidx * P.s_row_bstride : nullptr;
+  uint8_t* SC = P.s_col ? (uint8_t*)P.s_col + bidx * P.s_col_bstride : nullptr;
+  const int64_t r0 = (tile / P.tiles_c) * 128;
+  const int64_t c0 = (tile % P.tiles_c) * 128;
   const int64_t col = c0 + cs * 8;
   const bool cok = col < P.cols;
 
@@ -65,7 +74,7 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
 #pragma unroll
   for (int p = 0; p < 8; ++p) {
     const int64_t row = r0 + rb * 8 + p;
-    v[p] = (cok && row < P.rows) ? ldg_nc_v4(P.x + row * P.ld_x + col) : make_uint4(0, 0, 0, 0);
+    v[p] = (cok && row < P.rows) ? ldg_nc_v4(X + row * P.ld_x + col) : make_uint4(0, 0, 0, 0);
   }
 
   // ---------------------------------------------------------------- amax reductions
@@ -84,8 +93,8 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
 #pragma unroll
     for (int w = 1; w < 8; ++w) bm = max(bm, red[w][0]);
     blk_sf = e4m3_sf(bf16_bits_to_float(bm));
-    if (t == 0 && P.s_row != nullptr)
-      ((float*)P.s_row)[(c0 >> 7) * P.ld_s_row + (r0 >> 7)] = __frcp_rn(blk_sf);
+    if (t == 0 && SR != nullptr)
+      ((float*)SR)[(c0 >> 7) * P.ld_s_row + (r0 >> 7)] = __frcp_rn(blk_sf);
   } else if (ROW) {
     const int lanes = (MODE == kTile1x128) ? 16 : 4;
 #pragma unroll
@@ -121,7 +130,7 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
           const float sf = e4m3_sf(bf16_bits_to_float(h ? (m >> 16) : (m & 0xFFFFu)));
           colsf[cc + h] = sf;
           if (c0 + cc + h < P.cols)
-            ((float*)P.s_col)[(r0 >> 7) * P.ld_s_col + c0 + cc + h] = __frcp_rn(sf);
+            ((float*)SC)[(r0 >> 7) * P.ld_s_col + c0 + cc + h] = __frcp_rn(sf);
         }
       }
       __syncthreads();
@@ -141,7 +150,7 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
       if (t < 128) {
         const int64_t cg = c0 + t;
         const uint32_t e4 = *(const uint32_t*)&colexp[t * 4];
-        uint8_t* dst = (uint8_t*)P.s_col;
+        uint8_t* dst = SC;
         const int64_t nsf = P.rows >> 5;
         if (P.sf_tiled) {  // padding rows of the tiled image get code 0 (their amax is 0)
           const int64_t s4 = (nsf + 3) >> 2;
@@ -187,13 +196,13 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
           const float2 y = __fmul2_rn(make_float2(elem(v[p], 2 * q), elem(v[p], 2 * q + 1)), s2);
           c[q] = cvt_e4m3x2(y.x, y.y);
         }
-        *(uint2*)(P.q_row + row * P.cols + col) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+        *(uint2*)(QR + row * P.cols + col) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
       }
       if (MODE == kTile1x128 && cs == 0 && row < P.rows)
-        ((float*)P.s_row)[(c0 >> 7) * P.ld_s_row + row] = __frcp_rn(sf);
+        ((float*)SR)[(c0 >> 7) * P.ld_s_row + row] = __frcp_rn(sf);
       if (MODE == kTileMX && (cs & 3) == 0) {
         const int64_t kc = (col >> 5);
-        uint8_t* dst = (uint8_t*)P.s_row;
+        uint8_t* dst = SR;
         const int64_t nsf = P.cols >> 5;
         if (P.sf_tiled) {
           const int64_t s4 = (nsf + 3) >> 2;
@@ -233,7 +242,7 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
       const uint2 a = *(const uint2*)&tq[c * 128 + tq_chunk(c, 2 * h) * 8];
       const uint2 b = *(const uint2*)&tq[c * 128 + tq_chunk(c, 2 * h + 1) * 8];
       if (cg < P.cols && rg < P.rows)
-        *(uint4*)(P.q_col + cg * P.rows + rg) = make_uint4(a.x, a.y, b.x, b.y);
+        *(uint4*)(QC + cg * P.rows + rg) = make_uint4(a.x, a.y, b.x, b.y);
     }
   }
 }

@@ -109,6 +109,15 @@ fp8q_status fp8q_quantize_1x128(const void* x, int64_t rows, int64_t cols, int64
 fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t ld_w,
                                   uint8_t* q_t, uint8_t* q, float* s, void* stream);
 
+/* [DSV3] "Fine-grained quantization" for a stack of weight matrices (the experts of a MoE
+ * layer), in one launch: groups matrices w[g] = w + g * K * ld_w, each BF16 K x N with row
+ * stride ld_w, quantized exactly as fp8q_quantize_128x128 quantizes one.  Outputs are
+ * contiguous per matrix: q_t[g] = q_t + g * N * K (N x K codes, the grouped GEMM's B
+ * operand), q[g] = q + g * K * N, s[g] = s + g * (N/128) * (K/128).  Same requirements as
+ * fp8q_quantize_128x128; groups == 0 -> FP8Q_OK, nothing launched. */
+fp8q_status fp8q_quantize_128x128_grouped(const void* w, int64_t groups, int64_t K, int64_t N, int64_t ld_w,
+                                          uint8_t* q_t, uint8_t* q, float* s, void* stream);
+
 /* [NeMo] MXFP8: 32-element blocks, E8M0 scale = smallest e with amax <= 448 * 2^e
  * (amax == 0 -> e = -127; e clamped to [-127, 127]; byte e + 127), codes
  * E4M3(fp32(x * 2^-e)).

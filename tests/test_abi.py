@@ -150,3 +150,11 @@ def test_product_path_has_no_cpu_fallback():
 def test_selftest_rejects_limits_out_of_range(L):
     assert L.fp8q_selftest_bounded_wait(10, None) == fq.FP8Q_ERR_SHAPE          # below 1 us
     assert L.fp8q_selftest_bounded_wait(5_000_000_000, None) == fq.FP8Q_ERR_SHAPE   # above 1 s
+
+
+def test_grouped_weight_quantizer_validates_before_launching(L):
+    s = None
+    assert fq.fp8q_quantize_128x128_grouped(ALIGNED, -1, 128, 128, 128, ALIGNED, None, ALIGNED, s) == fq.FP8Q_ERR_SHAPE
+    assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 2, 128, 100, 128, ALIGNED, None, ALIGNED, s) == fq.FP8Q_ERR_SHAPE
+    assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 2, 128, 128, 128, ALIGNED, None, None, s) == fq.FP8Q_ERR_NULL
+    assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 0, 128, 128, 128, ALIGNED, None, ALIGNED, s) == fq.FP8Q_OK

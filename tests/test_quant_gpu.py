@@ -77,6 +77,22 @@ def test_128x128_parity(cuda_lib, K, N):
 
 
 # ----------------------------------------------------------------------------- MX
+def test_128x128_grouped_matches_each_matrix(cuda_lib):
+    """A stack of expert weight matrices quantized in one grouped call equals quantizing
+    each matrix on its own (oracle), codes of both layouts and scales bit for bit."""
+    fq = cuda_lib
+    G, K, N = 3, 256, 384
+    ws = [workloads.normal_bf16((K, N), 0.006, 40 + g, 1e-3, 30.0) for g in range(G)]
+    w = torch.stack(ws).cuda()
+    out = fq.quantize_128x128_grouped(w)
+    assert fq.device_status() == 0
+    for g in range(G):
+        oq, oqt, os_ = Q.quantize_128x128(workloads.bf16_bits(ws[g]))
+        assert np.array_equal(out["q"][g].cpu().numpy(), oq)
+        assert np.array_equal(out["q_t"][g].cpu().numpy(), oqt)
+        assert np.array_equal(out["s"][g].cpu().numpy().view(np.uint32), os_.astype(np.float32).view(np.uint32))
+
+
 @pytest.mark.parametrize("layout", [0, 1])
 @pytest.mark.parametrize("R,C,row,col", [(300, 672, True, False), (352, 656, False, True),
                                          (384, 640, True, True), (64, 32, True, True)])
