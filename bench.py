@@ -12,8 +12,8 @@ quantization included) with per-kernel TFLOP/s and GB/s as fractions of the roof
 Contract: python bench.py --gpus N --steps K --warmup W [--impl ours|reference]
   * N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs the step on
     its own tokens (weak scaling, no data-path collective); timing is the max over ranks.
-  * Inputs live in HBM before the timed region; the L2 is flushed (256 MiB write) between
-    steps, outside the per-step events.
+  * Inputs live in HBM before the timed region; the L2 is flushed between steps (a 256 MiB
+    write, then a 256 MiB read so no dirty lines remain), outside the per-step events.
   * --impl reference times the CPU oracle (rank 0 only) on a bounded sample of the step.
 """
 import argparse
@@ -520,6 +520,7 @@ def run_ours(args, rank, world, local_rank):
     launches = step.launches()
     n_launch = getattr(step, "launch_count", lambda: len(launches))()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
+    clean = torch.zeros(64 << 20, dtype=torch.int32, device="cuda")   # 256 MiB, read after the flush
     stream = torch.cuda.current_stream()
 
     def barrier():
@@ -540,7 +541,11 @@ def run_ours(args, rank, world, local_rank):
     time.sleep(0.15)
     t_wall = time.perf_counter()
     for k in range(args.steps):
-        flush.fill_(k & 0xFF)                     # L2 flush (256 MiB write), outside the events
+        # L2 flush outside the events: a 256 MiB write, then a 256 MiB read, so the step starts
+        # from an L2 holding none of its data and no dirty lines (else the first kernel of
+        # the step would pay the write-back of the flush buffer)
+        flush.fill_(k & 0xFF)
+        clean.max()
         for L, (a, b) in zip(launches, ev[k]):
             a.record(stream)
             L.fn()
@@ -599,7 +604,7 @@ def run_ours(args, rank, world, local_rank):
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
         "vs_baseline": None, "dtype": "fp8_e4m3" if args.workload != "nvfp4" else "fp4_e2m1",
         "data": "synthetic (seeded normal BF16 with outliers; see workloads.py)",
-        "config": {"workload": step.workload, "l2": "flushed between steps (256 MiB write)",
+        "config": {"workload": step.workload, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "gemm_tflop_per_step": round(step.gemm_flop / 1e12, 4),
                    "parallelism": f"dp{world} (independent replicas, no collective)"},
         "roofline": roof, "kernels": kern, "gpu_launches": n_launch * args.steps,
