@@ -218,6 +218,74 @@ class TinyStep(LlamaStep):
         return self.gemm_flop, time.perf_counter() - t0, "the whole tiny step"
 
 
+class WgradAccStep:
+    """Llama-3-8B weight gradient with FP32 main-gradient accumulation: X and dY quantized
+    in 1x128 tiles along the tokens (transposed outputs), then dW (FP32, 4096 x 14336) +=
+    X^T . dY with the blockwise promotion."""
+    name = "wgrad_acc"
+    workload = "llama3-8b wgrad into FP32 main gradients: X 8192x4096, dY 8192x14336, dW 4096x14336 fp32 +="
+
+    def __init__(self, fq, rank, M=8192, K=4096, N=14336):
+        self.fq, self.M, self.K, self.N = fq, M, K, N
+        d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
+        self.X, self.dY = d["X"], d["dY"]
+        del d
+        dev = self.X.device
+        self.qx_c = torch.empty((K, M), dtype=torch.uint8, device=dev)
+        self.sx_c = torch.empty((M // 128, K), dtype=torch.float32, device=dev)
+        self.qd_c = torch.empty((N, M), dtype=torch.uint8, device=dev)
+        self.sd_c = torch.empty((M // 128, N), dtype=torch.float32, device=dev)
+        self.dW = torch.zeros((K, N), dtype=torch.float32, device=dev)
+        self.gemm_flop = 2.0 * M * N * K
+
+    def inputs(self):
+        return [self.X, self.dY]
+
+    def outputs(self):
+        return [self.dW]
+
+    def launches(self):
+        fq, M, K, N = self.fq, self.M, self.K, self.N
+        P = lambda t: t.data_ptr()  # noqa: E731
+
+        def qcol(x, q, sc, C):
+            def f():
+                assert fq.fp8q_quantize_1x128(P(x), M, C, C, None, None, 0, P(q), P(sc), sc.shape[1],
+                                              fq._stream()) == 0
+            return f
+
+        def g():
+            fq.gemm(self.qx_c, self.qd_c, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=self.sx_c, b_scale=self.sd_c,
+                    ld_sb=N, out=self.dW, accumulate_fp32=True)
+
+        return [Launch("quantize_1x128 X colwise", qcol(self.X, self.qx_c, self.sx_c, K), "quantize",
+                       bytes_=b_1x128_row(M, K)),
+                Launch("quantize_1x128 dY colwise", qcol(self.dY, self.qd_c, self.sd_c, N), "quantize",
+                       bytes_=b_1x128_row(M, N)),
+                Launch("gemm blockwise wgrad FP32 accumulate", g, "gemm_blockwise_acc",
+                       flop=self.gemm_flop)]
+
+    def cpu_sample(self, tiles=1):
+        """Oracle on a bounded sample: `tiles` sampled 128x128 tiles of dW, operands quantized
+        by the oracle, FP64 product added to the FP32 values the tiles held."""
+        from oracle import gemm as G
+        from oracle import quant as Q
+        M, K, N = self.M, self.K, self.N
+        if not hasattr(self, "_host_bits"):
+            self._host_bits = tuple(workloads.bf16_bits(t) for t in (self.X, self.dY))
+        Xb, dYb = self._host_bits
+        t0 = time.perf_counter()
+        flop = 0.0
+        for m0, n0 in G.sample_tiles(K, N, tiles, seed=5):
+            oa, sa = Q.quantize_1x128_colwise(Xb[:, m0:m0 + 128])
+            ob, sb = Q.quantize_1x128_colwise(dYb[:, n0:n0 + 128])
+            G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
+            flop += 2.0 * 128 * 128 * M
+        dt = time.perf_counter() - t0
+        return flop, dt, (f"{tiles} sampled 128x128 dW tile(s), operands quantized by the oracle from the BF16 "
+                          "inputs, FP64 reference product")
+
+
 class MxStep:
     name = "mxfp8"
     workload = "MXFP8 (and per-tensor) GEMMs (M,K,N) = (8192,4096,4096), (8192,4096,14336), (8192,14336,4096)"
@@ -443,7 +511,8 @@ class Nvfp4Step:
         return flop, time.perf_counter() - t0, "1 dgrad output tile; amax over 1024-row slabs"
 
 
-STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step}
+STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step,
+         "wgrad_acc": WgradAccStep}
 
 
 # ============================================================================ measurement

@@ -59,6 +59,7 @@ class GemmArgs(ctypes.Structure):
         ("a_global", ctypes.c_void_p), ("b_global", ctypes.c_void_p),
         ("c", ctypes.c_void_p), ("ldc", ctypes.c_int64),
         ("m_offsets", ctypes.c_void_p), ("num_groups", ctypes.c_int32),
+        ("c_fp32_accumulate", ctypes.c_int32),
     ]
 
 
@@ -300,14 +301,17 @@ def rht16_quantize_sr(x, rowwise=True, colwise=False, rht=0, rht_seed=0, sr=0, s
 
 
 def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
-         a_global=None, b_global=None, K=None, m_offsets=None, out=None, stream=None):
+         a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False, stream=None):
     """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
-    Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16."""
+    Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16.
+    accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T."""
     M = a.shape[0]
     grouped = m_offsets is not None
     N = b.shape[1] if grouped else b.shape[0]
     if K is None:
         K = a.shape[1] * (2 if recipe == FP8Q_NVFP4 else 1)
+    if accumulate_fp32 and (out is None or out.dtype != torch.float32):
+        raise ValueError("accumulate_fp32 needs an FP32 `out` tensor to update")
     c = out if out is not None else torch.empty((M, N), dtype=torch.bfloat16, device=a.device)
     args = GemmArgs()
     args.recipe, args.layout = recipe, layout
@@ -323,6 +327,7 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
     args.c, args.ldc = c.data_ptr(), c.stride(0)
     args.m_offsets = m_offsets.data_ptr() if grouped else None
     args.num_groups = (m_offsets.numel() - 1) if grouped else 0
+    args.c_fp32_accumulate = 1 if accumulate_fp32 else 0
     _check(fp8q_gemm_blockscaled(args, _stream(stream)), "fp8q_gemm_blockscaled")
     return c
 

@@ -317,12 +317,15 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (a->layout < FP8Q_FPROP || a->layout > FP8Q_WGRAD) return FP8Q_ERR_UNSUPPORTED;
   if (a->M < 0 || a->N < 0 || a->K < 0) return FP8Q_ERR_SHAPE;
   if (a->M >= (1ll << 31) || a->N >= (1ll << 31) || a->K >= (1ll << 31)) return FP8Q_ERR_SHAPE;
+  const bool acc32 = a->c_fp32_accumulate != 0;
+  if (acc32 && a->recipe != FP8Q_BLOCKWISE) return FP8Q_ERR_UNSUPPORTED;
   if (a->M == 0 || a->N == 0) return FP8Q_OK;
   if (!a->c) return FP8Q_ERR_NULL;
-  if (a->ldc < a->N || a->ldc % 8 != 0) return FP8Q_ERR_SHAPE;
+  if (a->ldc < a->N || a->ldc % (acc32 ? 4 : 8) != 0) return FP8Q_ERR_SHAPE;
   if (!aligned16(a->c)) return FP8Q_ERR_ALIGN;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
-  if (a->K == 0) {  // empty sum
+  if (a->K == 0) {  // empty sum: C = 0, or C unchanged when accumulating
+    if (acc32) return FP8Q_OK;
     return from_cuda(cudaMemset2DAsync(a->c, (size_t)a->ldc * 2, 0, (size_t)a->N * 2, (size_t)a->M, s));
   }
   const bool fp4 = a->recipe == FP8Q_NVFP4;
@@ -345,7 +348,8 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   p.M = (int)a->M;
   p.N = (int)a->N;
   p.K = (int)a->K;
-  p.c = static_cast<uint16_t*>(a->c);
+  p.c = acc32 ? nullptr : static_cast<uint16_t*>(a->c);
+  p.c32 = acc32 ? static_cast<float*>(a->c) : nullptr;
   p.ldc = a->ldc;
   p.m_offsets = a->m_offsets;
   p.num_groups = a->num_groups;

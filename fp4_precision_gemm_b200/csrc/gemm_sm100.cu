@@ -93,6 +93,22 @@ __device__ __forceinline__ void store8_bf16(const GemmParams& p, int m, int n, u
 }
 
 
+// C[m, n..n+3] += four FP32 values (FP32 accumulate mode); scalar past column N.
+__device__ __forceinline__ void add4_f32(const GemmParams& p, int m, int n, uint4 v) {
+  float* dst = p.c32 + (int64_t)m * p.ldc + n;
+  const float x[4] = {__uint_as_float(v.x), __uint_as_float(v.y), __uint_as_float(v.z), __uint_as_float(v.w)};
+  if (n + 4 <= p.N) {
+    float4 o = *reinterpret_cast<float4*>(dst);
+    o.x = __fadd_rn(o.x, x[0]);
+    o.y = __fadd_rn(o.y, x[1]);
+    o.z = __fadd_rn(o.z, x[2]);
+    o.w = __fadd_rn(o.w, x[3]);
+    *reinterpret_cast<float4*>(dst) = o;
+  } else {
+    for (int i = 0; i < 4 && n + i < p.N; ++i) dst[i] = __fadd_rn(dst[i], x[i]);
+  }
+}
+
 // ------------------------------------------------------------------ hardware-scaled kernel
 // MXFP8, NVFP4 and per-tensor: 128 x 256 output tiles accumulated across all of K in TMEM
 // (256 columns per accumulator); the scale factors of MX / NVFP4 stages are copied from
@@ -439,7 +455,7 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 
 }  // namespace
 
-template <int L, bool GROUPED>
+template <int L, bool GROUPED, bool ACC32>
 __global__ void __launch_bounds__(kBwThreads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
@@ -666,30 +682,53 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         ++chunk;
       }
       if (!ok) break;
-      // Epilogue through this warp's staging buffer, epi_cols columns at a time: each lane
-      // writes its row's BF16 values as 16-byte chunks XOR-swizzled by row (conflict-free),
-      // then CPR lanes per row store the row's contiguous bytes (128 B for 64 columns),
-      // 32 / CPR rows per instruction.
+      // Epilogue through this warp's staging buffer: each lane writes its row's values as
+      // 16-byte chunks XOR-swizzled by row (conflict-free), then CPR lanes per row move the
+      // row's contiguous bytes (128 B per row for fprop/dgrad, 64 B for wgrad), 32 / CPR
+      // rows per instruction.  BF16 output: 8 values per chunk, stored.  FP32 accumulate:
+      // 4 values per chunk, added to C in FP32.
       constexpr int EC = S::epi_cols, CPR = EC / 8, RPI = 32 / CPR;
       auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
       uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
+      if constexpr (!ACC32) {
 #pragma unroll
-      for (int h = 0; h < 64 / EC; ++h) {
+        for (int h = 0; h < 64 / EC; ++h) {
 #pragma unroll
-        for (int c = 0; c < CPR; ++c) {
-          const float2* a4 = acc + h * (EC / 2) + c * 4;
-          stg[lane * CPR + (c ^ swz(lane))] = make_uint4(pack_bf16(a4[0].x, a4[0].y), pack_bf16(a4[1].x, a4[1].y),
-                                                         pack_bf16(a4[2].x, a4[2].y), pack_bf16(a4[3].x, a4[3].y));
+          for (int c = 0; c < CPR; ++c) {
+            const float2* a4 = acc + h * (EC / 2) + c * 4;
+            stg[lane * CPR + (c ^ swz(lane))] = make_uint4(pack_bf16(a4[0].x, a4[0].y), pack_bf16(a4[1].x, a4[1].y),
+                                                           pack_bf16(a4[2].x, a4[2].y), pack_bf16(a4[3].x, a4[3].y));
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < CPR; ++i) {
+            const int r = i * RPI + lane / CPR, c = lane % CPR;
+            const uint4 v = stg[r * CPR + (c ^ swz(r))];
+            const int mr = T.m0 + q * 32 + r, n = ncol0 + h * EC + c * 8;
+            if (mr < T.mend && n < p.N) store8_bf16(p, mr, n, v);
+          }
+          __syncwarp();
         }
-        __syncwarp();
+      } else {
+        constexpr int EC32 = EC / 2;   // FP32 columns per pass (same bytes per row)
 #pragma unroll
-        for (int i = 0; i < CPR; ++i) {
-          const int r = i * RPI + lane / CPR, c = lane % CPR;
-          const uint4 v = stg[r * CPR + (c ^ swz(r))];
-          const int mr = T.m0 + q * 32 + r, n = ncol0 + h * EC + c * 8;
-          if (mr < T.mend && n < p.N) store8_bf16(p, mr, n, v);
+        for (int h = 0; h < 64 / EC32; ++h) {
+#pragma unroll
+          for (int c = 0; c < CPR; ++c) {
+            const float2* a2 = acc + h * (EC32 / 2) + c * 2;
+            stg[lane * CPR + (c ^ swz(lane))] = make_uint4(__float_as_uint(a2[0].x), __float_as_uint(a2[0].y),
+                                                           __float_as_uint(a2[1].x), __float_as_uint(a2[1].y));
+          }
+          __syncwarp();
+#pragma unroll
+          for (int i = 0; i < CPR; ++i) {
+            const int r = i * RPI + lane / CPR, c = lane % CPR;
+            const uint4 v = stg[r * CPR + (c ^ swz(r))];
+            const int mr = T.m0 + q * 32 + r, n = ncol0 + h * EC32 + c * 4;
+            if (mr < T.mend && n < p.N) add4_f32(p, mr, n, v);
+          }
+          __syncwarp();
         }
-        __syncwarp();
       }
     }
   }
@@ -718,10 +757,10 @@ static int raster_group(const GemmParams& p, int row_tiles, int tile_m) {
   return (int)(g < row_tiles ? g : row_tiles);
 }
 
-template <int L, bool G>
+template <int L, bool G, bool ACC32 = false>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
-  auto kern = gemm_blockwise_kernel<L, G>;
+  auto kern = gemm_blockwise_kernel<L, G, ACC32>;
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -792,6 +831,12 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, int num_sms, cudaStream_t s) {
   if (p.recipe == kBlockwise) {
+    if (p.c32 != nullptr) {   // FP32 accumulate epilogue: its own instantiations
+      if (p.num_groups > 0) return launch_blockwise<kFprop, true, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      return launch_blockwise<kWgrad, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
+    }
     if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
     if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, num_sms, s);
     if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, num_sms, s);

@@ -69,7 +69,8 @@ struct GemmParams {
   int64_t ld_sb;
   const float* a_global;
   const float* b_global;
-  uint16_t* c;      // BF16 row-major
+  uint16_t* c;      // BF16 row-major (nullptr when accumulating into c32)
+  float* c32;       // BLOCKWISE FP32 accumulate target (C += A.B^T), else nullptr
   int64_t ldc;
   const uint8_t* sfa;  // MX / NVFP4: MMA-tiled scale images
   const uint8_t* sfb;

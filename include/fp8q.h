@@ -185,7 +185,8 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                                    fp8q_sf_layout sf_layout, void* stream);
 
 /* Arguments of fp8q_gemm_blockscaled: C[M x N] = A[M x K] . B[N x K]^T, both operands
- * K-major codes, C BF16 row-major (ldc >= N, ldc % 8 == 0, c 16-byte aligned).
+ * K-major codes, C BF16 row-major (ldc >= N, ldc % 8 == 0, c 16-byte aligned) unless
+ * c_fp32_accumulate is set (below).
  *   BLOCKWISE [DSV3] "Increased accumulation precision": for every 128-element K chunk the
  *     tensor cores form the E4M3 partial product in FP32 and CUDA cores add it into an
  *     FP32 accumulator with the chunk's scales applied:
@@ -204,7 +205,13 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
  *   (expert g at g * (N/128) * ld_sb floats).  The kernel reads the offsets on the device
  *   and builds its tile schedule there (at most M/128 + G row tiles), so the host needs
  *   no copy of them.
- * M, N >= 0 arbitrary (tails masked at the store). */
+ * M, N >= 0 arbitrary (tails masked at the store).
+ * c_fp32_accumulate (BLOCKWISE only; 0 for the other recipes): C is an FP32 row-major
+ *   matrix (ldc % 4 == 0, c 16-byte aligned) that is updated in place,
+ *     C[m,n] = fp32( C[m,n] + sum_kb ... )   (the FP32 sum above, before any BF16 rounding),
+ *   the FP32 main-gradient accumulation that follows wgrad in training ([DSV3]
+ *   "Mixed-precision framework": gradients and master weights stay in FP32).  K == 0
+ *   leaves C unchanged. */
 typedef struct {
   fp8q_recipe recipe;
   fp8q_layout layout;
@@ -221,6 +228,7 @@ typedef struct {
   int64_t ldc;
   const int32_t* m_offsets;
   int32_t num_groups;
+  int32_t c_fp32_accumulate;
 } fp8q_gemm_args;
 
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);

@@ -158,3 +158,9 @@ def test_grouped_weight_quantizer_validates_before_launching(L):
     assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 2, 128, 100, 128, ALIGNED, None, ALIGNED, s) == fq.FP8Q_ERR_SHAPE
     assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 2, 128, 128, 128, ALIGNED, None, None, s) == fq.FP8Q_ERR_NULL
     assert fq.fp8q_quantize_128x128_grouped(ALIGNED, 0, 128, 128, 128, ALIGNED, None, ALIGNED, s) == fq.FP8Q_OK
+
+
+def test_fp32_accumulate_is_blockwise_only_and_needs_ldc_multiple_of_4(L):
+    s = None
+    assert fq.fp8q_gemm_blockscaled(_args(recipe=fq.FP8Q_MXFP8, c_fp32_accumulate=1), s) == fq.FP8Q_ERR_UNSUPPORTED
+    assert fq.fp8q_gemm_blockscaled(_args(c_fp32_accumulate=1, ldc=258), s) == fq.FP8Q_ERR_SHAPE

@@ -87,6 +87,42 @@ def test_blockwise_dgrad(cuda_lib, M, Kw, Nw):
     check(c, ref, t, "dgrad")
 
 
+@pytest.mark.parametrize("layout", ["wgrad", "fprop"])
+def test_blockwise_fp32_accumulate(cuda_lib, layout):
+    """FP32 main-gradient update: C_out = fp32(C_in + A.B^T) with the FP32 sum unrounded to
+    BF16.  Checked elementwise: (C_out - C_in) against the oracle product within the GEMM
+    tolerance, plus half an FP32 ulp of C_out for the final addition."""
+    fq = cuda_lib
+    if layout == "wgrad":
+        T, Kf, N = 256, 208, 400                      # tokens, output rows (M), output cols
+        X, dY = bf((T, Kf), 1.0, 61, 1e-3, 50.0), bf((T, N), 1e-3, 62)
+        qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
+        qd = fq.quantize_1x128(dY.cuda(), rowwise=False, colwise=True)
+        a, b, sa, sb, L, ld_sb = qx["q_col"], qd["q_col"], qx["s_col"], qd["s_col"], fq.FP8Q_WGRAD, None
+        ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
+        od, osd = Q.quantize_1x128_colwise(workloads.bf16_bits(dY))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od, osd, G.WGRAD))
+        M = Kf
+    else:
+        M, K, N = 300, 384, 384
+        X, W = bf((M, K), 1.0, 63, 1e-3, 50.0), bf((K, N), 0.02, 64)
+        qx = fq.quantize_1x128(X.cuda())
+        qw = fq.quantize_128x128(W.cuda())
+        a, b, sa, sb, L, ld_sb = qx["q_row"], qw["q_t"], qx["s_row"], qw["s"], fq.FP8Q_FPROP, None
+        ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+        _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+    g = torch.Generator().manual_seed(65)
+    c_in = (torch.randn((M, N), generator=g, dtype=torch.float64) * float(np.abs(ref).mean() + 1e-30)).float()
+    c = c_in.cuda().clone()
+    fq.gemm(a, b, fq.FP8Q_BLOCKWISE, L, a_scale=sa, b_scale=sb, ld_sb=ld_sb, out=c, accumulate_fp32=True)
+    assert fq.device_status() == 0
+    got = host(c).astype(np.float64)
+    cin = c_in.numpy().astype(np.float64)
+    excess = G.tolerance_violation(got - cin, ref, t) - np.abs(got) * 2.0 ** -24
+    assert float(excess.max()) <= 0, f"{int((excess > 0).sum())} elements outside tolerance"
+
+
 @pytest.mark.parametrize("T,Kf,N", [(256, 208, 400), (1024, 256, 512)])
 def test_blockwise_wgrad(cuda_lib, T, Kf, N):
     """dW = X^T . dY: both operands 1x128 along tokens (colwise, transposed)."""
