@@ -10,6 +10,10 @@ the public format definitions:
 * E4M3 ("E4M3FN", OCP 8-bit floating point spec): 1 sign, 4 exponent (bias 7), 3 mantissa
   bits; no infinities; exponent 15 with mantissa 7 is NaN; largest finite value
   1.75 * 2^8 = 448; smallest subnormal 2^-9.
+* E5M2 (OCP 8-bit floating point spec), the gradient format of the delayed-scaling recipe's
+  comparison variant: 1 sign, 5 exponent (bias 15), 2 mantissa bits; exponent 31 holds
+  infinity (mantissa 0) and NaN; largest finite value 1.75 * 2^15 = 57344; smallest
+  subnormal 2^-16.
 * E8M0 (OCP MX spec v1.0): unsigned 8-bit exponent, value 2^(c - 127); code 255 is NaN.
 * E2M1 (OCP MX spec v1.0): 1 sign, 2 exponent (bias 1), 1 mantissa bit; values
   {0, 0.5, 1, 1.5, 2, 3, 4, 6}; no NaN or infinity.
@@ -22,6 +26,7 @@ maps to the maximum).  The sign of zero is kept.
 import numpy as np
 
 E4M3_MAX = 448.0
+E5M2_MAX = 57344.0
 E2M1_MAX = 6.0
 FLT_MAX = np.float32(np.finfo(np.float32).max)
 
@@ -87,6 +92,55 @@ def e4m3_encode_bruteforce(y):
         a = abs(v)
         if a >= E4M3_MAX:
             c = 0x7E
+        else:
+            d = np.abs(vals - a)
+            best = np.flatnonzero(d == d.min())
+            c = int(best[0]) if len(best) == 1 else int([b for b in best if b % 2 == 0][0])
+        out[i] = c | (0x80 if np.signbit(v) else 0)
+    return out
+
+
+# ----------------------------------------------------------------------------- E5M2
+def e5m2_decode(codes):
+    """E5M2 codes (uint8) -> float64 values; +-inf for exponent 31 / mantissa 0, NaN for the
+    other exponent-31 codes."""
+    c = np.asarray(codes, dtype=np.uint8).astype(np.int64)
+    s = (c >> 7) & 1
+    e = (c >> 2) & 0x1F
+    m = c & 3
+    mag = np.where(e == 0, (m / 4.0) * 2.0 ** -14, (1.0 + m / 4.0) * np.exp2(e - 15.0))
+    mag = np.where(e == 31, np.where(m == 0, np.inf, np.nan), mag)
+    return np.where(s == 1, -mag, mag)
+
+
+def e5m2_encode(y):
+    """float32 -> E5M2 code, round to nearest even, saturating at +-57344.
+
+    As for E4M3 with 2 mantissa bits: on the grid of exponent E (E >= -14; subnormals share
+    the 2^-16 quantum of E = -14) a magnitude is q * 2^(E-2) with q in [4, 8); code =
+    4*(E+15) + (q - 4); a carry to q = 8 lands on the next exponent's first code.  The
+    largest finite code is 0x7B; NaN -> 0x7F.
+    """
+    y = np.asarray(y, dtype=np.float32)
+    a = np.abs(y.astype(np.float64))
+    E = np.maximum(_exponent_floor(a), -14)
+    q = np.rint(a / np.exp2(E - 2.0))             # exact scaling, ties to even
+    code = 4 * (E + 15) + (q.astype(np.int64) - 4)
+    code = np.clip(code, 0, 0x7B)                 # satfinite: never infinity or NaN
+    code = np.where(np.isnan(y), 0x7F, code | (np.signbit(y).astype(np.int64) << 7))
+    return code.astype(np.uint8)
+
+
+def e5m2_encode_bruteforce(y):
+    """Reference encoder for small arrays: nearest finite E5M2 value, tie -> even code."""
+    y = np.asarray(y, dtype=np.float32).ravel()
+    pos = np.arange(0, 0x7C, dtype=np.uint8)      # 0x00..0x7B, all finite non-negative
+    vals = e5m2_decode(pos)
+    out = np.empty(y.shape, dtype=np.uint8)
+    for i, v in enumerate(y.astype(np.float64)):
+        a = abs(v)
+        if a >= E5M2_MAX:
+            c = 0x7B
         else:
             d = np.abs(vals - a)
             best = np.flatnonzero(d == d.min())

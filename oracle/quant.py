@@ -25,6 +25,10 @@ the design notes):
   1; overflow -> FLT_MAX).  Per 16 elements: sb = E4M3_RNE_SAT(fp32(fp32(amax_b / 6) *
   S_g)); enc = 0 if sb == 0 else fp32(S_g / decode(sb)); y = fp32(x * enc); q = E2M1 of y
   by round-to-nearest-even or by stochastic rounding; stored g_dec = fp32(1 / S_g).
+* Delayed (per-tensor, amax history; the recipe [DSV3] "Online quantization" contrasts
+  with): sf = fp32(fmt_max / max(history)) (max 0 -> 1, overflow -> FLT_MAX), fmt_max 448
+  for E4M3 or 57344 for E5M2; q = FMT_RNE_SAT(fp32(x * sf)); s = fp32(1 / sf); the
+  tensor's own amax is returned for the caller's history and does not affect its codes.
 * Stochastic rounding: a = |y|; a >= 6 -> 6; else lo <= a < hi adjacent E2M1 values,
   p = (a - lo) / (hi - lo) (exact in FP32); r = word (idx & 3) of Philox4x32-10 with
   counter (idx >> 2 low 32 bits, idx >> 2 high 32 bits, 0, tag) and key sr_seed, where
@@ -40,8 +44,8 @@ the original row index (the wgrad operands).
 """
 import numpy as np
 
-from .formats import (FLT_MAX, bf16_bits_to_f32, e2m1_encode_rne, e2m1_grid_neighbours,
-                      e4m3_decode, e4m3_encode, pack_e2m1)
+from .formats import (E4M3_MAX, E5M2_MAX, FLT_MAX, bf16_bits_to_f32, e2m1_encode_rne, e2m1_grid_neighbours,
+                      e4m3_decode, e4m3_encode, e5m2_encode, pack_e2m1)
 from .philox import philox4x32_10, seed_to_key
 from .rht import rht16_lastdim, rht_signs
 
@@ -143,6 +147,37 @@ def quantize_tensor(x):
     for r0, r1 in _row_chunks(R, C):
         q[r0:r1] = e4m3_encode((as_f32(x[r0:r1]) * sf).astype(np.float32))
     return q, np.float32(np.float32(1.0) / sf)
+
+
+# ------------------------------------------------------------ delayed scaling (history)
+def quantize_tensor_delayed(x, amax_history, fmt="e4m3"):
+    """Per-tensor delayed scaling, the recipe "Can you explain the role of FP8 precision in
+    DeepSeek-V3 training" (section "Online quantization") contrasts with its own: the scale
+    comes from the amaxes of previous iterations, not from the tensor being cast.
+
+    sf = fmt_max / max(amax_history) in FP32 (max 0 -> 1, overflow -> FLT_MAX); codes
+    fmt(x * sf) with saturation (values beyond the historical range clip); stored decode
+    scale fp32(1 / sf).  Also returns this tensor's amax, which the caller records in the
+    history for later iterations (it does not affect this cast).  fmt: "e4m3" (448) or
+    "e5m2" (57344).
+    """
+    x = np.asarray(x)
+    R, C = x.shape
+    fmax = np.float32(E4M3_MAX if fmt == "e4m3" else E5M2_MAX)
+    hmax = np.float32(np.max(np.asarray(amax_history, dtype=np.float32))) if np.size(amax_history) else np.float32(0)
+    with np.errstate(divide="ignore", over="ignore"):
+        sf = np.float32(1.0) if hmax == 0 else np.float32(fmax / hmax)
+    if np.isinf(sf):
+        sf = FLT_MAX
+    enc = e4m3_encode if fmt == "e4m3" else e5m2_encode
+    q = np.empty((R, C), dtype=np.uint8)
+    amax = np.float32(0.0)
+    for r0, r1 in _row_chunks(R, C):
+        xf = as_f32(x[r0:r1])
+        q[r0:r1] = enc((xf * sf).astype(np.float32))
+        if r1 > r0:
+            amax = max(amax, np.float32(np.max(np.abs(xf))))
+    return q, np.float32(np.float32(1.0) / sf), np.float32(amax)
 
 
 # ------------------------------------------------------------------- MX (E8M0, 32)

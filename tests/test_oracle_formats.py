@@ -139,3 +139,48 @@ def test_bf16_conversions_match_torch():
     bits = t.view(torch.int16).numpy().view(np.uint16)
     assert np.array_equal(F.f32_to_bf16_bits(x), bits)
     assert np.array_equal(F.bf16_bits_to_f32(bits), t.to(torch.float32).numpy())
+
+
+# ----------------------------------------------------------------------------- E5M2
+def test_e5m2_decode_matches_ml_dtypes_and_torch_all_codes():
+    ours = F.e5m2_decode(ALL8)
+    lib = ALL8.view(ml_dtypes.float8_e5m2).astype(np.float64)
+    tor = torch.from_numpy(ALL8.copy()).view(torch.float8_e5m2).to(torch.float64).numpy()
+    for ref in (lib, tor):
+        assert np.array_equal(np.isnan(ours), np.isnan(ref))
+        ok = ~np.isnan(ref)
+        assert np.array_equal(ours[ok], ref[ok])
+    # published extremes: largest finite 57344, infinity at 0x7C, smallest subnormal 2^-16
+    assert ours[0x7B] == 57344.0 and ours[0x7C] == np.inf and ours[0xFC] == -np.inf
+    assert ours[0x01] == 2.0 ** -16 and ours[0x04] == 2.0 ** -14
+
+
+def _e5m2_midpoints_and_neighbours():
+    pos = np.sort(F.e5m2_decode(np.arange(0x7C, dtype=np.uint8)))
+    mids = (pos[:-1] + pos[1:]) / 2
+    m32 = mids.astype(np.float32)
+    x = np.concatenate([pos.astype(np.float32), m32, np.nextafter(m32, np.float32(0)),
+                        np.nextafter(m32, np.float32(np.inf))])
+    x = np.concatenate([x, -x, np.float32([57345, 61439.9, 61440, 61440.1, 65536, 1e9, 3e38])])
+    return x.astype(np.float32)
+
+
+def test_e5m2_encode_roundtrip_every_finite_code():
+    vals = F.e5m2_decode(ALL8)
+    ok = np.isfinite(vals)
+    assert np.array_equal(F.e5m2_encode(vals[ok].astype(np.float32)), ALL8[ok])
+
+
+def test_e5m2_encode_bruteforce_midpoints_and_saturation():
+    x = _e5m2_midpoints_and_neighbours()
+    got = F.e5m2_encode(x)
+    assert np.array_equal(got, F.e5m2_encode_bruteforce(x))
+    assert np.all((got & 0x7F) <= 0x7B)            # satfinite: never infinity or NaN
+
+
+def test_e5m2_encode_matches_torch_in_range():
+    rng = np.random.default_rng(7)
+    x = (rng.standard_normal(20000) * np.exp2(rng.integers(-20, 14, 20000))).astype(np.float32)
+    x = x[np.abs(x) < 57344]
+    t = torch.from_numpy(x).to(torch.float8_e5m2).view(torch.uint8).numpy()
+    assert np.array_equal(F.e5m2_encode(x), t)

@@ -258,3 +258,40 @@ def test_sf_tiled_layout_is_a_permutation():
         assert np.count_nonzero(flat) == R * S
         rr, cc = np.meshgrid(np.arange(R), np.arange(S), indexing="ij")
         assert len(np.unique(Q.sf_tiled_offset(rr, cc, S))) == R * S
+
+
+# ----------------------------------------------------------------------------- delayed
+def test_delayed_with_own_amax_in_history_equals_current_scaling():
+    """History holding exactly this tensor's amax: delayed scaling reduces to current
+    (per-tensor) scaling, codes and decode scale identical."""
+    x = Q.as_f32(workloads.bf16_bits(workloads.tiny()["A"]))
+    q, s = Q.quantize_tensor(x)
+    amax = np.float32(np.max(np.abs(x)))
+    qd, sd, a = Q.quantize_tensor_delayed(x, np.float32([0.0, amax, amax / 3]))
+    assert np.array_equal(qd, q) and sd == s and a == amax
+
+
+def test_delayed_scale_from_history_max_and_saturation():
+    """The scale comes from the largest historical amax (a power of two here, so it is exact);
+    values beyond the history's range saturate; the returned amax is the tensor's own."""
+    rng = np.random.default_rng(11)
+    x = (rng.standard_normal((64, 96)) * 4.0).astype(np.float32)
+    x[3, 5] = 100.0                              # beyond the historical range
+    hist = np.float32([2.0, 7.0, 8.0, 0.0])      # max 8 -> sf = 448 / 8 = 56
+    q, s, a = Q.quantize_tensor_delayed(x, hist)
+    assert s == np.float32(1.0 / 56.0) and a == np.float32(100.0)
+    assert q[3, 5] == 0x7E                        # saturated at +448
+    assert np.array_equal(q, F.e4m3_encode_bruteforce((x * np.float32(56.0)).ravel()).reshape(x.shape))
+
+
+def test_delayed_e5m2_and_empty_history():
+    x = np.float32([[1.0, -2.0, 3.0, 0.5]])
+    q, s, a = Q.quantize_tensor_delayed(x, np.float32([0.0, 0.0]), fmt="e5m2")   # no history -> sf 1
+    assert s == np.float32(1.0) and a == np.float32(3.0)
+    assert np.array_equal(F.e5m2_decode(q).astype(np.float32), x)
+    q, s, _ = Q.quantize_tensor_delayed(x, np.float32([3584.0]), fmt="e5m2")      # sf = 57344 / 3584 = 16
+    assert s == np.float32(1.0 / 16.0)
+    assert np.array_equal(F.e5m2_decode(q) * float(s), x.astype(np.float64))
+    q, s, _ = Q.quantize_tensor_delayed(x, np.float32([4.0]), fmt="e5m2")         # sf = 14336, not exact
+    assert s == np.float32(np.float32(1.0) / np.float32(14336.0))
+    assert np.array_equal(q, F.e5m2_encode_bruteforce(x.ravel() * np.float32(14336.0)).reshape(x.shape))
