@@ -20,9 +20,10 @@ __all__ = [
     "FP8Q_FPROP", "FP8Q_DGRAD", "FP8Q_WGRAD", "FP8Q_SF_ROWMAJOR", "FP8Q_SF_MMA_TILED",
     "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
-    "fp8q_quantize_tensor_noalloc", "fp8q_quantize_128x128_grouped", "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
+    "fp8q_quantize_tensor_noalloc", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
+    "fp4q_rht16_quantize_sr", "FP8Q_E4M3", "FP8Q_E5M2", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
     "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
-    "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
+    "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_tensor_delayed", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
     "gemm", "device_status", "EXPORTED_SYMBOLS",
 ]
 
@@ -32,12 +33,13 @@ FP8Q_BLOCKWISE, FP8Q_MXFP8, FP8Q_PERTENSOR, FP8Q_NVFP4 = 0, 1, 2, 3
 FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD = 0, 1, 2
 FP8Q_SF_ROWMAJOR, FP8Q_SF_MMA_TILED = 0, 1
 FP4Q_ROW, FP4Q_COL = 1, 2
+FP8Q_E4M3, FP8Q_E5M2 = 0, 1
 
 EXPORTED_SYMBOLS = [
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
-    "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped",
+    "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -60,6 +62,7 @@ class GemmArgs(ctypes.Structure):
         ("c", ctypes.c_void_p), ("ldc", ctypes.c_int64),
         ("m_offsets", ctypes.c_void_p), ("num_groups", ctypes.c_int32),
         ("c_fp32_accumulate", ctypes.c_int32),
+        ("a_format", ctypes.c_int32), ("b_format", ctypes.c_int32),
     ]
 
 
@@ -81,6 +84,8 @@ def lib():
         L.fp8q_quantize_mx32.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_quantize_tensor.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
         L.fp8q_quantize_tensor_noalloc.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp]
+        L.fp8q_quantize_tensor_delayed.argtypes = [_vp, _i64, _i64, _i64, _vp, ctypes.c_int32, ctypes.c_int32, _int,
+                                                   _vp, _vp, _vp]
         L.fp4q_rht16_quantize_sr.argtypes = [_vp, _i64, _i64, _i64, _int, _u64, _int, _u64,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
@@ -99,7 +104,8 @@ def lib():
                                                      "fp8q_quantize_mx32", "fp8q_quantize_tensor",
                                                      "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
                                                      "fp8q_get_device_status", "fp8q_release_scratch",
-                                                     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped"):
+                                                     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped",
+                                                     "fp8q_quantize_tensor_delayed"):
                 f.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -146,6 +152,10 @@ def fp8q_quantize_mx32(x, rows, cols, ld_x, q_row, e_row, q_col, e_col, sf_layou
 
 def fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream):
     return lib().fp8q_quantize_tensor(x, rows, cols, ld_x, q, s_dec, stream)
+
+
+def fp8q_quantize_tensor_delayed(x, rows, cols, ld_x, hist, hlen, hpos, fmt, q, s_dec, stream):
+    return lib().fp8q_quantize_tensor_delayed(x, rows, cols, ld_x, hist, hlen, hpos, fmt, q, s_dec, stream)
 
 
 def fp8q_quantize_tensor_noalloc(x, rows, cols, ld_x, q, s_dec, stream):
@@ -276,6 +286,21 @@ def quantize_tensor(x, stream=None):
     return out
 
 
+def quantize_tensor_delayed(x, amax_history, history_pos, fmt=FP8Q_E4M3, stream=None):
+    """Per-tensor delayed scaling: scale from max(amax_history) (float32 CUDA tensor, updated
+    in place at history_pos with this tensor's amax).  Returns q (R, C) uint8, s_dec (1,)."""
+    _check_bf16(x)
+    if not (amax_history.is_cuda and amax_history.dtype == torch.float32 and amax_history.dim() == 1):
+        raise ValueError("amax_history must be a 1-D float32 CUDA tensor")
+    R, C = x.shape
+    out = {"q": torch.empty((R, C), dtype=torch.uint8, device=x.device),
+           "s_dec": torch.empty((1,), dtype=torch.float32, device=x.device)}
+    st = fp8q_quantize_tensor_delayed(_ptr(x), R, C, x.stride(0), _ptr(amax_history), amax_history.numel(),
+                                      history_pos, fmt, _ptr(out["q"]), _ptr(out["s_dec"]), _stream(stream))
+    _check(st, "fp8q_quantize_tensor_delayed")
+    return out
+
+
 def rht16_quantize_sr(x, rowwise=True, colwise=False, rht=0, rht_seed=0, sr=0, sr_seed=0,
                       sf_layout=FP8Q_SF_ROWMAJOR, stream=None):
     """NVFP4.  rht / sr are FP4Q_ROW | FP4Q_COL masks.  Returns q_row (R, C/2), sf_row,
@@ -301,7 +326,8 @@ def rht16_quantize_sr(x, rowwise=True, colwise=False, rht=0, rht_seed=0, sr=0, s
 
 
 def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
-         a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False, stream=None):
+         a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False,
+         a_format=0, b_format=0, stream=None):
     """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
     Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16.
     accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T."""
@@ -328,6 +354,7 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
     args.m_offsets = m_offsets.data_ptr() if grouped else None
     args.num_groups = (m_offsets.numel() - 1) if grouped else 0
     args.c_fp32_accumulate = 1 if accumulate_fp32 else 0
+    args.a_format, args.b_format = a_format, b_format
     _check(fp8q_gemm_blockscaled(args, _stream(stream)), "fp8q_gemm_blockscaled")
     return c
 

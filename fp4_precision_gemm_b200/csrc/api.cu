@@ -262,6 +262,25 @@ fp8q_status fp8q_quantize_tensor(const void* x, int64_t rows, int64_t cols, int6
   return from_cuda(e);
 }
 
+fp8q_status fp8q_quantize_tensor_delayed(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                         float* amax_history, int32_t history_len, int32_t history_pos,
+                                         fp8q_fp8_format fmt, uint8_t* q, float* s_dec, void* stream) {
+  fp8q_status st = check_input(x, rows, cols, ld_x);
+  if (st != FP8Q_OK) return st;
+  if (!q || !s_dec || !amax_history) return FP8Q_ERR_NULL;
+  if (fmt != FP8Q_E4M3 && fmt != FP8Q_E5M2) return FP8Q_ERR_UNSUPPORTED;
+  if (history_len < 1 || history_len > 1024 || history_pos < 0 || history_pos >= history_len) return FP8Q_ERR_SHAPE;
+  if (cols % 8 != 0) return FP8Q_ERR_SHAPE;
+  if (!aligned16(q)) return FP8Q_ERR_ALIGN;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceScratch* d = nullptr;
+  if ((st = scratch(&d)) != FP8Q_OK) return st;
+  uint32_t* amax = nullptr;
+  if ((st = amax_slot(d, s, &amax)) != FP8Q_OK) return st;
+  return from_cuda(launch_tensor_delayed(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax_history,
+                                         history_len, history_pos, fmt == FP8Q_E5M2, q, s_dec, amax, s));
+}
+
 fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, int64_t ld_x, int rht,
                                    uint64_t rht_seed, int sr, uint64_t sr_seed, uint8_t* q_row, uint8_t* sf_row,
                                    float* g_dec_row, uint8_t* q_col, uint8_t* sf_col, float* g_dec_col,
@@ -319,6 +338,8 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (a->M >= (1ll << 31) || a->N >= (1ll << 31) || a->K >= (1ll << 31)) return FP8Q_ERR_SHAPE;
   const bool acc32 = a->c_fp32_accumulate != 0;
   if (acc32 && a->recipe != FP8Q_BLOCKWISE) return FP8Q_ERR_UNSUPPORTED;
+  if (a->a_format < 0 || a->a_format > 1 || a->b_format < 0 || a->b_format > 1) return FP8Q_ERR_UNSUPPORTED;
+  if ((a->a_format || a->b_format) && a->recipe != FP8Q_PERTENSOR) return FP8Q_ERR_UNSUPPORTED;
   if (a->M == 0 || a->N == 0) return FP8Q_OK;
   if (!a->c) return FP8Q_ERR_NULL;
   if (a->ldc < a->N || a->ldc % (acc32 ? 4 : 8) != 0) return FP8Q_ERR_SHAPE;
@@ -350,6 +371,8 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   p.K = (int)a->K;
   p.c = acc32 ? nullptr : static_cast<uint16_t*>(a->c);
   p.c32 = acc32 ? static_cast<float*>(a->c) : nullptr;
+  p.a_fmt = a->a_format;
+  p.b_fmt = a->b_format;
   p.ldc = a->ldc;
   p.m_offsets = a->m_offsets;
   p.num_groups = a->num_groups;

@@ -39,6 +39,13 @@ __device__ __forceinline__ uint32_t cvt_e4m3x2(float lo, float hi) {
   return (uint32_t)r;
 }
 
+// Two FP32 values to E5M2 (round to nearest even, saturating at +-57344): lo in bits 0-7.
+__device__ __forceinline__ uint32_t cvt_e5m2x2(float lo, float hi) {
+  uint16_t r;
+  asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(hi), "f"(lo));
+  return (uint32_t)r;
+}
+
 // Tile scale: sf = 448 / amax (IEEE division); amax == 0 -> 1; overflow -> FLT_MAX.
 __device__ __forceinline__ float e4m3_sf(float amax) {
   if (amax == 0.0f) return 1.0f;

@@ -51,6 +51,10 @@ struct Fp4QuantParams {
   uint32_t* amax_bits;  // [0]: rowwise output's global amax, [1]: colwise output's
 };
 
+cudaError_t launch_tensor_delayed(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x, float* hist,
+                                  int hlen, int pos, bool e5m2, uint8_t* q, float* s_dec, uint32_t* amax_bits,
+                                  cudaStream_t s);
+
 cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 
@@ -79,6 +83,7 @@ struct GemmParams {
   int num_groups;
   int tiles_m, tiles_n;    // output tile grid (non-grouped)
   int group_m;             // raster: row tiles per column sweep (set by the launcher)
+  int a_fmt, b_fmt;        // PERTENSOR: element format of A / B (0 E4M3, 1 E5M2)
   uint32_t* status;        // device status word
 };
 

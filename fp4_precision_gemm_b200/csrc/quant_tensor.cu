@@ -5,6 +5,7 @@
 // on the FP32 bit pattern, which orders like the value for non-negative floats) and a cast.
 // Both are 2-D grids over (16-byte column chunks, rows) so no thread divides by the row
 // length; the row loop strides by gridDim.y.
+#include <cfloat>
 #include <mutex>
 
 #include "../../include/fp8q.h"
@@ -74,6 +75,78 @@ cudaError_t launch_tensor_cast(const uint16_t* x, int64_t rows, int64_t cols, in
                                const uint32_t* amax_bits, uint8_t* q, float* s_dec,
                                cudaStream_t s) {
   tensor_cast_kernel<<<tensor_grid(rows, cols), 256, 0, s>>>(x, rows, cols, ld_x, amax_bits, q, s_dec);
+  return cudaGetLastError();
+}
+
+// ------------------------------------------------------------------ delayed scaling
+// One pass: the scale comes from the largest amax of earlier iterations (the history), so
+// every CTA can cast as it reads; the tensor's own amax is reduced on the way (one
+// atomicMax per CTA into a scratch word) and recorded into the history by a one-thread
+// kernel afterwards, so no CTA reads a history slot while it is being replaced.
+template <bool E5M2>
+__global__ void __launch_bounds__(256) tensor_delayed_kernel(const uint16_t* __restrict__ x, int64_t rows,
+                                                             int64_t cols, int64_t ld_x, const float* hist, int hlen,
+                                                             uint8_t* q, float* s_dec, uint32_t* amax_bits) {
+  __shared__ float sf_sh;
+  __shared__ uint32_t red[8];
+  if (threadIdx.x < 32) {
+    float hm = 0.0f;
+    for (int i = threadIdx.x; i < hlen; i += 32) hm = fmaxf(hm, hist[i]);
+#pragma unroll
+    for (int s = 16; s > 0; s >>= 1) hm = fmaxf(hm, __shfl_xor_sync(0xFFFFFFFFu, hm, s));
+    if (threadIdx.x == 0) {
+      float sf = 1.0f;
+      if (hm > 0.0f) {
+        sf = __fdiv_rn(E5M2 ? 57344.0f : 448.0f, hm);
+        if (sf > FLT_MAX) sf = FLT_MAX;
+      }
+      sf_sh = sf;
+    }
+  }
+  __syncthreads();
+  const float sf = sf_sh;
+  if (blockIdx.x == 0 && blockIdx.y == 0 && threadIdx.x == 0) *s_dec = __frcp_rn(sf);
+  const int64_t c8 = (int64_t)blockIdx.x * blockDim.x + threadIdx.x;
+  uint32_t m = 0;
+  if (c8 * 8 < cols) {
+    for (int64_t r = blockIdx.y; r < rows; r += gridDim.y) {
+      const uint4 v = ldg_nc_v4(x + r * ld_x + c8 * 8);
+      m = max2(m, max2(max2(abs2(v.x), abs2(v.y)), max2(abs2(v.z), abs2(v.w))));
+      const uint32_t w[4] = {v.x, v.y, v.z, v.w};
+      uint32_t c[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        const float a = __fmul_rn(bf16_lo(w[i]), sf), b = __fmul_rn(bf16_hi(w[i]), sf);
+        c[i] = E5M2 ? cvt_e5m2x2(a, b) : cvt_e4m3x2(a, b);
+      }
+      *(uint2*)(q + r * cols + c8 * 8) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
+    }
+  }
+  m = hmax(m);
+#pragma unroll
+  for (int s = 16; s > 0; s >>= 1) m = max(m, __shfl_xor_sync(0xFFFFFFFFu, m, s));
+  if ((threadIdx.x & 31) == 0) red[threadIdx.x >> 5] = m;
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    uint32_t b = red[0];
+    for (int w = 1; w < (int)(blockDim.x >> 5); ++w) b = max(b, red[w]);
+    if (b) atomicMax(amax_bits, b << 16);
+  }
+}
+
+__global__ void tensor_delayed_record(const uint32_t* amax_bits, float* hist, int pos) {
+  hist[pos] = __uint_as_float(*amax_bits);
+}
+
+cudaError_t launch_tensor_delayed(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x, float* hist,
+                                  int hlen, int pos, bool e5m2, uint8_t* q, float* s_dec, uint32_t* amax_bits,
+                                  cudaStream_t s) {
+  const dim3 grid = (rows > 0 && cols > 0) ? tensor_grid(rows, cols) : dim3(1, 1);
+  if (e5m2) tensor_delayed_kernel<true><<<grid, 256, 0, s>>>(x, rows, cols, ld_x, hist, hlen, q, s_dec, amax_bits);
+  else tensor_delayed_kernel<false><<<grid, 256, 0, s>>>(x, rows, cols, ld_x, hist, hlen, q, s_dec, amax_bits);
+  cudaError_t e = cudaGetLastError();
+  if (e != cudaSuccess) return e;
+  tensor_delayed_record<<<1, 1, 0, s>>>(amax_bits, hist, pos);
   return cudaGetLastError();
 }
 

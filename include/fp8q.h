@@ -80,6 +80,12 @@ typedef enum {
   FP8Q_WGRAD = 2   /* B = dY^T (N x K codes, K = tokens); sb[(k/128) * ld_sb + n] (1x128)*/
 } fp8q_layout;
 
+/* FP8 element format of a per-tensor operand (OCP 8-bit floating point). */
+typedef enum {
+  FP8Q_E4M3 = 0,  /* max 448, the format of every other call                            */
+  FP8Q_E5M2 = 1   /* max 57344, the gradient format of the delayed-scaling comparison  */
+} fp8q_fp8_format;
+
 /* NVFP4 per-direction flags for `rht` and `sr`. */
 #define FP4Q_ROW 1  /* apply to the rowwise output (quantized along columns)           */
 #define FP4Q_COL 2  /* apply to the colwise output (quantized along rows, transposed)  */
@@ -136,6 +142,20 @@ fp8q_status fp8q_quantize_mx32(const void* x, int64_t rows, int64_t cols, int64_
  * Two kernels (amax, cast) on `stream`; the amax lives in the library's scratch pool. */
 fp8q_status fp8q_quantize_tensor(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
                                  uint8_t* q, float* s_dec, void* stream);
+
+/* Per-tensor DELAYED scaling, the recipe [DSV3] "Online quantization" contrasts with its
+ * own: the scale comes from the amaxes of earlier iterations instead of the tensor being
+ * cast, so one pass over x both casts and measures.
+ *   amax_history: device float[history_len] (1 <= history_len <= 1024), non-negative;
+ *   sf = fmt_max / max(amax_history) (FP32 IEEE division; max 0 -> 1; overflow -> FLT_MAX),
+ *   fmt_max = 448 (FP8Q_E4M3) or 57344 (FP8Q_E5M2); codes q[r * cols + c] =
+ *   fmt(x * sf) rounded to nearest even and saturated (values beyond the historical range
+ *   clip); *s_dec = fp32(1 / sf).  After the cast this tensor's amax is written to
+ *   amax_history[history_pos] (0 <= history_pos < history_len; the caller rotates it),
+ *   so it takes effect from the next call.  cols % 8 == 0. */
+fp8q_status fp8q_quantize_tensor_delayed(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                                         float* amax_history, int32_t history_len, int32_t history_pos,
+                                         fp8q_fp8_format fmt, uint8_t* q, float* s_dec, void* stream);
 
 /* Allocation-free variant of fp8q_quantize_tensor (no counterpart in the pages: it is a
  * library-integration entry point, not part of the method).  Same arguments, rules and
@@ -194,7 +214,9 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
  *     sb by `layout`.  K % 128 == 0.  a_scale/b_scale are float*.
  *   MXFP8: codes E4M3, scales E8M0 in FP8Q_SF_MMA_TILED layout for (M, K/32) and
  *     (N, K/32), applied by the hardware.  K % 32 == 0.
- *   PERTENSOR: codes E4M3; C = (*a_global) * (*b_global) * (A . B^T).  K % 16 == 0.
+ *   PERTENSOR: codes E4M3, or E5M2 per operand (a_format / b_format, e.g. an E5M2
+ *     gradient times E4M3 weights in dgrad); C = (*a_global) * (*b_global) * (A . B^T).
+ *     K % 16 == 0.
  *   NVFP4: packed E2M1 (lda/ldb in BYTES, K/2 bytes per row), E4M3 scales in
  *     FP8Q_SF_MMA_TILED layout for (M, K/16) and (N, K/16), C scaled by
  *     (*a_global) * (*b_global).  K % 32 == 0.
@@ -229,6 +251,7 @@ typedef struct {
   const int32_t* m_offsets;
   int32_t num_groups;
   int32_t c_fp32_accumulate;
+  int32_t a_format, b_format;   /* fp8q_fp8_format of A / B codes (PERTENSOR; else 0) */
 } fp8q_gemm_args;
 
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);

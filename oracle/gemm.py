@@ -21,7 +21,7 @@ Operand conventions (both K-major, C = A . B^T, C row-major M x N):
 """
 import numpy as np
 
-from .formats import e2m1_decode, e4m3_decode, e8m0_decode, unpack_e2m1
+from .formats import e2m1_decode, e4m3_decode, e5m2_decode, e8m0_decode, unpack_e2m1
 
 FPROP, DGRAD, WGRAD = 0, 1, 2
 TOL_REL = 2.0 ** -7
@@ -64,10 +64,11 @@ def dequant_mx(q, e8m0, rows=None):
                                             axis=1)[:, :K]
 
 
-def dequant_tensor(q, s, rows=None):
+def dequant_tensor(q, s, rows=None, fmt="e4m3"):
+    """Per-tensor operand: X_dq = fmt(q) * s (FP64); fmt "e4m3" or "e5m2"."""
     q = np.asarray(q)
     rows = np.arange(q.shape[0]) if rows is None else np.asarray(rows)
-    return e4m3_decode(q[rows]) * float(s)
+    return (e4m3_decode(q[rows]) if fmt == "e4m3" else e5m2_decode(q[rows])) * float(s)
 
 
 def dequant_nvfp4(packed, sf, g_dec, rows=None):

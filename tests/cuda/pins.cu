@@ -2,7 +2,7 @@
 //   * cuRAND's Philox4x32-10 (curand_Philox4x32_10) on given counters and keys, so the
 //     oracle's Philox can be checked word for word against CUDA's outputs;
 //   * the conversion instructions the quantize kernels rely on, on arbitrary FP32 inputs,
-//     so the oracle's E4M3 / E2M1 encoders can be checked against the hardware.
+//     so the oracle's E4M3 / E5M2 / E2M1 encoders can be checked against the hardware.
 #include <cstdint>
 #include <cuda_runtime.h>
 #include <curand_kernel.h>
@@ -17,6 +17,15 @@ __global__ void cvt_e4m3_kernel(const float* x, uint8_t* out, int n) {
   if (i < n) {
     uint16_t r;
     asm("cvt.rn.satfinite.e4m3x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x[i]));
+    out[i] = (uint8_t)(r & 0xFF);
+  }
+}
+
+__global__ void cvt_e5m2_kernel(const float* x, uint8_t* out, int n) {
+  int i = blockIdx.x * blockDim.x + threadIdx.x;
+  if (i < n) {
+    uint16_t r;
+    asm("cvt.rn.satfinite.e5m2x2.f32 %0, %1, %2;" : "=h"(r) : "f"(0.0f), "f"(x[i]));
     out[i] = (uint8_t)(r & 0xFF);
   }
 }
@@ -39,6 +48,10 @@ int pins_curand_philox(const void* ctr, const void* key, void* out, int n, void*
 }
 int pins_cvt_e4m3(const void* x, void* out, int n, void* stream) {
   cvt_e4m3_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>((const float*)x, (uint8_t*)out, n);
+  return (int)cudaGetLastError();
+}
+int pins_cvt_e5m2(const void* x, void* out, int n, void* stream) {
+  cvt_e5m2_kernel<<<(n + 255) / 256, 256, 0, (cudaStream_t)stream>>>((const float*)x, (uint8_t*)out, n);
   return (int)cudaGetLastError();
 }
 int pins_cvt_e2m1(const void* x, void* out, int n, void* stream) {

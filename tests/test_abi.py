@@ -164,3 +164,15 @@ def test_fp32_accumulate_is_blockwise_only_and_needs_ldc_multiple_of_4(L):
     s = None
     assert fq.fp8q_gemm_blockscaled(_args(recipe=fq.FP8Q_MXFP8, c_fp32_accumulate=1), s) == fq.FP8Q_ERR_UNSUPPORTED
     assert fq.fp8q_gemm_blockscaled(_args(c_fp32_accumulate=1, ldc=258), s) == fq.FP8Q_ERR_SHAPE
+
+
+def test_delayed_quantizer_and_fp8_format_validation(L):
+    s = None
+    f = fq.fp8q_quantize_tensor_delayed
+    assert f(ALIGNED, 8, 16, 16, ALIGNED, 0, 0, 0, ALIGNED, ALIGNED, s) == fq.FP8Q_ERR_SHAPE       # no history
+    assert f(ALIGNED, 8, 16, 16, ALIGNED, 4, 4, 0, ALIGNED, ALIGNED, s) == fq.FP8Q_ERR_SHAPE       # pos out of range
+    assert f(ALIGNED, 8, 16, 16, ALIGNED, 4, 0, 2, ALIGNED, ALIGNED, s) == fq.FP8Q_ERR_UNSUPPORTED # format
+    assert f(ALIGNED, 8, 16, 16, None, 4, 0, 0, ALIGNED, ALIGNED, s) == fq.FP8Q_ERR_NULL
+    g = fq.fp8q_gemm_blockscaled
+    assert g(_args(a_format=1), s) == fq.FP8Q_ERR_UNSUPPORTED          # E5M2 is per-tensor only
+    assert g(_args(recipe=fq.FP8Q_PERTENSOR, b_format=3), s) == fq.FP8Q_ERR_UNSUPPORTED

@@ -206,6 +206,25 @@ def test_per_tensor(cuda_lib, M, K, N):
     check(c, ref, t, "per-tensor")
 
 
+def test_per_tensor_e5m2_gradient_times_e4m3_weights(cuda_lib):
+    """dgrad of the delayed-scaling recipe: an E5M2 gradient (A) times E4M3 weights (B),
+    per-tensor scales, against the FP64 product of the dequantized operands."""
+    fq = cuda_lib
+    M, K, N = 300, 512, 400
+    dY, W = bf((M, K), 1e-3, 81, 5e-4, 100.0), bf((N, K), 0.02, 82)
+    ha = torch.tensor([0.0], dtype=torch.float32, device="cuda")
+    hb = torch.tensor([0.0], dtype=torch.float32, device="cuda")
+    fq.quantize_tensor_delayed(dY.cuda(), ha, 0, fq.FP8Q_E5M2)        # records the amaxes
+    fq.quantize_tensor_delayed(W.cuda(), hb, 0, fq.FP8Q_E4M3)
+    qa = fq.quantize_tensor_delayed(dY.cuda(), ha, 0, fq.FP8Q_E5M2)   # scaled by them
+    qb = fq.quantize_tensor_delayed(W.cuda(), hb, 0, fq.FP8Q_E4M3)
+    c = fq.gemm(qa["q"], qb["q"], fq.FP8Q_PERTENSOR, a_global=qa["s_dec"], b_global=qb["s_dec"], a_format=fq.FP8Q_E5M2)
+    assert fq.device_status() == 0
+    ref, t = G.reference(G.dequant_tensor(host(qa["q"]), host(qa["s_dec"])[0], fmt="e5m2"),
+                         G.dequant_tensor(host(qb["q"]), host(qb["s_dec"])[0]))
+    check(c, ref, t, "per-tensor e5m2 x e4m3")
+
+
 @pytest.mark.parametrize("M,K,N,rht", [(300, 512, 400, False), (256, 1024, 256, True)])
 def test_nvfp4(cuda_lib, M, K, N, rht):
     fq = cuda_lib

@@ -25,7 +25,7 @@ def pins():
     if not os.path.exists(PINS):
         pytest.fail("tests/cuda/libpins.so missing: run __graft_entry__.build()")
     L = ctypes.CDLL(PINS)
-    for f in ("pins_curand_philox", "pins_cvt_e4m3", "pins_cvt_e2m1"):
+    for f in ("pins_curand_philox", "pins_cvt_e4m3", "pins_cvt_e5m2", "pins_cvt_e2m1"):
         getattr(L, f).restype = ctypes.c_int
     return L
 
@@ -94,5 +94,27 @@ def test_e2m1_cvt_matches_oracle(pins):
     got = _cvt(pins, "pins_cvt_e2m1", x)
     want = F.e2m1_encode_rne(x)
     # compare magnitudes and signs separately so a -0 convention difference is visible
+    bad = np.flatnonzero(got != want)
+    assert bad.size == 0, f"{bad.size} mismatches, e.g. x={x[bad[:5]]} hw={got[bad[:5]]} oracle={want[bad[:5]]}"
+
+
+@pytest.mark.gpu
+def test_e5m2_cvt_matches_oracle(pins):
+    """The oracle's E5M2 encoder equals cvt.rn.satfinite.e5m2x2.f32 on every BF16 value in
+    range, every rounding midpoint and its neighbours, random FP32 bit patterns and the
+    saturation region."""
+    bf = np.arange(1 << 16, dtype=np.uint16)
+    x_bf = F.bf16_bits_to_f32(bf)
+    x_bf = x_bf[np.isfinite(x_bf)]
+    pos = np.sort(F.e5m2_decode(np.arange(0x7C, dtype=np.uint8))).astype(np.float32)
+    mids = ((pos[:-1].astype(np.float64) + pos[1:]) / 2).astype(np.float32)
+    around = np.concatenate([mids, np.nextafter(mids, np.float32(0)), np.nextafter(mids, np.float32(1e30))])
+    rng = np.random.default_rng(8)
+    bits = rng.integers(0, 1 << 32, 1 << 22, dtype=np.uint64).astype(np.uint32)
+    x_rand = bits.view(np.float32)
+    x_rand = x_rand[np.isfinite(x_rand)]
+    x = np.concatenate([x_bf, around, -around, x_rand, np.float32([0.0, -0.0, 57344, 61440, 1e30, -1e30])])
+    got = _cvt(pins, "pins_cvt_e5m2", x)
+    want = F.e5m2_encode(x)
     bad = np.flatnonzero(got != want)
     assert bad.size == 0, f"{bad.size} mismatches, e.g. x={x[bad[:5]]} hw={got[bad[:5]]} oracle={want[bad[:5]]}"

@@ -257,3 +257,24 @@ def test_nvfp4_gradient_fullsize_sampled(cuda_lib):
     nsf = bits.shape[0] // 16
     rr, cc = np.meshgrid(cols, np.arange(nsf), indexing="ij")
     assert np.array_equal(tiled[Q.sf_tiled_offset(rr, cc, nsf)], sf)
+
+
+@pytest.mark.parametrize("fmt", ["e4m3", "e5m2"])
+def test_tensor_delayed_parity_and_history(cuda_lib, fmt):
+    """Delayed scaling over two iterations: codes and decode scale bit-exact with the oracle
+    for the history given, and the tensor's amax recorded into the history slot."""
+    fq = cuda_lib
+    f = fq.FP8Q_E4M3 if fmt == "e4m3" else fq.FP8Q_E5M2
+    x1 = workloads.normal_bf16((300, 648), 1.0, 71, 1e-3, 50.0)
+    x2 = workloads.normal_bf16((300, 648), 3.0, 72, 1e-3, 50.0)     # wider than the history
+    hist = torch.tensor([0.0, 20.0, 5.0, 0.0], dtype=torch.float32, device="cuda")
+    h_host = hist.cpu().numpy().copy()
+    for x, pos in ((x1, 1), (x2, 3)):
+        out = fq.quantize_tensor_delayed(x.cuda(), hist, pos, f)
+        assert fq.device_status() == 0
+        xb = workloads.bf16_bits(x)
+        oq, os_, oa = Q.quantize_tensor_delayed(xb, h_host, fmt)
+        assert np.array_equal(out["q"].cpu().numpy(), oq)
+        assert out["s_dec"].cpu().numpy().view(np.uint32)[0] == np.float32(os_).view(np.uint32)
+        h_host[pos] = oa
+        assert np.array_equal(hist.cpu().numpy().view(np.uint32), h_host.view(np.uint32))
