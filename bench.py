@@ -286,6 +286,102 @@ class WgradAccStep:
                           "inputs, FP64 reference product")
 
 
+class DelayedStep:
+    """Per-tensor delayed scaling (amax history of 16 steps, rotated each step) on the
+    Llama-3-8B up-projection: fprop X . W^T with E4M3 operands, dgrad dY . W with an E5M2
+    gradient and E4M3 weights.  Each quantizer is one pass over its tensor."""
+    name = "delayed"
+    workload = ("llama3-8b up-proj, per-tensor delayed scaling (history 16): fprop X 8192x4096 e4m3 . W^T, "
+                "dgrad dY 8192x14336 e5m2 . W e4m3")
+    H = 16
+
+    def __init__(self, fq, rank, M=8192, K=4096, N=14336):
+        self.fq, self.M, self.K, self.N = fq, M, K, N
+        d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
+        self.X, self.W, self.dY = d["X"], d["W"], d["dY"]
+        self.Wt = self.W.t().contiguous()                     # N x K, the fprop B operand
+        dev = self.X.device
+        u8, f32 = torch.uint8, torch.float32
+        self.hist = {k: torch.zeros(self.H, dtype=f32, device=dev) for k in ("x", "wt", "dy", "w")}
+        self.q = {"x": torch.empty((M, K), dtype=u8, device=dev), "wt": torch.empty((N, K), dtype=u8, device=dev),
+                  "dy": torch.empty((M, N), dtype=u8, device=dev), "w": torch.empty((K, N), dtype=u8, device=dev)}
+        self.s = {k: torch.empty((1,), dtype=f32, device=dev) for k in self.q}
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty((M, K), dtype=torch.bfloat16, device=dev)
+        self.step = 0
+        self.gemm_flop = 2 * 2.0 * M * N * K
+
+    def inputs(self):
+        return [self.X, self.W, self.dY]
+
+    def outputs(self):
+        return [self.Y, self.dX]
+
+    def launches(self):
+        fq = self.fq
+        P = lambda t: t.data_ptr()  # noqa: E731
+        src = {"x": self.X, "wt": self.Wt, "dy": self.dY, "w": self.W}
+        fmt = {"x": fq.FP8Q_E4M3, "wt": fq.FP8Q_E4M3, "dy": fq.FP8Q_E5M2, "w": fq.FP8Q_E4M3}
+
+        def quant(k):
+            def f():
+                x = src[k]
+                pos = self.step % self.H
+                if k == "w":
+                    self.step += 1                            # last quantizer of the step
+                assert fq.fp8q_quantize_tensor_delayed(P(x), x.shape[0], x.shape[1], x.stride(0), P(self.hist[k]),
+                                                       self.H, pos, fmt[k], P(self.q[k]), P(self.s[k]),
+                                                       fq._stream()) == 0
+            return f
+
+        def fprop():
+            fq.gemm(self.q["x"], self.q["wt"], fq.FP8Q_PERTENSOR, a_global=self.s["x"], b_global=self.s["wt"],
+                    out=self.Y)
+
+        def dgrad():
+            fq.gemm(self.q["dy"], self.q["w"], fq.FP8Q_PERTENSOR, a_global=self.s["dy"], b_global=self.s["w"],
+                    out=self.dX, a_format=fq.FP8Q_E5M2)
+
+        M, K, N = self.M, self.K, self.N
+        return [Launch("quantize_tensor_delayed X e4m3", quant("x"), "quantize", bytes_=M * K * 3.0),
+                Launch("quantize_tensor_delayed W^T e4m3", quant("wt"), "quantize", bytes_=N * K * 3.0),
+                Launch("gemm per-tensor fprop e4m3", fprop, "gemm_pertensor", flop=2.0 * M * N * K),
+                Launch("quantize_tensor_delayed dY e5m2", quant("dy"), "quantize", bytes_=M * N * 3.0),
+                Launch("quantize_tensor_delayed W e4m3", quant("w"), "quantize", bytes_=K * N * 3.0),
+                Launch("gemm per-tensor dgrad e5m2 x e4m3", dgrad, "gemm_pertensor", flop=2.0 * M * N * K)]
+
+    def launch_count(self):
+        return 4 * 2 + 2
+
+    def cpu_sample(self, tiles=1):
+        """Oracle on a bounded sample: the rows of `tiles` sampled 128x128 output tiles of each
+        GEMM, quantized with the current histories (rows are independent under delayed
+        scaling), then the FP64 reference tiles."""
+        from oracle import gemm as G
+        from oracle import quant as Q
+        M, K, N = self.M, self.K, self.N
+        if not hasattr(self, "_host_bits"):
+            self._host_bits = tuple(workloads.bf16_bits(t) for t in (self.X, self.Wt, self.dY, self.W))
+            self._host_hist = {k: v.cpu().numpy() for k, v in self.hist.items()}
+        Xb, Wtb, dYb, Wb = self._host_bits
+        h = self._host_hist
+        t0 = time.perf_counter()
+        flop = 0.0
+        for m0, n0 in G.sample_tiles(M, N, tiles, seed=6):
+            qa, sa, _ = Q.quantize_tensor_delayed(Xb[m0:m0 + 128], h["x"])
+            qb, sb, _ = Q.quantize_tensor_delayed(Wtb[n0:n0 + 128], h["wt"])
+            G.reference(G.dequant_tensor(qa, sa), G.dequant_tensor(qb, sb))
+            flop += 2.0 * 128 * 128 * K
+        for m0, n0 in G.sample_tiles(M, K, tiles, seed=7):
+            qa, sa, _ = Q.quantize_tensor_delayed(dYb[m0:m0 + 128], h["dy"], fmt="e5m2")
+            qb, sb, _ = Q.quantize_tensor_delayed(Wb[n0:n0 + 128], h["w"])
+            G.reference(G.dequant_tensor(qa, sa, fmt="e5m2"), G.dequant_tensor(qb, sb))
+            flop += 2.0 * 128 * 128 * N
+        dt = time.perf_counter() - t0
+        return flop, dt, (f"{tiles} sampled 128x128 output tile(s) of fprop and dgrad, rows quantized by the oracle "
+                          "with the step's amax histories, FP64 reference product")
+
+
 class MxStep:
     name = "mxfp8"
     workload = "MXFP8 (and per-tensor) GEMMs (M,K,N) = (8192,4096,4096), (8192,4096,14336), (8192,14336,4096)"
@@ -512,7 +608,7 @@ class Nvfp4Step:
 
 
 STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step,
-         "wgrad_acc": WgradAccStep}
+         "wgrad_acc": WgradAccStep, "delayed": DelayedStep}
 
 
 # ============================================================================ measurement
