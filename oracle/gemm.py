@@ -101,6 +101,18 @@ def sample_tiles(M, N, n_tiles=64, seed=0, tile=128):
     return [(int(p // tn) * tile, int(p % tn) * tile) for p in sorted(pick)]
 
 
+def sample_band_tiles(M, N, n_row_bands=8, n_col_bands=8, seed=0, tile=128):
+    """Every pairing of n_row_bands distinct random row bands with n_col_bands distinct
+    random column bands (drawn with default_rng(seed + 2000)): n_row_bands * n_col_bands
+    distinct (m0, n0) tiles whose operand bands are few, for operands that are costly to
+    quantize band by band."""
+    tm, tn = -(-M // tile), -(-N // tile)
+    rng = np.random.default_rng(seed + 2000)
+    rb = np.sort(rng.choice(tm, size=min(n_row_bands, tm), replace=False))
+    cb = np.sort(rng.choice(tn, size=min(n_col_bands, tn), replace=False))
+    return [(int(r) * tile, int(c) * tile) for r in rb for c in cb]
+
+
 def sample_group_tiles(m_offsets, N, n_tiles=64, seed=0, tile=128):
     """Tiles across experts in proportion to their row counts, at least one per
     non-empty expert when n_tiles allows.  Returns (group, m0_global, m1_global, n0)."""

@@ -25,6 +25,9 @@ the design notes):
   1; overflow -> FLT_MAX).  Per 16 elements: sb = E4M3_RNE_SAT(fp32(fp32(amax_b / 6) *
   S_g)); enc = 0 if sb == 0 else fp32(S_g / decode(sb)); y = fp32(x * enc); q = E2M1 of y
   by round-to-nearest-even or by stochastic rounding; stored g_dec = fp32(1 / S_g).
+* NVFP4 weights for the forward path: one E4M3 scale per 16x16 block, from the amax over
+  its 256 elements by the same formula, round-to-nearest-even codes, emitted rowwise and
+  colwise (the same codes transposed), so fprop and dgrad read one quantized matrix.
 * Delayed (per-tensor, amax history; the recipe [DSV3] "Online quantization" contrasts
   with): sf = fp32(fmt_max / max(history)) (max 0 -> 1, overflow -> FLT_MAX), fmt_max 448
   for E4M3 or 57344 for E5M2; q = FMT_RNE_SAT(fp32(x * sf)); s = fp32(1 / sf); the
@@ -317,6 +320,46 @@ def quantize_nvfp4_colwise(x, rht=False, rht_seed=0, sr=False, sr_seed=0, rows=N
     """NVFP4 along rows (tokens), output transposed (C, R/2 packed), tag 1 for SR."""
     return quantize_nvfp4_rowwise(np.ascontiguousarray(np.asarray(x).T), rht, rht_seed,
                                   sr, sr_seed, tag=1, rows=rows)
+
+
+def quantize_nvfp4_2d(x, amax=None):
+    """NVFP4 weights with one E4M3 scale per 16x16 block, emitted in both operand layouts.
+
+    [NVFP4] "How it works" fixes the per-16 E4M3 scales and the per-tensor FP32 scale but
+    not how a weight tensor serves both the forward GEMM (quantized along one axis) and the
+    backward-data GEMM (along the other).  Reading taken: the 16 x 16 elements of a block
+    share one scale, computed as for a 16-element group with the amax over all 256, and the
+    codes are round-to-nearest-even (no transform, no stochastic rounding: these are
+    weights, not gradient inputs).  The rowwise and colwise outputs then hold the same codes
+    transposed, so both dequantize to one matrix.
+
+    x: (R, C) with R % 16 == C % 16 == 0; ``amax`` (optional) is the global amax G when x
+    is a 16-aligned sub-rectangle of a larger tensor (sampled checks).
+    Returns q_row (R, C/2), sf_row (R, C/16), q_col (C, R/2), sf_col (C, R/16) (E4M3
+    scale codes, row-major, each block's code repeated over its 16 rows or columns) and
+    g_dec = fp32(1 / S_g).
+    """
+    v = as_f32(x)
+    R, C = v.shape
+    assert R % 16 == 0 and C % 16 == 0
+    G = np.float32(np.max(np.abs(v))) if amax is None else np.float32(amax)
+    if R * C == 0:
+        G = np.float32(0.0) if amax is None else G
+    S_g = nvfp4_global_scale(G)
+    blocks = v.reshape(R // 16, 16, C // 16, 16)
+    amax_b = np.max(np.abs(blocks), axis=(1, 3)) if R * C else np.zeros((R // 16, C // 16), np.float32)
+    sb = e4m3_encode(((amax_b / np.float32(6.0)).astype(np.float32) * S_g).astype(np.float32))
+    dec = e4m3_decode(sb).astype(np.float32)
+    with np.errstate(divide="ignore"):
+        enc = np.where(sb == 0, np.float32(0.0),
+                       (S_g / np.where(sb == 0, np.float32(1.0), dec)).astype(np.float32)).astype(np.float32)
+    y = (blocks * enc[:, None, :, None]).astype(np.float32).reshape(R, C)
+    codes = e2m1_encode_rne(y)
+    q_row = pack_e2m1(codes)
+    q_col = pack_e2m1(np.ascontiguousarray(codes.T))
+    sf_row = np.repeat(sb, 16, axis=0).astype(np.uint8)
+    sf_col = np.repeat(np.ascontiguousarray(sb.T), 16, axis=0).astype(np.uint8)
+    return q_row, sf_row, q_col, sf_col, np.float32(np.float32(1.0) / S_g)
 
 
 # ------------------------------------------------------------------- scale layouts

@@ -292,6 +292,8 @@ def test_llama8b_fprop_dgrad_wgrad_sampled(cuda_lib):
 
 
 def test_mxfp8_and_per_tensor_fullsize_sampled(cuda_lib):
+    """MXFP8 and per-tensor current-scaling GEMMs at the three Llama-3-8B attention/MLP shapes,
+    64 sampled output tiles each."""
     fq = cuda_lib
     d = workloads.mxfp8(device="cuda")
     for i, (M, K, N) in enumerate(workloads.MXFP8_GEMMS):
@@ -301,23 +303,23 @@ def test_mxfp8_and_per_tensor_fullsize_sampled(cuda_lib):
         c = host(fq.gemm(qa["q_row"], qb["q_col"], fq.FP8Q_MXFP8, a_scale=qa["e8m0_row"],
                          b_scale=qb["e8m0_col"]).float())
         Ab, Wb = workloads.bf16_bits(A), workloads.bf16_bits(W)
-        for m0, n0 in _tiles(M, N, 10 + i)[:16]:
+        for m0, n0 in _tiles(M, N, 10 + i):
             oa, ea = Q.quantize_mx_rowwise(Ab[m0:m0 + 128])
             ob, eb = Q.quantize_mx_colwise(Wb[:, n0:n0 + 128])
             ref, t = G.reference(G.dequant_mx(oa, ea), G.dequant_mx(ob, eb))
             check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"mxfp8 {i} tile {m0},{n0}")
-        del qa, qb
-    # per-tensor comparison variant on the first shape
-    A, W = d["A0"], d["W0"]
-    qa = fq.quantize_tensor(A)
-    Wt = W.t().contiguous()
-    qb = fq.quantize_tensor(Wt)
-    c = host(fq.gemm(qa["q"], qb["q"], fq.FP8Q_PERTENSOR, a_global=qa["s_dec"], b_global=qb["s_dec"]).float())
-    oa, sa = Q.quantize_tensor(workloads.bf16_bits(A))
-    ob, sb = Q.quantize_tensor(workloads.bf16_bits(Wt))       # global scales over whole tensors
-    for m0, n0 in _tiles(8192, 4096, 20)[:8]:
-        ref, t = G.reference(G.dequant_tensor(oa[m0:m0 + 128], sa), G.dequant_tensor(ob[n0:n0 + 128], sb))
-        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"per-tensor tile {m0},{n0}")
+        del qa, qb, c
+        # per-tensor comparison variant on the same tensors
+        Wt = W.t().contiguous()
+        qa = fq.quantize_tensor(A)
+        qb = fq.quantize_tensor(Wt)
+        c = host(fq.gemm(qa["q"], qb["q"], fq.FP8Q_PERTENSOR, a_global=qa["s_dec"], b_global=qb["s_dec"]).float())
+        oa, sa = Q.quantize_tensor(Ab)
+        ob, sb = Q.quantize_tensor(workloads.bf16_bits(Wt))     # global scales over whole tensors
+        for m0, n0 in _tiles(M, N, 20 + i):
+            ref, t = G.reference(G.dequant_tensor(oa[m0:m0 + 128], sa), G.dequant_tensor(ob[n0:n0 + 128], sb))
+            check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"per-tensor {i} tile {m0},{n0}")
+        del qa, qb, c, Wt
 
 
 def test_moe_grouped_fullsize_sampled(cuda_lib):
@@ -338,7 +340,7 @@ def test_moe_grouped_fullsize_sampled(cuda_lib):
                          ld_sb=K // 128, m_offsets=offs.cuda()).float())
         tiles = G.sample_group_tiles(offs.numpy(), N, 64, seed=4)
         Ab = workloads.bf16_bits(A)
-        for g, m0, m1, n0 in tiles[:24]:
+        for g, m0, m1, n0 in tiles:
             oa, sa = Q.quantize_1x128_rowwise(Ab[m0:m1])
             _, owt, sw = Q.quantize_128x128(workloads.bf16_bits(W[g][:, n0:n0 + 128]))
             ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
@@ -347,7 +349,10 @@ def test_moe_grouped_fullsize_sampled(cuda_lib):
 
 
 def test_nvfp4_fullsize_sampled(cuda_lib):
-    """Llama-3.1-405B-shaped NVFP4 dgrad (8192, 53248, 16384) and wgrad (16384, 8192, 53248)."""
+    """Llama-3.1-405B-shaped NVFP4 dgrad (8192, 53248, 16384) and wgrad (16384, 8192, 53248).
+    64 output tiles each: every pairing of 8 random 128-row bands with 8 random 128-column
+    bands, so the oracle quantizes 8 bands of each operand (a stochastically rounded band of
+    dY costs seconds in the oracle) while 64 tiles are compared."""
     fq = cuda_lib
     d = workloads.nvfp4(device="cuda")
     X, W, dY = d["X"], d["W"], d["dY"]
@@ -357,7 +362,7 @@ def test_nvfp4_fullsize_sampled(cuda_lib):
     qw = fq.rht16_quantize_sr(W, rowwise=True, sf_layout=1)
     c = host(fq.gemm(qd["q_row"], qw["q_row"], fq.FP8Q_NVFP4, a_scale=qd["sf_row"], b_scale=qw["sf_row"],
                      a_global=qd["g_row"], b_global=qw["g_row"], K=53248).float())
-    tiles = _tiles(8192, 16384, 5)[:8]
+    tiles = G.sample_band_tiles(8192, 16384, 8, 8, seed=5)
     rows_a = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
     rows_b = np.unique(np.concatenate([np.arange(n0, n0 + 128) for _, n0 in tiles]))
     oa, sa, ga = Q.quantize_nvfp4_rowwise(dYb, sr=True, sr_seed=6, rows=rows_a)
@@ -373,7 +378,7 @@ def test_nvfp4_fullsize_sampled(cuda_lib):
     qx = fq.rht16_quantize_sr(X, rowwise=False, colwise=True, rht=fq.FP4Q_COL, rht_seed=5, sf_layout=1)
     c = host(fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_NVFP4, a_scale=qx["sf_col"], b_scale=qd["sf_col"],
                      a_global=qx["g_col"], b_global=qd["g_col"], K=8192).float())
-    tiles = _tiles(16384, 53248, 6)[:8]
+    tiles = G.sample_band_tiles(16384, 53248, 8, 8, seed=6)
     cols_a = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
     cols_b = np.unique(np.concatenate([np.arange(n0, n0 + 128) for _, n0 in tiles]))
     oa, sa, ga = Q.quantize_nvfp4_colwise(Xb, rht=True, rht_seed=5, rows=cols_a)

@@ -101,6 +101,10 @@ def test_sample_tiles_distinct_and_in_range():
     gt = G.sample_group_tiles(offs.numpy(), 2048, 64, seed=4)
     assert len(gt) == 64
     assert {g for g, *_ in gt} >= {g for g in range(32) if counts[g] > 0} or len(gt) == 64
+    bt = G.sample_band_tiles(16384, 53248, 8, 8, seed=6)
+    assert len(set(bt)) == 64
+    assert len({m for m, _ in bt}) == 8 and len({n for _, n in bt}) == 8
+    assert all(0 <= m < 16384 and 0 <= n < 53248 and m % 128 == 0 and n % 128 == 0 for m, n in bt)
 
 
 def test_fine_grained_beats_per_tensor_on_wide_range():

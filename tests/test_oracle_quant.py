@@ -295,3 +295,72 @@ def test_delayed_e5m2_and_empty_history():
     q, s, _ = Q.quantize_tensor_delayed(x, np.float32([4.0]), fmt="e5m2")         # sf = 14336, not exact
     assert s == np.float32(np.float32(1.0) / np.float32(14336.0))
     assert np.array_equal(q, F.e5m2_encode_bruteforce(x.ravel() * np.float32(14336.0)).reshape(x.shape))
+
+
+# ------------------------------------------------------------ NVFP4 16x16 weight blocks
+def test_nvfp4_2d_exact_grid_roundtrip():
+    """Each 16x16 block on the E2M1 grid times 2^j, with one element at +-6 * 2^j: every code
+    is exact, the block scale decodes to 448 * 2^(j - jmax) and both layouts round-trip."""
+    rng = np.random.default_rng(17)
+    x, js = exact_matrix(48, 64, 16, 16, rng, top=6.0, grid="e2m1", jrange=(-5, 5))
+    q_row, sf_row, q_col, sf_col, g = Q.quantize_nvfp4_2d(x)
+    assert np.allclose(_deq_nvfp4(q_row, sf_row, g), x.astype(np.float64), rtol=2.0 ** -23, atol=0)
+    assert np.allclose(_deq_nvfp4(q_col, sf_col, g), x.T.astype(np.float64), rtol=2.0 ** -23, atol=0)
+    want = 448.0 * np.exp2(js - js.max())                    # (R/16, C/16)
+    assert np.array_equal(F.e4m3_decode(sf_row), np.repeat(want, 16, axis=0))
+    assert np.array_equal(F.e4m3_decode(sf_col), np.repeat(want.T, 16, axis=0))
+
+
+def test_nvfp4_2d_reduces_to_1d_when_block_rows_or_columns_repeat():
+    """If the 16 rows of every block band are equal, a 16x16 block's amax is each row
+    group's amax and the rowwise output is the 1x16 quantizer's; likewise for columns."""
+    rng = np.random.default_rng(18)
+    base = (rng.standard_normal((4, 96)) * 0.02).astype(np.float32)
+    base[1, 5] = 0.9                                          # an outlier block
+    rows_rep = np.repeat(base, 16, axis=0)                    # (64, 96)
+    q_row, sf_row, _, _, g = Q.quantize_nvfp4_2d(rows_rep)
+    q1, sf1, g1 = Q.quantize_nvfp4_rowwise(rows_rep)
+    assert np.array_equal(q_row, q1) and np.array_equal(sf_row, sf1) and g == g1
+    cols_rep = np.ascontiguousarray(rows_rep.T)               # (96, 64): columns repeat
+    _, _, q_col, sf_col, g = Q.quantize_nvfp4_2d(cols_rep)
+    q2, sf2, g2 = Q.quantize_nvfp4_colwise(cols_rep)
+    assert np.array_equal(q_col, q2) and np.array_equal(sf_col, sf2) and g == g2
+
+
+def test_nvfp4_2d_bruteforce_and_layout_consistency():
+    """Per block: amax over 256 values by a plain loop, the scale by the brute-force E4M3
+    encoder, each code by the brute-force E2M1 encoder; both layouts hold the same codes
+    and dequantize to one matrix."""
+    d = workloads.nvfp4(M=64, H=32, F=48, which=("W",))
+    x = Q.as_f32(workloads.bf16_bits(d["W"]))                 # (32, 48) weights
+    x[3, 7] = np.float32(0.75)
+    q_row, sf_row, q_col, sf_col, g = Q.quantize_nvfp4_2d(x)
+    S_g = np.float32(np.float32(2688.0) / np.float32(np.abs(x).max()))
+    assert g == np.float32(np.float32(1.0) / S_g)
+    codes = np.zeros(x.shape, np.uint8)
+    for bi in range(2):
+        for bj in range(3):
+            blk = x[16 * bi:16 * bi + 16, 16 * bj:16 * bj + 16]
+            m = max(abs(float(v)) for v in blk.ravel())
+            sb = int(F.e4m3_encode_bruteforce(np.float32(np.float32(np.float32(m) / np.float32(6.0)) * S_g))[0])
+            assert np.all(sf_row[16 * bi:16 * bi + 16, bj] == sb) and np.all(sf_col[16 * bj:16 * bj + 16, bi] == sb)
+            enc = np.float32(0.0) if sb == 0 else np.float32(S_g / np.float32(F.e4m3_decode(np.uint8(sb))))
+            codes[16 * bi:16 * bi + 16, 16 * bj:16 * bj + 16] = F.e2m1_encode_bruteforce(
+                (blk * enc).astype(np.float32)).reshape(16, 16)
+    assert np.array_equal(F.unpack_e2m1(q_row), codes)
+    assert np.array_equal(F.unpack_e2m1(q_col), codes.T)
+    assert np.array_equal(_deq_nvfp4(q_row, sf_row, g), _deq_nvfp4(q_col, sf_col, g).T)
+
+
+def test_nvfp4_2d_sub_rectangle_with_global_amax():
+    """A 16-aligned sub-rectangle quantized with the whole tensor's amax equals the matching
+    slice of the whole tensor's result (what the sampled full-size checks rely on)."""
+    rng = np.random.default_rng(19)
+    x = (rng.standard_normal((64, 80)) * 0.02).astype(np.float32)
+    x[50, 3] = np.float32(-1.5)
+    q_row, sf_row, q_col, sf_col, g = Q.quantize_nvfp4_2d(x)
+    G = np.abs(x).max()
+    a_row, a_sfr, a_col, a_sfc, ga = Q.quantize_nvfp4_2d(x[16:48, 32:80], amax=G)
+    assert ga == g
+    assert np.array_equal(a_row, q_row[16:48, 16:40]) and np.array_equal(a_sfr, sf_row[16:48, 2:5])
+    assert np.array_equal(a_col, q_col[32:80, 8:24]) and np.array_equal(a_sfc, sf_col[32:80, 1:3])
