@@ -4,7 +4,7 @@ Default workload (one "step"), Llama-3-8B up-projection, blockwise recipe, forwa
 backward with M = 8192 tokens, hidden K = 4096, FFN N = 14336:
   quantize X (1x128 rowwise + fused transposed colwise), quantize W (128x128, both
   layouts), quantize dY (1x128 rowwise + colwise), GEMM fprop, dgrad, wgrad.
-Other workloads (--workload): tiny, mxfp8, moe, nvfp4 (one JSON line each).
+Other workloads (--workload): tiny, mxfp8, moe, nvfp4, nvfp4_train, wgrad_acc, delayed (one JSON line each).
 
 Metric: block-scaled GEMM TFLOP/s (the step's GEMM FLOPs over the whole step's device time,
 quantization included) with per-kernel TFLOP/s and GB/s as fractions of the roofline.
@@ -607,8 +607,92 @@ class Nvfp4Step:
         return flop, time.perf_counter() - t0, "1 dgrad output tile; amax over 1024-row slabs"
 
 
+class Nvfp4TrainStep:
+    """The NVFP4 training step of one Llama-3.1-405B MLP projection: fprop, dgrad and wgrad,
+    with the weights quantized once in 16x16 blocks for both fprop and dgrad."""
+    name = "nvfp4_train"
+    workload = ("NVFP4 Llama-3.1-405B training step: fprop (8192,16384,53248) with 16x16-block weights, "
+                "dgrad (8192,53248,16384), wgrad (16384,8192,53248)")
+
+    def __init__(self, fq, rank, M=8192, H=16384, F=53248):
+        self.fq, self.M, self.H, self.F = fq, M, H, F
+        d = workloads.nvfp4(device="cuda", M=M, H=H, F=F)
+        self.X, self.W, self.dY = d["X"], d["W"], d["dY"]
+        dev = self.X.device
+        u8 = torch.uint8
+        sfb = lambda o, i: torch.empty(fq.fp8q_sf_bytes(fq.FP8Q_NVFP4, o, i, 1), dtype=u8, device=dev)  # noqa: E731
+        self.qx_r, self.sx_r = torch.empty((M, H // 2), dtype=u8, device=dev), sfb(M, H)
+        self.qx_c, self.sx_c = torch.empty((H, M // 2), dtype=u8, device=dev), sfb(H, M)
+        self.qw_r, self.sw_r = torch.empty((H, F // 2), dtype=u8, device=dev), sfb(H, F)
+        self.qw_c, self.sw_c = torch.empty((F, H // 2), dtype=u8, device=dev), sfb(F, H)
+        self.qd_r, self.sd_r = torch.empty((M, F // 2), dtype=u8, device=dev), sfb(M, F)
+        self.qd_c, self.sd_c = torch.empty((F, M // 2), dtype=u8, device=dev), sfb(F, M)
+        self.g = torch.empty((5,), dtype=torch.float32, device=dev)
+        self.Y = torch.empty((M, F), dtype=torch.bfloat16, device=dev)
+        self.dX = torch.empty((M, H), dtype=torch.bfloat16, device=dev)
+        self.dW = torch.empty((H, F), dtype=torch.bfloat16, device=dev)
+        self.gemm_flop = 3 * 2.0 * M * H * F
+
+    def inputs(self):
+        return [self.X, self.W, self.dY]
+
+    def outputs(self):
+        return [self.Y, self.dX, self.dW]
+
+    def launches(self):
+        fq, M, H, F = self.fq, self.M, self.H, self.F
+        P = lambda t: t.data_ptr()  # noqa: E731
+        g = self.g
+
+        def qx():   # rowwise RNE for fprop, colwise RHT RNE for wgrad
+            assert fq.fp4q_rht16_quantize_sr(P(self.X), M, H, H, fq.FP4Q_COL, 5, 0, 6, P(self.qx_r), P(self.sx_r),
+                                             P(g[0:1]), P(self.qx_c), P(self.sx_c), P(g[1:2]), 1, fq._stream()) == 0
+
+        def qw():   # one 16x16-block quantization, both layouts
+            assert fq.fp4q_quantize_2d16(P(self.W), H, F, F, P(self.qw_r), P(self.sw_r), P(self.qw_c), P(self.sw_c),
+                                         P(g[2:3]), 1, fq._stream()) == 0
+
+        def qd():   # rowwise SR for dgrad, colwise RHT SR for wgrad
+            assert fq.fp4q_rht16_quantize_sr(P(self.dY), M, F, F, fq.FP4Q_COL, 5, fq.FP4Q_ROW | fq.FP4Q_COL, 6,
+                                             P(self.qd_r), P(self.sd_r), P(g[3:4]), P(self.qd_c), P(self.sd_c),
+                                             P(g[4:5]), 1, fq._stream()) == 0
+
+        def fprop():
+            fq.gemm(self.qx_r, self.qw_c, fq.FP8Q_NVFP4, a_scale=self.sx_r, b_scale=self.sw_c, a_global=g[0:1],
+                    b_global=g[2:3], K=H, out=self.Y)
+
+        def dgrad():
+            fq.gemm(self.qd_r, self.qw_r, fq.FP8Q_NVFP4, a_scale=self.sd_r, b_scale=self.sw_r, a_global=g[3:4],
+                    b_global=g[2:3], K=F, out=self.dX)
+
+        def wgrad():
+            fq.gemm(self.qx_c, self.qd_c, fq.FP8Q_NVFP4, a_scale=self.sx_c, b_scale=self.sd_c, a_global=g[1:2],
+                    b_global=g[4:5], K=M, out=self.dW)
+
+        nv2 = lambda r, c: r * c * 4.0 + 2 * r * c * (0.5 + 1 / 16)  # noqa: E731  two outputs
+        return [Launch("fp4q quantize X (row RNE + col RHT RNE)", qx, "quantize_nvfp4", bytes_=nv2(M, H)),
+                Launch("fp4q quantize W 16x16 blocks (both layouts)", qw, "quantize_nvfp4", bytes_=nv2(H, F)),
+                Launch("gemm nvfp4 fprop (16x16 weights)", fprop, "gemm_nvfp4", flop=2.0 * M * H * F),
+                Launch("fp4q quantize dY (row SR + col RHT SR)", qd, "quantize_nvfp4", bytes_=nv2(M, F)),
+                Launch("gemm nvfp4 dgrad (16x16 weights)", dgrad, "gemm_nvfp4", flop=2.0 * M * H * F),
+                Launch("gemm nvfp4 wgrad", wgrad, "gemm_nvfp4", flop=2.0 * M * H * F)]
+
+    def cpu_sample(self, tiles=1):
+        from oracle import gemm as G
+        from oracle import quant as Q
+        t0 = time.perf_counter()
+        Xb = workloads.bf16_bits(self.X[:1024])
+        Wb = workloads.bf16_bits(self.W[:, :128])
+        # global amax over the sampled slabs stands in for the full tensors' (sample timing only)
+        oa, sa, ga = Q.quantize_nvfp4_rowwise(Xb, rows=list(range(128)))
+        _, _, ob, sb, gb = Q.quantize_nvfp4_2d(Wb)
+        G.reference(G.dequant_nvfp4(oa, sa, ga), G.dequant_nvfp4(ob, sb, gb))
+        flop = 2.0 * 128 * 128 * self.H
+        return flop, time.perf_counter() - t0, "1 fprop output tile; amax over the sampled slabs"
+
+
 STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step,
-         "wgrad_acc": WgradAccStep, "delayed": DelayedStep}
+         "wgrad_acc": WgradAccStep, "delayed": DelayedStep, "nvfp4_train": Nvfp4TrainStep}
 
 
 # ============================================================================ measurement
@@ -767,7 +851,7 @@ def run_ours(args, rank, world, local_rank):
     out = {
         "metric": METRIC, "value": round(value, 2), "unit": "TFLOP/s", "n_gpus": world, "steps": args.steps,
         "warmup": args.warmup, "ms_per_step": round(ms, 4), "higher_is_better": True, "scaling": "weak",
-        "vs_baseline": None, "dtype": "fp8_e4m3" if args.workload != "nvfp4" else "fp4_e2m1",
+        "vs_baseline": None, "dtype": "fp4_e2m1" if args.workload.startswith("nvfp4") else "fp8_e4m3",
         "data": "synthetic (seeded normal BF16 with outliers; see workloads.py)",
         "config": {"workload": step.workload, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "gemm_tflop_per_step": round(step.gemm_flop / 1e12, 4),

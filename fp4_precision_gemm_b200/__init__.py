@@ -21,10 +21,10 @@ __all__ = [
     "FP4Q_ROW", "FP4Q_COL", "Fp8qError", "lib", "library_path",
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp8q_quantize_tensor_noalloc", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
-    "fp4q_rht16_quantize_sr", "FP8Q_E4M3", "FP8Q_E5M2", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
+    "fp4q_rht16_quantize_sr", "fp4q_quantize_2d16", "FP8Q_E4M3", "FP8Q_E5M2", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
     "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
     "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_tensor_delayed", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
-    "gemm", "device_status", "EXPORTED_SYMBOLS",
+    "quantize_nvfp4_2d16", "gemm", "device_status", "EXPORTED_SYMBOLS",
 ]
 
 FP8Q_OK = 0
@@ -40,6 +40,7 @@ EXPORTED_SYMBOLS = [
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
+    "fp4q_quantize_2d16",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -88,6 +89,7 @@ def lib():
                                                    _vp, _vp, _vp]
         L.fp4q_rht16_quantize_sr.argtypes = [_vp, _i64, _i64, _i64, _int, _u64, _int, _u64,
                                              _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
+        L.fp4q_quantize_2d16.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
         L.fp8q_sf_bytes.argtypes = [_int, _i64, _i64, _int]
         L.fp8q_sf_bytes.restype = ctypes.c_size_t
@@ -105,7 +107,7 @@ def lib():
                                                      "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
                                                      "fp8q_get_device_status", "fp8q_release_scratch",
                                                      "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped",
-                                                     "fp8q_quantize_tensor_delayed"):
+                                                     "fp8q_quantize_tensor_delayed", "fp4q_quantize_2d16"):
                 f.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -168,6 +170,10 @@ def fp4q_rht16_quantize_sr(x, rows, cols, ld_x, rht, rht_seed, sr, sr_seed, q_ro
                            q_col, sf_col, g_col, sf_layout, stream):
     return lib().fp4q_rht16_quantize_sr(x, rows, cols, ld_x, rht, rht_seed, sr, sr_seed, q_row, sf_row, g_row,
                                         q_col, sf_col, g_col, sf_layout, stream)
+
+
+def fp4q_quantize_2d16(x, rows, cols, ld_x, q_row, sf_row, q_col, sf_col, g_dec, sf_layout, stream):
+    return lib().fp4q_quantize_2d16(x, rows, cols, ld_x, q_row, sf_row, q_col, sf_col, g_dec, sf_layout, stream)
 
 
 def fp8q_gemm_blockscaled(args, stream):
@@ -322,6 +328,26 @@ def rht16_quantize_sr(x, rowwise=True, colwise=False, rht=0, rht_seed=0, sr=0, s
                                 _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out.get("g_col")),
                                 sf_layout, _stream(stream))
     _check(st, "fp4q_rht16_quantize_sr")
+    return out
+
+
+def quantize_nvfp4_2d16(w, rowwise=True, colwise=True, sf_layout=FP8Q_SF_MMA_TILED, stream=None):
+    """NVFP4 weights with one scale per 16x16 block.  Returns q_row (R, C/2), sf_row and/or
+    q_col (C, R/2), sf_col, and g (1,), the decode scale both layouts share."""
+    _check_bf16(w, "w")
+    R, C = w.shape
+    dev = w.device
+    out = {"g": torch.empty((1,), dtype=torch.float32, device=dev)}
+    if rowwise:
+        out["q_row"] = torch.empty((R, C // 2), dtype=torch.uint8, device=dev)
+        out["sf_row"] = torch.empty(fp8q_sf_bytes(FP8Q_NVFP4, R, C, sf_layout), dtype=torch.uint8, device=dev)
+    if colwise:
+        out["q_col"] = torch.empty((C, R // 2), dtype=torch.uint8, device=dev)
+        out["sf_col"] = torch.empty(fp8q_sf_bytes(FP8Q_NVFP4, C, R, sf_layout), dtype=torch.uint8, device=dev)
+    st = fp4q_quantize_2d16(_ptr(w), R, C, w.stride(0), _ptr(out.get("q_row")), _ptr(out.get("sf_row")),
+                            _ptr(out.get("q_col")), _ptr(out.get("sf_col")), _ptr(out["g"]), sf_layout,
+                            _stream(stream))
+    _check(st, "fp4q_quantize_2d16")
     return out
 
 

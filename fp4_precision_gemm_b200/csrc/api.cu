@@ -329,6 +329,42 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
   return from_cuda(e);
 }
 
+fp8q_status fp4q_quantize_2d16(const void* x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t* q_row,
+                               uint8_t* sf_row, uint8_t* q_col, uint8_t* sf_col, float* g_dec,
+                               fp8q_sf_layout sf_layout, void* stream) {
+  fp8q_status st = check_input(x, rows, cols, ld_x);
+  if (st != FP8Q_OK) return st;
+  const bool row = q_row || sf_row, col = q_col || sf_col;
+  if ((!row && !col) || !g_dec) return FP8Q_ERR_NULL;
+  if ((row && (!q_row || !sf_row)) || (col && (!q_col || !sf_col))) return FP8Q_ERR_NULL;
+  if (sf_layout != FP8Q_SF_ROWMAJOR && sf_layout != FP8Q_SF_MMA_TILED) return FP8Q_ERR_UNSUPPORTED;
+  if (rows % 16 != 0 || cols % 16 != 0) return FP8Q_ERR_SHAPE;
+  if ((row && !aligned16(q_row)) || (col && !aligned16(q_col))) return FP8Q_ERR_ALIGN;
+  if (rows == 0 || cols == 0) return FP8Q_OK;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  DeviceScratch* d = nullptr;
+  if ((st = scratch(&d)) != FP8Q_OK) return st;
+  uint32_t* amax = nullptr;
+  if ((st = amax_slot(d, s, &amax)) != FP8Q_OK) return st;
+  Fp4QuantParams p;
+  p.x = static_cast<const uint16_t*>(x);
+  p.rows = rows;
+  p.cols = cols;
+  p.ld_x = ld_x;
+  p.rht_row = p.rht_col = p.sr_row = p.sr_col = 0;
+  p.rht_k0 = p.rht_k1 = p.sr_k0 = p.sr_k1 = 0;
+  p.q_row = row ? q_row : nullptr;
+  p.sf_row = sf_row;
+  p.g_row = g_dec;
+  p.q_col = col ? q_col : nullptr;
+  p.sf_col = sf_col;
+  p.g_col = nullptr;
+  p.sf_tiled = sf_layout == FP8Q_SF_MMA_TILED;
+  p.tiles_c = (int)((cols + 127) / 128);
+  p.amax_bits = amax;
+  return from_cuda(launch_fp4_quant_2d(p, tiles_of(rows, cols), s));
+}
+
 // ------------------------------------------------------------------ GEMM
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (!a) return FP8Q_ERR_NULL;

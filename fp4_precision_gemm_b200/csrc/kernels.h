@@ -57,6 +57,9 @@ cudaError_t launch_tensor_delayed(const uint16_t* x, int64_t rows, int64_t cols,
 
 cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
+// 16x16-block weight quantizer: global amax into amax_bits[0], then codes in the layouts
+// whose q pointer is set; g_row receives the decode scale.
+cudaError_t launch_fp4_quant_2d(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMM
 // Output tile width of the blockwise (FP32-promotion) kernel; the B and wgrad-scale TMA boxes

@@ -289,6 +289,115 @@ __global__ void __launch_bounds__(256, 3) fp4_quant_col_kernel(const __grid_cons
   }
 }
 
+// ------------------------------------------------------------------ 16x16 weight blocks
+// One scale per 16x16 block, codes emitted in both layouts (the forward GEMM reads the
+// weights along one axis, the backward-data GEMM along the other, and both must see one
+// quantized matrix).  Same tile mapping as the colwise kernel: a block is the 16x4
+// sub-blocks of 4 consecutive lanes, so its amax is an in-thread max plus two xor-shuffles.
+// Codes are computed once, row-paired (2 bytes per row per lane, a warp stores 64 contiguous
+// bytes of each row); the colwise words are the same nibbles regrouped along the rows and go
+// out through the shared staging tile like the colwise kernel's.
+__global__ void __launch_bounds__(256, 3) fp4_quant_2d_kernel(const __grid_constant__ Fp4QuantParams P) {
+  __shared__ __align__(16) uint8_t tq[128 * 64];
+  __shared__ float enc_tab[128];
+  const Tile T = tile_coords(P, blockIdx.x);
+  float x[16][4];
+  load16x4(P, T, x);
+  const float S_g = global_scale(P.amax_bits[0]);
+  if (threadIdx.x < 128) fill_enc_tab(enc_tab, S_g);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_row = __frcp_rn(S_g);
+  __syncthreads();
+
+  float m = 0.0f;
+#pragma unroll
+  for (int i = 0; i < 16; ++i)
+#pragma unroll
+    for (int j = 0; j < 4; ++j) m = fmaxf(m, fabsf(x[i][j]));
+  m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+  m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
+  uint32_t sb;
+  float enc;
+  block_scale(m, S_g, enc_tab, sb, enc);
+
+  // rc[k]: the 4 codes of row 2k (low half) and of row 2k+1 (high half), column 4*lane + j in
+  // nibble j of each half
+  uint32_t rc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    uint32_t v = 0;
+#pragma unroll
+    for (int h = 0; h < 2; ++h) {
+      const int i = 2 * k + h;
+      v |= (e2m1x2_rne(__fmul_rn(x[i][1], enc), __fmul_rn(x[i][0], enc)) |
+            (e2m1x2_rne(__fmul_rn(x[i][3], enc), __fmul_rn(x[i][2], enc)) << 8)) << (16 * h);
+    }
+    rc[k] = v;
+  }
+
+  const int64_t row0 = T.r0 + T.w * 16;
+  const int64_t kc = (T.c0 >> 4) + (T.lane >> 2);      // this block's scale column (rowwise)
+  const int64_t kr = (T.r0 >> 4) + T.w;                 // its scale column in the colwise output
+  if (P.q_row) {
+    const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) {
+      const int64_t row = row0 + i;
+      if (T.cok && row < P.rows)
+        *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)(rc[i >> 1] >> (16 * (i & 1)));
+    }
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {                        // lane & 3 == q writes rows 4q..4q+3
+      const int64_t row = row0 + 4 * (T.lane & 3) + i;
+      if (P.sf_tiled) {
+        if (kc < s4 * 4) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+      } else if (row < P.rows && kc < nsf) {
+        P.sf_row[row * nsf + kc] = (uint8_t)sb;
+      }
+    }
+  }
+  if (P.q_col) {
+    const int64_t nsf = P.rows >> 4, s4 = (nsf + 3) >> 2;
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      uint32_t lo = 0, hi = 0;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) {           // row i: half i & 1 of rc[i >> 1]
+        lo |= ((rc[i >> 1] >> (16 * (i & 1) + 4 * j)) & 0xFu) << (4 * i);
+        hi |= ((rc[4 + (i >> 1)] >> (16 * (i & 1) + 4 * j)) & 0xFu) << (4 * i);
+      }
+      const int c = T.lane * 4 + j;
+      const int64_t cg = T.col + j;
+      *(uint2*)&tq[c * 64 + ((T.w ^ ((c >> 2) & 7)) * 8)] = make_uint2(lo, hi);
+      if (P.sf_tiled) {
+        if (kr < s4 * 4) P.sf_col[sf_tiled_offset(cg, kr, s4)] = (uint8_t)sb;
+      } else if (cg < P.cols && kr < nsf) {
+        P.sf_col[cg * nsf + kr] = (uint8_t)sb;
+      }
+    }
+    __syncthreads();
+#pragma unroll
+    for (int pass = 0; pass < 2; ++pass) {
+      const int c = pass * 64 + (threadIdx.x >> 2), h = threadIdx.x & 3;
+      const int64_t cg = T.c0 + c, rg = T.r0 + 32 * h;
+      const uint2 a = *(const uint2*)&tq[c * 64 + (((2 * h) ^ ((c >> 2) & 7)) * 8)];
+      const uint2 b = *(const uint2*)&tq[c * 64 + (((2 * h + 1) ^ ((c >> 2) & 7)) * 8)];
+      uint8_t* dst = P.q_col + cg * (P.rows >> 1) + (rg >> 1);
+      if (cg < P.cols) {
+        if (rg + 32 <= P.rows) {
+          if (((P.rows >> 1) & 15) == 0) {
+            *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
+          } else {
+            *(uint2*)dst = a;
+            *(uint2*)(dst + 8) = b;
+          }
+        } else if (rg + 16 <= P.rows) {
+          *(uint2*)dst = a;
+        }
+      }
+    }
+  }
+}
+
 // ------------------------------------------------------------------ rowwise-only path
 // When only the rowwise output is requested, one thread owns one 16-element group of a row
 // (two 16-byte loads): the group's transform, amax, scale and codes stay in-thread and a warp
@@ -392,6 +501,12 @@ cudaError_t launch_fp4_amax(const Fp4QuantParams& p, int64_t tiles, cudaStream_t
   if (row && col) fp4_amax_kernel<true, true><<<tile_grid, 256, 0, s>>>(p, tiles);
   else if (row) fp4_amax_row_kernel<<<blocks_for(p.rows * (p.cols >> 4)), 256, 0, s>>>(p);
   else fp4_amax_kernel<false, true><<<tile_grid, 256, 0, s>>>(p, tiles);
+  return cudaGetLastError();
+}
+
+cudaError_t launch_fp4_quant_2d(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
+  fp4_amax_row_kernel<<<blocks_for(p.rows * (p.cols >> 4)), 256, 0, s>>>(p);
+  fp4_quant_2d_kernel<<<(unsigned)tiles, 256, 0, s>>>(p);
   return cudaGetLastError();
 }
 

@@ -204,6 +204,29 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
                                    uint8_t* q_col, uint8_t* sf_col, float* g_dec_col,
                                    fp8q_sf_layout sf_layout, void* stream);
 
+/* NVFP4 weights with one E4M3 scale per 16x16 block, in both GEMM operand layouts, so that
+ * the forward GEMM (weights read along one axis) and the backward-data GEMM (along the
+ * other) use one quantized matrix.  The [NVFP4] page ("How it works") fixes the 4-bit
+ * values, the per-16 E4M3 scales and the per-tensor FP32 scale; the 16x16 block shape of a
+ * weight scale is this library's reading for that two-layout use.
+ *   G = amax |x| over the tensor; S_g = 2688 / G (G == 0 -> 1);
+ *   per 16x16 block: sb = E4M3(fp32(amax_b / 6) * S_g) over its 256 elements,
+ *   enc = S_g / decode(sb) (0 if sb == 0), q = E2M1_RNE(x * enc); *g_dec = 1 / S_g.
+ *   No transform and no stochastic rounding (weights, not gradient inputs).
+ * x: BF16 rows x cols, row stride ld_x elements (ld_x % 8 == 0), 16-byte aligned;
+ *   rows % 16 == 0 and cols % 16 == 0.
+ * Rowwise (q_row, sf_row): q_row rows x cols/2 bytes (even element in the low nibble),
+ *   sf_row scale bytes for (rows, cols/16), each block's code repeated over its 16 rows.
+ * Colwise (q_col, sf_col): the same codes transposed, q_col cols x rows/2, sf_col for
+ *   (cols, rows/16).  Either pair may be NULL, not both; g_dec (device float) is required.
+ * Scale bytes in sf_layout (FP8Q_SF_MMA_TILED for the NVFP4 GEMM; padding bytes 0).
+ * Two passes over x (global amax, then quantize); asynchronous on `stream`.
+ * Errors: FP8Q_ERR_NULL, FP8Q_ERR_SHAPE, FP8Q_ERR_ALIGN (q pointers 16-byte aligned),
+ *   FP8Q_ERR_UNSUPPORTED (sf_layout), FP8Q_ERR_CUDA. */
+fp8q_status fp4q_quantize_2d16(const void* x, int64_t rows, int64_t cols, int64_t ld_x,
+                               uint8_t* q_row, uint8_t* sf_row, uint8_t* q_col, uint8_t* sf_col,
+                               float* g_dec, fp8q_sf_layout sf_layout, void* stream);
+
 /* Arguments of fp8q_gemm_blockscaled: C[M x N] = A[M x K] . B[N x K]^T, both operands
  * K-major codes, C BF16 row-major (ldc >= N, ldc % 8 == 0, c 16-byte aligned) unless
  * c_fp32_accumulate is set (below).

@@ -176,3 +176,17 @@ def test_delayed_quantizer_and_fp8_format_validation(L):
     g = fq.fp8q_gemm_blockscaled
     assert g(_args(a_format=1), s) == fq.FP8Q_ERR_UNSUPPORTED          # E5M2 is per-tensor only
     assert g(_args(recipe=fq.FP8Q_PERTENSOR, b_format=3), s) == fq.FP8Q_ERR_UNSUPPORTED
+
+
+def test_nvfp4_2d16_validation(L):
+    s = None
+    f = fq.fp4q_quantize_2d16
+    assert f(ALIGNED, 16, 24, 24, ALIGNED, ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_SHAPE      # cols % 16
+    assert f(ALIGNED, 24, 16, 16, ALIGNED, ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_SHAPE      # rows % 16
+    assert f(ALIGNED, 16, 16, 16, ALIGNED, ALIGNED, ALIGNED, ALIGNED, None, 0, s) == fq.FP8Q_ERR_NULL   # no g_dec
+    assert f(ALIGNED, 16, 16, 16, None, None, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_NULL            # no output
+    assert f(ALIGNED, 16, 16, 16, ALIGNED, None, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_NULL         # half a pair
+    assert f(ALIGNED, 16, 16, 16, ALIGNED, ALIGNED, None, None, ALIGNED, 2, s) == fq.FP8Q_ERR_UNSUPPORTED
+    assert f(ALIGNED, 16, 16, 16, P(0x10008), ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_ALIGN
+    assert f(ALIGNED, 16, 16, 12, ALIGNED, ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_SHAPE      # ld_x < cols
+    assert f(ALIGNED, 0, 16, 16, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 0, s) == fq.FP8Q_OK       # empty

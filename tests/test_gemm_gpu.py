@@ -241,6 +241,28 @@ def test_nvfp4(cuda_lib, M, K, N, rht):
     check(c, ref, t, "nvfp4")
 
 
+@pytest.mark.parametrize("M,K,N", [(300, 512, 768), (128, 256, 256)])
+def test_nvfp4_forward_and_dgrad_with_16x16_weights(cuda_lib, M, K, N):
+    """One 16x16-block quantization of W (K x N) feeds both fprop (X . W, W read along K:
+    its colwise output) and dgrad (dY . W^T, W read along N: its rowwise output)."""
+    fq = cuda_lib
+    X, W, dY = bf((M, K), 1.0, M + 3 * K, 1e-3, 50.0), bf((K, N), 0.02, K + 5 * N), bf((M, N), 1e-3, M + 7 * N)
+    qw = fq.quantize_nvfp4_2d16(W.cuda())
+    qx = fq.rht16_quantize_sr(X.cuda(), sf_layout=fq.FP8Q_SF_MMA_TILED)
+    y = fq.gemm(qx["q_row"], qw["q_col"], fq.FP8Q_NVFP4, a_scale=qx["sf_row"], b_scale=qw["sf_col"],
+                a_global=qx["g_row"], b_global=qw["g"], K=K)
+    qd = fq.rht16_quantize_sr(dY.cuda(), sr=fq.FP4Q_ROW, sr_seed=6, sf_layout=fq.FP8Q_SF_MMA_TILED)
+    dx = fq.gemm(qd["q_row"], qw["q_row"], fq.FP8Q_NVFP4, a_scale=qd["sf_row"], b_scale=qw["sf_row"],
+                 a_global=qd["g_row"], b_global=qw["g"], K=N)
+    ow_row, sw_row, ow_col, sw_col, gw = Q.quantize_nvfp4_2d(workloads.bf16_bits(W))
+    ox, sx, gx = Q.quantize_nvfp4_rowwise(workloads.bf16_bits(X))
+    ref, t = G.reference(G.dequant_nvfp4(ox, sx, gx), G.dequant_nvfp4(ow_col, sw_col, gw))
+    check(y, ref, t, "nvfp4 fprop, 16x16 weights")
+    od, sd, gd = Q.quantize_nvfp4_rowwise(workloads.bf16_bits(dY), sr=True, sr_seed=6)
+    ref, t = G.reference(G.dequant_nvfp4(od, sd, gd), G.dequant_nvfp4(ow_row, sw_row, gw))
+    check(dx, ref, t, "nvfp4 dgrad, 16x16 weights")
+
+
 def test_k_zero_gives_zeros(cuda_lib):
     fq = cuda_lib
     a = torch.zeros((4, 128), dtype=torch.uint8, device="cuda")
@@ -251,6 +273,11 @@ def test_k_zero_gives_zeros(cuda_lib):
 
 
 # ----------------------------------------------------------------------------- full size, sampled
+def amax_bf16(bits, rows=1024):
+    """max |x| of a BF16 bit-pattern matrix, by row chunks (no full FP32 copy)."""
+    return max(np.float32(np.abs(Q.as_f32(bits[r:r + rows])).max()) for r in range(0, bits.shape[0], rows))
+
+
 def _tiles(M, N, seed):
     return G.sample_tiles(M, N, 64, seed=seed)
 
@@ -346,6 +373,30 @@ def test_moe_grouped_fullsize_sampled(cuda_lib):
             ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
             check(c[m0:m1, n0:n0 + 128].astype(np.float64), ref, t, f"moe {proj} expert {g} tile {m0},{n0}")
         del qa, B, SB, d
+
+
+def test_nvfp4_fprop_16x16_weights_fullsize_sampled(cuda_lib):
+    """Llama-3.1-405B-shaped NVFP4 forward GEMM (8192, 16384, 53248): X rowwise 1x16 scales,
+    W with 16x16 block scales (colwise output), 64 sampled output tiles."""
+    fq = cuda_lib
+    d = workloads.nvfp4(device="cuda", which=("X", "W"))
+    X, W = d["X"], d["W"]
+    qx = fq.rht16_quantize_sr(X, sf_layout=1)
+    qw = fq.quantize_nvfp4_2d16(W, rowwise=False, colwise=True)
+    c = host(fq.gemm(qx["q_row"], qw["q_col"], fq.FP8Q_NVFP4, a_scale=qx["sf_row"], b_scale=qw["sf_col"],
+                     a_global=qx["g_row"], b_global=qw["g"], K=16384).float())
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    tiles = _tiles(8192, 53248, 7)
+    rows_a = np.unique(np.concatenate([np.arange(m0, m0 + 128) for m0, _ in tiles]))
+    oa, sa, ga = Q.quantize_nvfp4_rowwise(Xb, rows=rows_a)
+    ia = {r: i for i, r in enumerate(rows_a)}
+    G_w = amax_bf16(Wb)
+    for m0, n0 in tiles:
+        ra = [ia[r] for r in range(m0, m0 + 128)]
+        _, _, ob, sb, gb = Q.quantize_nvfp4_2d(Wb[:, n0:n0 + 128], amax=G_w)
+        ref, t = G.reference(G.dequant_nvfp4(oa[ra], sa[ra], ga), G.dequant_nvfp4(ob, sb, gb))
+        check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"nvfp4 fprop tile {m0},{n0}")
+    assert fq.device_status() == 0
 
 
 def test_nvfp4_fullsize_sampled(cuda_lib):

@@ -278,3 +278,59 @@ def test_tensor_delayed_parity_and_history(cuda_lib, fmt):
         assert out["s_dec"].cpu().numpy().view(np.uint32)[0] == np.float32(os_).view(np.uint32)
         h_host[pos] = oa
         assert np.array_equal(hist.cpu().numpy().view(np.uint32), h_host.view(np.uint32))
+
+
+# ----------------------------------------------------------------------------- NVFP4 16x16 weights
+@pytest.mark.parametrize("layout", [0, 1])
+@pytest.mark.parametrize("R,C,row,col", [
+    (304, 656, True, True), (48, 400, True, False), (368, 96, False, True), (16, 16, True, True),
+    (256, 512, True, True)])
+def test_nvfp4_2d16_parity(cuda_lib, layout, R, C, row, col):
+    """16x16-block weight quantizer: codes, scales (both layouts) and decode scale bit-exact."""
+    fq = cuda_lib
+    x = workloads.normal_bf16((R, C), 0.02, 7 * R + C, 1e-3, 50.0)
+    if R >= 32 and C >= 32:
+        x[16:32, 16:32] = 0.0                                    # an all-zero block: scale code 0
+    out = fq.quantize_nvfp4_2d16(x.cuda(), rowwise=row, colwise=col, sf_layout=layout)
+    q_row, sf_row, q_col, sf_col, g = Q.quantize_nvfp4_2d(workloads.bf16_bits(x))
+    assert f32bits(host(out["g"]))[0] == f32bits(np.float32([g]))[0]
+    if row:
+        assert np.array_equal(host(out["q_row"]), q_row)
+        assert np.array_equal(host(out["sf_row"]), Q.sf_to_tiled(sf_row) if layout == 1 else sf_row.ravel())
+    if col:
+        assert np.array_equal(host(out["q_col"]), q_col)
+        assert np.array_equal(host(out["sf_col"]), Q.sf_to_tiled(sf_col) if layout == 1 else sf_col.ravel())
+    assert "q_row" in out or not row
+    assert "q_col" in out or not col
+
+
+def test_nvfp4_2d16_zero_tensor(cuda_lib):
+    fq = cuda_lib
+    x = torch.zeros((32, 48), dtype=torch.bfloat16)
+    out = fq.quantize_nvfp4_2d16(x.cuda(), sf_layout=0)
+    q_row, sf_row, q_col, sf_col, g = Q.quantize_nvfp4_2d(workloads.bf16_bits(x))
+    assert np.array_equal(host(out["q_row"]), q_row) and np.array_equal(host(out["q_col"]), q_col)
+    assert int(host(out["sf_row"]).max()) == 0 and host(out["g"])[0] == 1.0
+
+
+def test_nvfp4_2d16_weight_fullsize_sampled(cuda_lib):
+    """Llama-3.1-405B weight (16384 x 53248): sampled 128-row bands of the rowwise output and
+    128-column bands of the colwise output, against the oracle on the same bands with the
+    whole tensor's amax."""
+    fq = cuda_lib
+    W = workloads.nvfp4(device="cuda", which=("W",))["W"]
+    out = fq.quantize_nvfp4_2d16(W, sf_layout=0)
+    bits = workloads.bf16_bits(W)
+    G_amax = max(np.float32(np.abs(Q.as_f32(bits[r:r + 1024])).max()) for r in range(0, bits.shape[0], 1024))
+    rng = np.random.default_rng(23)
+    R, C = bits.shape
+    q_row_d, q_col_d = host(out["q_row"]), host(out["q_col"])
+    sf_row_d = host(out["sf_row"]).reshape(R, C // 16)
+    sf_col_d = host(out["sf_col"]).reshape(C, R // 16)
+    for r0 in sorted({0, R - 128, int(rng.integers(0, R // 128)) * 128}):
+        q_row, sf_row, _, _, g = Q.quantize_nvfp4_2d(bits[r0:r0 + 128], amax=G_amax)
+        assert np.array_equal(q_row_d[r0:r0 + 128], q_row) and np.array_equal(sf_row_d[r0:r0 + 128], sf_row)
+    for c0 in sorted({0, C - 128, int(rng.integers(0, C // 128)) * 128}):
+        _, _, q_col, sf_col, g = Q.quantize_nvfp4_2d(bits[:, c0:c0 + 128], amax=G_amax)
+        assert np.array_equal(q_col_d[c0:c0 + 128], q_col) and np.array_equal(sf_col_d[c0:c0 + 128], sf_col)
+    assert f32bits(host(out["g"]))[0] == f32bits(np.float32([g]))[0]
