@@ -362,29 +362,39 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ blockwise (promotion) kernel
-// CTA pairs (clusters of 2) share 256 x 192 output tiles with the pair MMA
-// (tcgen05.mma.cta_group::2, M = 256): each CTA loads its own 128 rows of A and its half (96
-// rows) of B, so an SM moves 28 KB per 128-element K chunk instead of 40 KB, and each CTA's
+// CTA pairs (clusters of 2) share 256 x BN output tiles with the pair MMA
+// (tcgen05.mma.cta_group::2, M = 256): BN = 256 for fprop/dgrad (and the grouped MoE GEMM),
+// 192 for wgrad.  Each CTA loads its own 128 rows of A and its half (BN/2 rows) of B, so an
+// SM moves 32 KB (28 KB) per 128-element K chunk instead of 48 KB (40 KB), and each CTA's
 // TMEM receives its 128 rows of the chunk's partial.  The leader CTA's single MMA thread
 // issues for both; the TMA completions of both CTAs are counted on the leader's barrier and
 // the MMA commits arrive on both CTAs' barriers (multicast commit, no multicast loads).
-// In each CTA warps 0-11 promote (warp w: TMEM lanes 32*(w%4).., columns 64*(w/4)..),
-// warp 12 drives the A/B TMA, warp 13 owns TMEM (and, in the leader, issues the MMAs) and
-// warp 14 stages each chunk's scales in a shared-memory ring.  With at most four warps per SM
-// sub-partition a thread may use 128 registers: its 64 FP32 accumulators stay in registers
-// for the whole tile.  Two 192-column TMEM partial buffers alternate per K chunk, so the MMAs
-// of chunk k + 1 run while chunk k is promoted; the stage's single commit tells both the
-// producers (stage free) and the promotion warps (partial complete) of both CTAs.
+// In each CTA the first 4 * BN/64 warps promote (warp w: TMEM lanes 32*(w%4).., columns
+// 64*(w/4)..), then one warp drives the A/B TMA, one owns TMEM (and, in the leader, issues
+// the MMAs) and one stages each chunk's scales in a shared-memory ring.  Every promotion
+// thread keeps its 64 FP32 accumulators in registers for the whole tile (19 warps leave 96
+// registers a thread at BN = 256, 15 warps leave 128 at BN = 192, which wgrad's column
+// scales need).  Two BN-column TMEM partial buffers alternate per K chunk, so the MMAs of
+// chunk k + 1 run while chunk k is promoted; the stage's single commit tells both the
+// producers (stage free) and the promotion warps (partial complete) of both CTAs.  The
+// per-chunk hand-off between the MMA issuer and the promotion warps costs about the same
+// for any BN, so the wider tile does more MMA work per hand-off.
 namespace {
 
-constexpr int kBwBN = (int)kBlockwiseTileN;     // 192 output columns per pair tile
-constexpr int kBwHalfBN = kBwBN / 2;            // B rows loaded by each CTA
 constexpr int kBwPairM = 2 * kBM;               // 256 output rows per pair tile
-constexpr int kBwEpiWarps = 12;
-constexpr int kBwProducerWarp = 12, kBwMmaWarp = 13, kBwScaleWarp = 14;
-constexpr int kBwThreads = 15 * 32;
 constexpr int kBwSb = 10;                       // scale ring: chunks of A/B scales staged ahead
-constexpr uint32_t kBwBStage = kBwHalfBN * kBKB;  // 12 KB
+
+// Per-layout shape: fprop/dgrad 256 x 256 pair tiles (16 promotion warps), wgrad 256 x 192
+// (12 promotion warps, which leave each thread the registers its column scales need).
+template <int L>
+struct BwCfg {
+  static constexpr int BN = (int)blockwise_tile_n(L);   // output columns per pair tile
+  static constexpr int HalfBN = BN / 2;                 // B rows loaded by each CTA
+  static constexpr int EpiWarps = 4 * (BN / 64);        // 32 rows x 64 columns each
+  static constexpr int ProducerWarp = EpiWarps, MmaWarp = EpiWarps + 1, ScaleWarp = EpiWarps + 2;
+  static constexpr int Threads = (EpiWarps + 3) * 32;
+  static constexpr uint32_t BStage = HalfBN * kBKB;    // 16 KB / 12 KB
+};
 
 
 // Shared memory of the blockwise kernel.  A scale-ring slot holds one chunk's scales:
@@ -392,20 +402,21 @@ constexpr uint32_t kBwBStage = kBwHalfBN * kBKB;  // 12 KB
 // fprop/dgrad: [A scales][the B scales of the tile's three 64-column groups].
 template <int L>
 struct BwSmem {
+  using C = BwCfg<L>;
   static constexpr bool wg = (L == kWgrad);
-  static constexpr int stages = 6;
+  static constexpr int stages = wg ? 6 : 5;
   static constexpr uint32_t slot_sbw = 0;
-  static constexpr uint32_t slot_sa = wg ? kBwBN * 4 : 0;
+  static constexpr uint32_t slot_sa = wg ? C::BN * 4 : 0;
   static constexpr uint32_t slot_sb = slot_sa + kBM * 4;
-  static constexpr uint32_t slot_bytes = ((slot_sb + (wg ? 0 : 16) + 127) / 128) * 128;
+  static constexpr uint32_t slot_bytes = ((slot_sb + (wg ? 0 : (C::BN / 64) * 4) + 127) / 128) * 128;
   static constexpr uint32_t a = 0;
   static constexpr uint32_t b = a + stages * kAStage;
-  static constexpr uint32_t ring = b + stages * kBwBStage;
+  static constexpr uint32_t ring = b + stages * C::BStage;
   // epilogue staging per promotion warp: 32 rows x epi_cols BF16 (wgrad: half the width)
-  static constexpr int epi_cols = wg ? 32 : 64;
+  static constexpr int epi_cols = 32;
   static constexpr uint32_t stage_c = 32 * epi_cols * 2;
   static constexpr uint32_t cst = ring + kBwSb * slot_bytes;
-  static constexpr uint32_t bars = cst + kBwEpiWarps * stage_c;
+  static constexpr uint32_t bars = cst + C::EpiWarps * stage_c;
   static constexpr uint32_t n_bars = 2 * stages + 2 + 2 * kBwSb + 1;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t groups = misc + 16;
@@ -414,8 +425,9 @@ struct BwSmem {
   static_assert(alloc <= 227 * 1024, "shared memory");
 };
 
-// Pair tile t: 256 rows x 192 columns, rasterized like tile_of; grouped GEMMs enumerate each
+// Pair tile t: 256 rows x BN columns, rasterized like tile_of; grouped GEMMs enumerate each
 // expert's 256-row tiles.  Returns this CTA's 128-row half.
+template <int BN>
 __device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
                                              const int* offs, uint32_t rank) {
   const int per = p.group_m * p.tiles_n;
@@ -424,7 +436,7 @@ __device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row
   const int local = t - grp * per;
   const int rt = first + local % gsz, nt = local / gsz;
   Tile T;
-  T.n0 = nt * kBwBN;
+  T.n0 = nt * BN;
   int end;
   if (p.num_groups > 0) {
     int g = 0;
@@ -458,11 +470,15 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 }  // namespace
 
 template <int L, bool GROUPED, bool ACC32>
-__global__ void __launch_bounds__(kBwThreads, 1)
+__global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
+  constexpr int kBwBN = BwCfg<L>::BN, kBwHalfBN = BwCfg<L>::HalfBN, kBwEpiWarps = BwCfg<L>::EpiWarps;
+  constexpr int kBwProducerWarp = BwCfg<L>::ProducerWarp, kBwMmaWarp = BwCfg<L>::MmaWarp;
+  constexpr int kBwScaleWarp = BwCfg<L>::ScaleWarp;
+  constexpr uint32_t kBwBStage = BwCfg<L>::BStage;
   constexpr int kStages = S::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -520,7 +536,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
-        const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
+        const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
         const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
@@ -552,7 +568,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
-      const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
       const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
       for (int kb = 0; kb < KB; ++kb, ++it) {
         const uint32_t r = it % kBwSb, rph = (it / kBwSb) & 1;
@@ -570,7 +586,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
           const bool in = m < p.M;
           cp_async_4(ssa + i * 32 + lane, p.sa + (in ? (int64_t)kb * p.ld_sa + m : 0), in ? 4u : 0u);
         }
-        if (!kWg && lane < 3) {
+        if (!kWg && lane < kBwBN / 64) {
           const int ncol0 = T.n0 + lane * 64, nblk = ncol0 / kBM;
           const bool in = ncol0 < p.N;
           const int64_t off = !in ? 0 : (L == kFprop) ? (int64_t)nblk * p.ld_sb + kb : (int64_t)kb * p.ld_sb + nblk;
@@ -629,7 +645,7 @@ __global__ void __launch_bounds__(kBwThreads, 1)
     uint32_t chunk = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
-      const Tile T = pair_tile_of(t, p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
       const int ncol0 = T.n0 + cgp * 64;
       float2 acc[32];
 #pragma unroll
@@ -649,14 +665,14 @@ __global__ void __launch_bounds__(kBwThreads, 1)
         const float2 s2 = make_float2(scale, scale);
         if constexpr (!kWg) {
 #pragma unroll
-          for (int h = 0; h < 2; ++h) {
-            uint32_t r[32];
-            tmem_ld_32x32b_x32(t_lane + pb * kBwBN + h * 32, r);
+          for (int h = 0; h < 4; ++h) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(t_lane + pb * kBwBN + h * 16, r);
             tmem_ld_wait(r);
 #pragma unroll
-            for (int i = 0; i < 16; ++i) {
+            for (int i = 0; i < 8; ++i) {
               const float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-              acc[h * 16 + i] = __ffma2_rn(pr, s2, acc[h * 16 + i]);
+              acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
             }
           }
         } else {
@@ -763,6 +779,7 @@ template <int L, bool G, bool ACC32 = false>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
   auto kern = gemm_blockwise_kernel<L, G, ACC32>;
+  constexpr int kBwBN = BwCfg<L>::BN;
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -773,7 +790,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
-  cfg.blockDim = dim3(kBwThreads);
+  cfg.blockDim = dim3(BwCfg<L>::Threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
