@@ -451,9 +451,9 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (!make_map(&ma, a->a, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, a->M, a->lda, 128, 128,
                 CU_TENSOR_MAP_SWIZZLE_128B))
     return FP8Q_ERR_CUDA;
-  // B box rows: each CTA of a blockwise pair loads half of its tile's columns; the other
+  // B box rows: each CTA of a blockwise pair loads half of its 256-column tile; the other
   // kernel loads its whole 256-column tile.  The wgrad scale box spans the full tile width.
-  const uint32_t bn = (a->recipe == FP8Q_BLOCKWISE) ? blockwise_tile_n((int)a->layout) : 256;
+  const uint32_t bn = (a->recipe == FP8Q_BLOCKWISE) ? kBlockwiseTileN : 256;
   const uint32_t b_box = (a->recipe == FP8Q_BLOCKWISE) ? bn / 2 : 256;
   if (!make_map(&mb, a->b, CU_TENSOR_MAP_DATA_TYPE_UINT8, kbytes, b_rows, a->ldb, 128, b_box,
                 CU_TENSOR_MAP_SWIZZLE_128B))

@@ -362,38 +362,36 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ------------------------------------------------------------------ blockwise (promotion) kernel
-// CTA pairs (clusters of 2) share 256 x BN output tiles with the pair MMA
-// (tcgen05.mma.cta_group::2, M = 256): BN = 256 for fprop/dgrad (and the grouped MoE GEMM),
-// 192 for wgrad.  Each CTA loads its own 128 rows of A and its half (BN/2 rows) of B, so an
-// SM moves 32 KB (28 KB) per 128-element K chunk instead of 48 KB (40 KB), and each CTA's
-// TMEM receives its 128 rows of the chunk's partial.  The leader CTA's single MMA thread
+// CTA pairs (clusters of 2) share 256 x 256 output tiles with the pair MMA
+// (tcgen05.mma.cta_group::2, M = 256).  Each CTA loads its own 128 rows of A and its half
+// (128 rows) of B, so an SM moves 32 KB per 128-element K chunk instead of 48 KB, and each
+// CTA's TMEM receives its 128 rows of the chunk's partial.  The leader CTA's single MMA thread
 // issues for both; the TMA completions of both CTAs are counted on the leader's barrier and
 // the MMA commits arrive on both CTAs' barriers (multicast commit, no multicast loads).
-// In each CTA the first 4 * BN/64 warps promote (warp w: TMEM lanes 32*(w%4).., columns
-// 64*(w/4)..), then one warp drives the A/B TMA, one owns TMEM (and, in the leader, issues
-// the MMAs) and one stages each chunk's scales in a shared-memory ring.  Every promotion
-// thread keeps its 64 FP32 accumulators in registers for the whole tile (19 warps leave 96
-// registers a thread at BN = 256, 15 warps leave 128 at BN = 192, which wgrad's column
-// scales need).  Two BN-column TMEM partial buffers alternate per K chunk, so the MMAs of
-// chunk k + 1 run while chunk k is promoted; the stage's single commit tells both the
-// producers (stage free) and the promotion warps (partial complete) of both CTAs.  The
-// per-chunk hand-off between the MMA issuer and the promotion warps costs about the same
-// for any BN, so the wider tile does more MMA work per hand-off.
+// In each CTA warps 0-15 promote (warp w: TMEM lanes 32*(w%4).., columns 64*(w/4)..), warp
+// 16 drives the A/B TMA, warp 17 owns TMEM (and, in the leader, issues the MMAs) and warp 18
+// stages each chunk's scales in a shared-memory ring.  Every promotion thread keeps its 64
+// FP32 accumulators in registers for the whole tile; 19 warps leave it 96 registers, so the
+// partials come out of TMEM 16 columns at a time and wgrad's column scales are read from
+// shared memory just before their use.  Two 256-column TMEM partial buffers (all 512
+// columns) alternate per K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted;
+// the stage's single commit tells both the producers (stage free) and the promotion warps
+// (partial complete) of both CTAs.  The per-chunk hand-off between the MMA issuer and the
+// promotion warps costs about the same for any tile width, so the widest tile does the most
+// MMA work per hand-off.
 namespace {
 
 constexpr int kBwPairM = 2 * kBM;               // 256 output rows per pair tile
 constexpr int kBwSb = 10;                       // scale ring: chunks of A/B scales staged ahead
 
-// Per-layout shape: fprop/dgrad 256 x 256 pair tiles (16 promotion warps), wgrad 256 x 192
-// (12 promotion warps, which leave each thread the registers its column scales need).
-template <int L>
+// Pair tile shape: 256 x 256 outputs, 16 promotion warps.
 struct BwCfg {
-  static constexpr int BN = (int)blockwise_tile_n(L);   // output columns per pair tile
+  static constexpr int BN = (int)kBlockwiseTileN;       // output columns per pair tile
   static constexpr int HalfBN = BN / 2;                 // B rows loaded by each CTA
   static constexpr int EpiWarps = 4 * (BN / 64);        // 32 rows x 64 columns each
   static constexpr int ProducerWarp = EpiWarps, MmaWarp = EpiWarps + 1, ScaleWarp = EpiWarps + 2;
   static constexpr int Threads = (EpiWarps + 3) * 32;
-  static constexpr uint32_t BStage = HalfBN * kBKB;    // 16 KB / 12 KB
+  static constexpr uint32_t BStage = HalfBN * kBKB;    // 16 KB
 };
 
 
@@ -402,9 +400,9 @@ struct BwCfg {
 // fprop/dgrad: [A scales][the B scales of the tile's three 64-column groups].
 template <int L>
 struct BwSmem {
-  using C = BwCfg<L>;
+  using C = BwCfg;
   static constexpr bool wg = (L == kWgrad);
-  static constexpr int stages = wg ? 6 : 5;
+  static constexpr int stages = 5;
   static constexpr uint32_t slot_sbw = 0;
   static constexpr uint32_t slot_sa = wg ? C::BN * 4 : 0;
   static constexpr uint32_t slot_sb = slot_sa + kBM * 4;
@@ -470,15 +468,15 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 }  // namespace
 
 template <int L, bool GROUPED, bool ACC32>
-__global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
+__global__ void __launch_bounds__(BwCfg::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
-  constexpr int kBwBN = BwCfg<L>::BN, kBwHalfBN = BwCfg<L>::HalfBN, kBwEpiWarps = BwCfg<L>::EpiWarps;
-  constexpr int kBwProducerWarp = BwCfg<L>::ProducerWarp, kBwMmaWarp = BwCfg<L>::MmaWarp;
-  constexpr int kBwScaleWarp = BwCfg<L>::ScaleWarp;
-  constexpr uint32_t kBwBStage = BwCfg<L>::BStage;
+  constexpr int kBwBN = BwCfg::BN, kBwHalfBN = BwCfg::HalfBN, kBwEpiWarps = BwCfg::EpiWarps;
+  constexpr int kBwProducerWarp = BwCfg::ProducerWarp, kBwMmaWarp = BwCfg::MmaWarp;
+  constexpr int kBwScaleWarp = BwCfg::ScaleWarp;
+  constexpr uint32_t kBwBStage = BwCfg::BStage;
   constexpr int kStages = S::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -676,8 +674,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
             }
           }
         } else {
-          // wgrad also scales each column: 16 columns per TMEM load keeps the column scales
-          // and the loaded partial sums within the register budget
+          // wgrad also scales each column (its B scales are per column and chunk)
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             uint32_t r[16];
@@ -686,7 +683,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
 #pragma unroll
             for (int i = 0; i < 8; ++i) {
               float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-              pr = __fmul2_rn(pr, *reinterpret_cast<const float2*>(sbw + h * 16 + 2 * i));
+              pr = __fmul2_rn(pr, ld_shared_f2(sbw + h * 16 + 2 * i));
               acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
             }
           }
@@ -779,7 +776,7 @@ template <int L, bool G, bool ACC32 = false>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
   auto kern = gemm_blockwise_kernel<L, G, ACC32>;
-  constexpr int kBwBN = BwCfg<L>::BN;
+  constexpr int kBwBN = BwCfg::BN;
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -790,7 +787,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
-  cfg.blockDim = dim3(BwCfg<L>::Threads);
+  cfg.blockDim = dim3(BwCfg::Threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];

@@ -62,10 +62,9 @@ cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_
 cudaError_t launch_fp4_quant_2d(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s);
 
 // ------------------------------------------------------------------ GEMM
-// Output tile width of the blockwise (FP32-promotion) kernel by layout (0 fprop, 1 dgrad,
-// 2 wgrad); the B and wgrad-scale TMA boxes are built with it.  Wgrad's per-column scales
-// need more registers per promotion thread, which only the narrower tile's warp count leaves.
-constexpr uint32_t blockwise_tile_n(int layout) { return layout == 2 ? 192u : 256u; }
+// Output tile width of the blockwise (FP32-promotion) kernel; the B and wgrad-scale TMA boxes
+// are built with it.
+constexpr uint32_t kBlockwiseTileN = 256;
 
 struct GemmParams {
   int recipe;       // fp8q_recipe

@@ -258,6 +258,14 @@ __device__ __forceinline__ void tmem_ld_32x32b_x32(uint32_t taddr, uint32_t (&r)
         "=r"(r[30]), "=r"(r[31])
       : "r"(taddr));
 }
+// Two floats from shared memory, loaded where the call stands: the volatile asm keeps the
+// compiler from hoisting a row of such loads ahead of their uses (and their registers live).
+__device__ __forceinline__ float2 ld_shared_f2(const float* p) {
+  float2 v;
+  asm volatile("ld.shared.v2.f32 {%0, %1}, [%2];" : "=f"(v.x), "=f"(v.y) : "r"(smem_u32(p)));
+  return v;
+}
+
 // 16 consecutive 32-bit TMEM columns of this thread's lane.
 __device__ __forceinline__ void tmem_ld_32x32b_x16(uint32_t taddr, uint32_t (&r)[16]) {
   asm volatile(
