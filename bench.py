@@ -4,7 +4,8 @@ Default workload (one "step"), Llama-3-8B up-projection, blockwise recipe, forwa
 backward with M = 8192 tokens, hidden K = 4096, FFN N = 14336:
   quantize X (1x128 rowwise + fused transposed colwise), quantize W (128x128, both
   layouts), quantize dY (1x128 rowwise + colwise), GEMM fprop, dgrad, wgrad.
-Other workloads (--workload): tiny, mxfp8, moe, nvfp4, nvfp4_train, wgrad_acc, delayed (one JSON line each).
+Other workloads (--workload): tiny, mxfp8, moe, nvfp4, nvfp4_train, wgrad_acc, delayed,
+fprop_quant (one JSON line each).
 
 Metric: block-scaled GEMM TFLOP/s (the step's GEMM FLOPs over the whole step's device time,
 quantization included) with per-kernel TFLOP/s and GB/s as fractions of the roofline.
@@ -216,6 +217,74 @@ class TinyStep(LlamaStep):
         _, owt, sw = Q.quantize_128x128(workloads.bf16_bits(self.B))
         G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
         return self.gemm_flop, time.perf_counter() - t0, "the whole tiny step"
+
+
+class FpropQuantStep:
+    """Llama-3-8B up-projection forward with online quantization of its output for the next
+    layer: X in 1x128 tiles, W in 128x128 blocks, then Y = X . W with the blockwise promotion,
+    written as BF16 and, from the GEMM's epilogue, as 1x128 E4M3 codes and scales."""
+    name = "fprop_quant"
+    workload = "llama3-8b up-proj fprop with fused 1x128 quantization of Y: X 8192x4096, W 4096x14336"
+
+    def __init__(self, fq, rank, M=8192, K=4096, N=14336):
+        self.fq, self.M, self.K, self.N = fq, M, K, N
+        d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
+        self.X, self.W = d["X"], d["W"]
+        del d
+        dev = self.X.device
+        u8, f32 = torch.uint8, torch.float32
+        self.qx_r, self.sx_r = torch.empty((M, K), dtype=u8, device=dev), torch.empty((K // 128, M), dtype=f32, device=dev)
+        self.qw_t, self.qw = torch.empty((N, K), dtype=u8, device=dev), torch.empty((K, N), dtype=u8, device=dev)
+        self.sw = torch.empty((N // 128, K // 128), dtype=f32, device=dev)
+        self.Y = torch.empty((M, N), dtype=torch.bfloat16, device=dev)
+        self.qy, self.sy = torch.empty((M, N), dtype=u8, device=dev), torch.empty((N // 128, M), dtype=f32, device=dev)
+        self.gemm_flop = 2.0 * M * N * K
+
+    def inputs(self):
+        return [self.X, self.W]
+
+    def outputs(self):
+        return [self.Y, self.qy, self.sy]
+
+    def launches(self):
+        fq, M, K, N = self.fq, self.M, self.K, self.N
+        P = lambda t: t.data_ptr()  # noqa: E731
+
+        def qx():
+            assert fq.fp8q_quantize_1x128(P(self.X), M, K, K, P(self.qx_r), P(self.sx_r), M, None, None, 0,
+                                          fq._stream()) == 0
+
+        def qw():
+            assert fq.fp8q_quantize_128x128(P(self.W), K, N, N, P(self.qw_t), P(self.qw), P(self.sw), fq._stream()) == 0
+
+        def g():
+            fq.gemm(self.qx_r, self.qw_t, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=self.sx_r, b_scale=self.sw,
+                    ld_sb=K // 128, out=self.Y, q_out=self.qy, s_out=self.sy)
+
+        return [Launch("quantize_1x128 X (row)", qx, "quantize", bytes_=b_1x128_row(M, K)),
+                Launch("quantize_128x128 W (both layouts)", qw, "quantize", bytes_=b_128(K, N)),
+                Launch("gemm blockwise fprop + fused 1x128 quantization of Y", g, "gemm_blockwise",
+                       flop=self.gemm_flop)]
+
+    def cpu_sample(self, tiles=1):
+        """Oracle on a bounded sample: `tiles` sampled 128x128 tiles of Y, operands quantized by
+        the oracle, FP64 product, then the product's 1x128 quantization."""
+        from oracle import gemm as G
+        from oracle import quant as Q
+        from oracle import formats as F
+        M, K, N = self.M, self.K, self.N
+        if not hasattr(self, "_host_bits"):
+            self._host_bits = tuple(workloads.bf16_bits(t) for t in (self.X, self.W))
+        Xb, Wb = self._host_bits
+        t0 = time.perf_counter()
+        flop = 0.0
+        for m0, n0 in G.sample_tiles(M, N, tiles, seed=7):
+            oa, sa = Q.quantize_1x128_rowwise(Xb[m0:m0 + 128])
+            _, owt, sw = Q.quantize_128x128(Wb[:, n0:n0 + 128])
+            ref, _ = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+            Q.quantize_1x128_rowwise(F.f32_to_bf16_bits(ref.astype("float32")))
+            flop += 2.0 * 128 * 128 * K
+        return flop, time.perf_counter() - t0, f"{tiles} sampled 128x128 tile(s) of Y and their 1x128 quantization"
 
 
 class WgradAccStep:
@@ -692,7 +761,8 @@ class Nvfp4TrainStep:
 
 
 STEPS = {"llama8b": LlamaStep, "tiny": TinyStep, "mxfp8": MxStep, "moe": MoeStep, "nvfp4": Nvfp4Step,
-         "wgrad_acc": WgradAccStep, "delayed": DelayedStep, "nvfp4_train": Nvfp4TrainStep}
+         "wgrad_acc": WgradAccStep, "delayed": DelayedStep, "nvfp4_train": Nvfp4TrainStep,
+         "fprop_quant": FpropQuantStep}
 
 
 # ============================================================================ measurement

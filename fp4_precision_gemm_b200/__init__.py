@@ -64,6 +64,8 @@ class GemmArgs(ctypes.Structure):
         ("m_offsets", ctypes.c_void_p), ("num_groups", ctypes.c_int32),
         ("c_fp32_accumulate", ctypes.c_int32),
         ("a_format", ctypes.c_int32), ("b_format", ctypes.c_int32),
+        ("q_out", ctypes.c_void_p), ("s_out", ctypes.c_void_p),
+        ("ld_q_out", ctypes.c_int64), ("ld_s_out", ctypes.c_int64),
     ]
 
 
@@ -353,10 +355,12 @@ def quantize_nvfp4_2d16(w, rowwise=True, colwise=True, sf_layout=FP8Q_SF_MMA_TIL
 
 def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
          a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False,
-         a_format=0, b_format=0, stream=None):
+         a_format=0, b_format=0, q_out=None, s_out=None, stream=None):
     """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
     Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16.
-    accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T."""
+    accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T.
+    q_out (M, N) uint8 and s_out (N/128, M) float32 (BLOCKWISE): also receive the 1x128
+    rowwise quantization of the BF16 C, made in the GEMM's epilogue."""
     M = a.shape[0]
     grouped = m_offsets is not None
     N = b.shape[1] if grouped else b.shape[0]
@@ -381,6 +385,11 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
     args.num_groups = (m_offsets.numel() - 1) if grouped else 0
     args.c_fp32_accumulate = 1 if accumulate_fp32 else 0
     args.a_format, args.b_format = a_format, b_format
+    if q_out is not None or s_out is not None:
+        args.q_out = q_out.data_ptr() if q_out is not None else None
+        args.s_out = s_out.data_ptr() if s_out is not None else None
+        args.ld_q_out = q_out.stride(0) if q_out is not None else 0
+        args.ld_s_out = s_out.stride(0) if s_out is not None else 0
     _check(fp8q_gemm_blockscaled(args, _stream(stream)), "fp8q_gemm_blockscaled")
     return c
 

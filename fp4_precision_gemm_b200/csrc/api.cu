@@ -376,6 +376,14 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   if (acc32 && a->recipe != FP8Q_BLOCKWISE) return FP8Q_ERR_UNSUPPORTED;
   if (a->a_format < 0 || a->a_format > 1 || a->b_format < 0 || a->b_format > 1) return FP8Q_ERR_UNSUPPORTED;
   if ((a->a_format || a->b_format) && a->recipe != FP8Q_PERTENSOR) return FP8Q_ERR_UNSUPPORTED;
+  const bool qout = a->q_out != nullptr || a->s_out != nullptr;
+  if (qout) {
+    if (a->recipe != FP8Q_BLOCKWISE || acc32 || a->num_groups != 0) return FP8Q_ERR_UNSUPPORTED;
+    if (!a->q_out || !a->s_out) return FP8Q_ERR_NULL;
+    if (a->N % 128 != 0 || a->K < 384 || a->ld_q_out < a->N || a->ld_q_out % 16 != 0 || a->ld_s_out < a->M)
+      return FP8Q_ERR_SHAPE;
+    if (!aligned16(a->q_out)) return FP8Q_ERR_ALIGN;
+  }
   if (a->M == 0 || a->N == 0) return FP8Q_OK;
   if (!a->c) return FP8Q_ERR_NULL;
   if (a->ldc < a->N || a->ldc % (acc32 ? 4 : 8) != 0) return FP8Q_ERR_SHAPE;
@@ -409,6 +417,10 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   p.c32 = acc32 ? static_cast<float*>(a->c) : nullptr;
   p.a_fmt = a->a_format;
   p.b_fmt = a->b_format;
+  p.q_out = qout ? a->q_out : nullptr;
+  p.s_out = qout ? a->s_out : nullptr;
+  p.ld_q_out = a->ld_q_out;
+  p.ld_s_out = a->ld_s_out;
   p.ldc = a->ldc;
   p.m_offsets = a->m_offsets;
   p.num_groups = a->num_groups;

@@ -75,6 +75,14 @@ __device__ __forceinline__ void raise_timeout(const GemmParams& p, volatile int*
   atomicExch(p.status, kDevTimeout);
 }
 
+// Blockwise epilogue modes: BF16 C; FP32 C += result; BF16 C plus its 1x128 E4M3 codes.
+enum { kEpiBf16 = 0, kEpiAcc32 = 1, kEpiQuant = 2 };
+
+// The two values rounded to BF16 (round to nearest even, as pack_bf16 stores them), as FP32.
+__device__ __forceinline__ float2 bf16x2_round(float2 v) {
+  return __bfloat1622float2(__floats2bfloat162_rn(v.x, v.y));
+}
+
 __device__ __forceinline__ uint32_t pack_bf16(float a, float b) {
   __nv_bfloat162 h = __floats2bfloat162_rn(a, b);
   return *reinterpret_cast<uint32_t*>(&h);
@@ -415,10 +423,12 @@ struct BwSmem {
   static constexpr uint32_t stage_c = 32 * epi_cols * 2;
   static constexpr uint32_t cst = ring + kBwSb * slot_bytes;
   static constexpr uint32_t bars = cst + C::EpiWarps * stage_c;
-  static constexpr uint32_t n_bars = 2 * stages + 2 + 2 * kBwSb + 1;
+  static constexpr uint32_t n_bars = 2 * stages + 2 + 2 * kBwSb + 1 + C::EpiWarps / 2;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t groups = misc + 16;
-  static constexpr uint32_t total = groups + 2 * (kMaxGroups + 1) * 4;
+  // fused output quantization: each promotion warp's 32 row amaxes, read by its partner warp
+  static constexpr uint32_t xchg = groups + 2 * (kMaxGroups + 1) * 4;
+  static constexpr uint32_t total = xchg + C::EpiWarps * 32 * 4;
   static constexpr uint32_t alloc = total + 1024;
   static_assert(alloc <= 227 * 1024, "shared memory");
 };
@@ -467,12 +477,13 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 
 }  // namespace
 
-template <int L, bool GROUPED, bool ACC32>
+template <int L, bool GROUPED, int EPI>
 __global__ void __launch_bounds__(BwCfg::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
+  constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
   constexpr int kBwBN = BwCfg::BN, kBwHalfBN = BwCfg::HalfBN, kBwEpiWarps = BwCfg::EpiWarps;
   constexpr int kBwProducerWarp = BwCfg::ProducerWarp, kBwMmaWarp = BwCfg::MmaWarp;
   constexpr int kBwScaleWarp = BwCfg::ScaleWarp;
@@ -486,6 +497,7 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
   uint64_t* sfull = pempty + 2;          // local scale ring: slot filled
   uint64_t* sempty = sfull + kBwSb;      // local scale ring: slot read by every promotion warp
   uint64_t* final_bar = sempty + kBwSb;
+  uint64_t* xbar = final_bar + 1;        // [EpiWarps/2] fused quantization: partner warps' amaxes
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::misc + 4);
   int* prefix = reinterpret_cast<int*>(smem + S::groups);
@@ -507,6 +519,7 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
       mbar_init(&sempty[i], kBwEpiWarps);
     }
     mbar_init(final_bar, 1);
+    for (int i = 0; i < kBwEpiWarps / 2; ++i) mbar_init(&xbar[i], 2);
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -640,9 +653,9 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
     const int rloc = q * 32 + lane;
     const uint32_t pempty_leader0 = mapa_shared(smem_u32(&pempty[0]), 0);
     const uint32_t pempty_leader1 = mapa_shared(smem_u32(&pempty[1]), 0);
-    uint32_t chunk = 0;
+    uint32_t chunk = 0, tile_it = 0;
     bool ok = true;
-    for (int t = cluster; t < total && ok; t += n_clusters) {
+    for (int t = cluster; t < total && ok; t += n_clusters, ++tile_it) {
       const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
       const int ncol0 = T.n0 + cgp * 64;
       float2 acc[32];
@@ -745,6 +758,50 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
           __syncwarp();
         }
       }
+      if constexpr (QOUT) {
+        // Fused 1x128 quantization of the BF16 output along N (the next layer's activation
+        // codes and scales, as the 1x128 rowwise quantizer would make them from C): a
+        // 128-column group of a row is this warp's 64 columns and those of warp ^ 4, so the
+        // two warps' row amaxes meet in shared memory behind a two-arrival barrier.
+        float am = 0.0f;
+#pragma unroll
+        for (int j = 0; j < 32; ++j) {     // the values just stored, rounded to BF16
+          acc[j] = bf16x2_round(acc[j]);
+          am = fmaxf(am, fmaxf(fabsf(acc[j].x), fabsf(acc[j].y)));
+        }
+        float* xch = reinterpret_cast<float*>(smem + S::xchg);
+        xch[warp * 32 + lane] = am;
+        __syncwarp();
+        uint64_t* xb = &xbar[q * 2 + (cgp >> 1)];
+        if (lane == 0) mbar_arrive(xb);   // release: the warp's amaxes are visible
+        if (!mbar_wait(xb, tile_it & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+        am = fmaxf(am, xch[(warp ^ 4) * 32 + lane]);
+        const float sf = e4m3_sf(am);
+        const float2 s2 = make_float2(sf, sf);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {        // 16 codes (16 bytes) per chunk of the lane's row
+          uint32_t w[4];
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const float2 y0 = __fmul2_rn(acc[c * 8 + 2 * k], s2);
+            const float2 y1 = __fmul2_rn(acc[c * 8 + 2 * k + 1], s2);
+            w[k] = cvt_e4m3x2(y0.x, y0.y) | (cvt_e4m3x2(y1.x, y1.y) << 16);
+          }
+          stg[lane * 4 + (c ^ swz(lane))] = make_uint4(w[0], w[1], w[2], w[3]);
+        }
+        __syncwarp();
+#pragma unroll
+        for (int i = 0; i < 4; ++i) {        // 8 rows x 64 bytes per instruction
+          const int r = i * 8 + lane / 4, c = lane % 4;
+          const uint4 v = stg[r * 4 + (c ^ swz(r))];
+          const int mr = T.m0 + q * 32 + r, n = ncol0 + c * 16;
+          if (mr < T.mend && n < p.N) *reinterpret_cast<uint4*>(p.q_out + (int64_t)mr * p.ld_q_out + n) = v;
+        }
+        __syncwarp();
+        const int mrow = T.m0 + q * 32 + lane;
+        if ((cgp & 1) == 0 && mrow < T.mend && ncol0 < p.N)
+          p.s_out[(int64_t)(ncol0 >> 7) * p.ld_s_out + mrow] = __frcp_rn(sf);
+      }
     }
   }
 
@@ -772,10 +829,10 @@ static int raster_group(const GemmParams& p, int row_tiles, int tile_m) {
   return (int)(g < row_tiles ? g : row_tiles);
 }
 
-template <int L, bool G, bool ACC32 = false>
+template <int L, bool G, int EPI = kEpiBf16>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
-  auto kern = gemm_blockwise_kernel<L, G, ACC32>;
+  auto kern = gemm_blockwise_kernel<L, G, EPI>;
   constexpr int kBwBN = BwCfg::BN;
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
@@ -848,10 +905,15 @@ cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUt
                         const CUtensorMap& tma_sb, int num_sms, cudaStream_t s) {
   if (p.recipe == kBlockwise) {
     if (p.c32 != nullptr) {   // FP32 accumulate epilogue: its own instantiations
-      if (p.num_groups > 0) return launch_blockwise<kFprop, true, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      return launch_blockwise<kWgrad, false, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
+    }
+    if (p.q_out != nullptr) {  // BF16 output plus its fused 1x128 quantization
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
     }
     if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
     if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, num_sms, s);

@@ -256,7 +256,14 @@ fp8q_status fp4q_quantize_2d16(const void* x, int64_t rows, int64_t cols, int64_
  *     C[m,n] = fp32( C[m,n] + sum_kb ... )   (the FP32 sum above, before any BF16 rounding),
  *   the FP32 main-gradient accumulation that follows wgrad in training ([DSV3]
  *   "Mixed-precision framework": gradients and master weights stay in FP32).  K == 0
- *   leaves C unchanged. */
+ *   leaves C unchanged.
+ * q_out / s_out (BLOCKWISE with BF16 output, not grouped; both NULL otherwise): the GEMM
+ *   also quantizes its BF16 output C in 1x128 tiles along N, as fp8q_quantize_1x128's
+ *   rowwise output would from C ([DSV3] "Online quantization": the next layer's activation
+ *   is quantized from its live amax), without a second pass over C:
+ *     q_out[m * ld_q_out + n] = E4M3 codes (M x N bytes, ld_q_out >= N, % 16 == 0,
+ *     q_out 16-byte aligned), s_out[(n / 128) * ld_s_out + m] = FP32 decode scales
+ *     (ld_s_out >= M).  Needs N % 128 == 0 and K >= 384 (else FP8Q_ERR_SHAPE). */
 typedef struct {
   fp8q_recipe recipe;
   fp8q_layout layout;
@@ -275,6 +282,9 @@ typedef struct {
   int32_t num_groups;
   int32_t c_fp32_accumulate;
   int32_t a_format, b_format;   /* fp8q_fp8_format of A / B codes (PERTENSOR; else 0) */
+  uint8_t* q_out;               /* optional fused 1x128 quantization of C (see above) */
+  float* s_out;
+  int64_t ld_q_out, ld_s_out;
 } fp8q_gemm_args;
 
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);

@@ -190,3 +190,17 @@ def test_nvfp4_2d16_validation(L):
     assert f(ALIGNED, 16, 16, 16, P(0x10008), ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_ALIGN
     assert f(ALIGNED, 16, 16, 12, ALIGNED, ALIGNED, None, None, ALIGNED, 0, s) == fq.FP8Q_ERR_SHAPE      # ld_x < cols
     assert f(ALIGNED, 0, 16, 16, ALIGNED, ALIGNED, ALIGNED, ALIGNED, ALIGNED, 0, s) == fq.FP8Q_OK       # empty
+
+
+def test_fused_output_quantization_validation(L):
+    s = None
+    base = dict(q_out=ALIGNED.value, s_out=ALIGNED.value, ld_q_out=256, ld_s_out=256, K=512, N=256, M=256, ldc=256)
+    g = fq.fp8q_gemm_blockscaled
+    assert g(_args(**{**base, "recipe": fq.FP8Q_MXFP8}), s) == fq.FP8Q_ERR_UNSUPPORTED      # blockwise only
+    assert g(_args(**{**base, "c_fp32_accumulate": 1}), s) == fq.FP8Q_ERR_UNSUPPORTED       # not with FP32 C
+    assert g(_args(**{**base, "s_out": None}), s) == fq.FP8Q_ERR_NULL
+    assert g(_args(**{**base, "N": 200, "ldc": 200}), s) == fq.FP8Q_ERR_SHAPE               # N % 128
+    assert g(_args(**{**base, "K": 256}), s) == fq.FP8Q_ERR_SHAPE                           # K >= 384
+    assert g(_args(**{**base, "ld_q_out": 264}), s) == fq.FP8Q_ERR_SHAPE                    # % 16
+    assert g(_args(**{**base, "ld_s_out": 100}), s) == fq.FP8Q_ERR_SHAPE                    # >= M
+    assert g(_args(**{**base, "q_out": MISALIGNED.value}), s) == fq.FP8Q_ERR_ALIGN

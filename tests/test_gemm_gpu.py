@@ -11,6 +11,7 @@ import pytest
 import torch
 
 import workloads
+from oracle import formats as F
 from oracle import gemm as G
 from oracle import quant as Q
 
@@ -19,6 +20,10 @@ pytestmark = pytest.mark.gpu
 
 def host(t):
     return t.detach().cpu().numpy()
+
+
+def f32bits(a):
+    return np.ascontiguousarray(a, dtype=np.float32).view(np.uint32)
 
 
 def check(c_gpu, c_ref, t, what):
@@ -121,6 +126,79 @@ def test_blockwise_fp32_accumulate(cuda_lib, layout):
     cin = c_in.numpy().astype(np.float64)
     excess = G.tolerance_violation(got - cin, ref, t) - np.abs(got) * 2.0 ** -24
     assert float(excess.max()) <= 0, f"{int((excess > 0).sum())} elements outside tolerance"
+
+
+def _fused_quant_checks(fq, c, q_out, s_out, ref, t, what):
+    """The fused 1x128 output quantization (1) equals the standalone 1x128 quantizer run on the
+    same BF16 output, bit for bit, and (2) dequantizes to the oracle's product within the GEMM
+    tolerance plus E4M3's rounding bound (half an ulp: 2^-4 relative for normal codes, 2^-10
+    times the decode scale below them), with decode scales within the GEMM tolerance of the
+    oracle's amax / 448 per 128-column group."""
+    M, N = ref.shape
+    qs = fq.quantize_1x128(c, rowwise=True, colwise=False)
+    assert np.array_equal(host(q_out), host(qs["q_row"])), f"{what}: codes differ from the 1x128 quantizer"
+    assert np.array_equal(f32bits(host(s_out)), f32bits(host(qs["s_row"])[:, :M])), f"{what}: scales differ"
+    q = host(q_out)
+    s = host(s_out).astype(np.float64)                       # (N/128, M)
+    deq = F.e4m3_decode(q).astype(np.float64) * np.repeat(s.T, 128, axis=1)
+    g_ref = np.abs(ref).reshape(M, N // 128, 128).max(axis=2)
+    g_t = t.reshape(M, N // 128, 128).max(axis=2)
+    s_bound = np.repeat((g_ref + g_t) / 448.0 * (1 + 2.0 ** -20), 128, axis=1)
+    bound = t + 2.0 ** -4 * (np.abs(ref) + t) + 2.0 ** -10 * s_bound
+    excess = np.abs(deq - ref) - bound
+    assert float(excess.max()) <= 0, f"{what}: {int((excess > 0).sum())} dequantized codes outside the bound"
+    s_ref = g_ref.T / 448.0
+    assert np.all(np.abs(s - s_ref) <= (2.0 ** -7 * s_ref + g_t.T / 448.0) * 1.01 + 1e-30), f"{what}: scales"
+
+
+@pytest.mark.parametrize("M,K,N", [(300, 512, 640), (256, 384, 256), (1, 1024, 128)])
+def test_blockwise_fprop_with_fused_output_quantization(cuda_lib, M, K, N):
+    """fprop whose epilogue also emits the next layer's 1x128 E4M3 codes and scales of Y."""
+    fq = cuda_lib
+    X, W = bf((M, K), 1.0, 71 + M, 1e-3, 50.0), bf((K, N), 0.02, 72 + N)
+    qx = fq.quantize_1x128(X.cuda())
+    qw = fq.quantize_128x128(W.cuda())
+    q_out = torch.empty((M, N), dtype=torch.uint8, device="cuda")
+    s_out = torch.empty((N // 128, M), dtype=torch.float32, device="cuda")
+    c = fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"], b_scale=qw["s"],
+                q_out=q_out, s_out=s_out)
+    assert fq.device_status() == 0
+    ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+    _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+    check(c, ref, t, "fprop (fused quantization)")
+    _fused_quant_checks(fq, c, q_out, s_out, ref, t, "fprop")
+
+
+def test_blockwise_dgrad_and_wgrad_with_fused_output_quantization(cuda_lib):
+    fq = cuda_lib
+    M, Kw, Nw = 256, 384, 512            # dgrad: dY (M x Nw) . W^T -> (M x Kw)
+    W, dY = bf((Kw, Nw), 0.02, 81), bf((M, Nw), 1e-3, 82)
+    qw = fq.quantize_128x128(W.cuda())
+    qd = fq.quantize_1x128(dY.cuda())
+    q_out = torch.empty((M, Kw), dtype=torch.uint8, device="cuda")
+    s_out = torch.empty((Kw // 128, M), dtype=torch.float32, device="cuda")
+    c = fq.gemm(qd["q_row"], qw["q"], fq.FP8Q_BLOCKWISE, fq.FP8Q_DGRAD, a_scale=qd["s_row"], b_scale=qw["s"],
+                ld_sb=(Kw + 127) // 128, q_out=q_out, s_out=s_out)
+    od, osd = Q.quantize_1x128_rowwise(workloads.bf16_bits(dY))
+    ow, _, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+    ref, t = G.reference(G.dequant_a_1x128(od, osd), G.dequant_b_blockwise(ow, osw, G.DGRAD))
+    check(c, ref, t, "dgrad (fused quantization)")
+    _fused_quant_checks(fq, c, q_out, s_out, ref, t, "dgrad")
+    T, Kf, N = 512, 256, 384             # wgrad: X^T . dY over T tokens -> (Kf x N)
+    X, dY2 = bf((T, Kf), 1.0, 83, 1e-3, 50.0), bf((T, N), 1e-3, 84)
+    qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
+    qd2 = fq.quantize_1x128(dY2.cuda(), rowwise=False, colwise=True)
+    q_out = torch.empty((Kf, N), dtype=torch.uint8, device="cuda")
+    s_out = torch.empty((N // 128, Kf), dtype=torch.float32, device="cuda")
+    c = fq.gemm(qx["q_col"], qd2["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                b_scale=qd2["s_col"], q_out=q_out, s_out=s_out)
+    ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
+    od2, osd2 = Q.quantize_1x128_colwise(workloads.bf16_bits(dY2))
+    ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od2, osd2, G.WGRAD))
+    check(c, ref, t, "wgrad (fused quantization)")
+    _fused_quant_checks(fq, c, q_out, s_out, ref, t, "wgrad")
+    assert fq.device_status() == 0
 
 
 @pytest.mark.parametrize("T,Kf,N", [(256, 208, 400), (1024, 256, 512)])
@@ -315,6 +393,38 @@ def test_llama8b_fprop_dgrad_wgrad_sampled(cuda_lib):
         ob, sb = Q.quantize_1x128_colwise(dYb[:, n0:n0 + 128])
         ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
         check(c[m0:m0 + 128, n0:n0 + 128].astype(np.float64), ref, t, f"wgrad tile {m0},{n0}")
+    assert fq.device_status() == 0
+
+
+def test_llama8b_fprop_fused_quantization_fullsize(cuda_lib):
+    """Full-size fprop (8192, 4096, 14336) with the fused 1x128 quantization of Y: codes and
+    scales equal the standalone quantizer's on the same Y everywhere; 64 sampled tiles are
+    checked against the oracle."""
+    fq = cuda_lib
+    d = workloads.llama8b(device="cuda")
+    X, W = d["X"], d["W"]
+    del d
+    M, K, N = X.shape[0], X.shape[1], W.shape[1]
+    qx = fq.quantize_1x128(X)
+    qw = fq.quantize_128x128(W)
+    q_out = torch.empty((M, N), dtype=torch.uint8, device="cuda")
+    s_out = torch.empty((N // 128, M), dtype=torch.float32, device="cuda")
+    c = fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"], b_scale=qw["s"],
+                q_out=q_out, s_out=s_out)
+    qs = fq.quantize_1x128(c, rowwise=True, colwise=False)
+    assert torch.equal(q_out, qs["q_row"]) and torch.equal(s_out.view(torch.int32), qs["s_row"][:, :M].view(torch.int32))
+    Xb, Wb = workloads.bf16_bits(X), workloads.bf16_bits(W)
+    q_h, s_h = host(q_out), host(s_out)
+    c_h = host(c.float()).astype(np.float64)
+    for m0, g0 in _tiles(M, N, 9):           # 128-aligned tiles: one scale group each
+        oa, sa = Q.quantize_1x128_rowwise(Xb[m0:m0 + 128])
+        _, owt, sw = Q.quantize_128x128(Wb[:, g0:g0 + 128])
+        ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+        check(c_h[m0:m0 + 128, g0:g0 + 128], ref, t, f"fprop tile {m0},{g0}")
+        deq = F.e4m3_decode(q_h[m0:m0 + 128, g0:g0 + 128]).astype(np.float64) * s_h[g0 // 128, m0:m0 + 128, None]
+        s_bound = (np.abs(ref).max(axis=1, keepdims=True) + t.max(axis=1, keepdims=True)) / 448.0 * (1 + 2.0 ** -20)
+        excess = np.abs(deq - ref) - (t + 2.0 ** -4 * (np.abs(ref) + t) + 2.0 ** -10 * s_bound)
+        assert float(excess.max()) <= 0, f"fused codes of tile {m0},{g0}"
     assert fq.device_status() == 0
 
 
