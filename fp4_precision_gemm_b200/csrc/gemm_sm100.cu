@@ -404,8 +404,8 @@ struct BwCfg {
 
 
 // Shared memory of the blockwise kernel.  A scale-ring slot holds one chunk's scales:
-// wgrad: [B scales of the 192 columns][A scales of the CTA's 128 rows];
-// fprop/dgrad: [A scales][the B scales of the tile's three 64-column groups].
+// wgrad: [B scales of the tile's 256 columns][A scales of the CTA's 128 rows];
+// fprop/dgrad: [A scales][the B scales of the tile's four 64-column groups].
 template <int L>
 struct BwSmem {
   using C = BwCfg;
@@ -647,7 +647,7 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
       mbar_wait_drain(final_bar, 0, kWaitLimitNs);
     }
   } else {
-    // ------------------------------------------------------------------ promotion warps 0-11
+    // ------------------------------------------------------------------ promotion warps 0-15
     const int q = warp & 3, cgp = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cgp * 64);
     const int rloc = q * 32 + lane;
