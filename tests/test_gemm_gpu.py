@@ -216,6 +216,52 @@ def test_blockwise_wgrad(cuda_lib, T, Kf, N):
     check(c, ref, t, "wgrad")
 
 
+@pytest.mark.parametrize("layout", ["fprop", "dgrad", "wgrad", "wgrad_acc32"])
+def test_blockwise_partial_last_wave(cuda_lib, layout):
+    """80 output tiles of 256 x 256 on the persistent grid (74 CTA pairs on 148 SMs): a second,
+    mostly empty wave, in every layout and the FP32-accumulate epilogue.  Every element is
+    checked against the oracle."""
+    fq = cuda_lib
+    M, N, K = 2048, 2560, 1024
+    if layout == "fprop":
+        X, W = bf((M, K), 1.0, 91, 1e-3, 50.0), bf((K, N), 0.02, 92)
+        qx, qw = fq.quantize_1x128(X.cuda()), fq.quantize_128x128(W.cuda())
+        c = fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"], b_scale=qw["s"])
+        ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+        _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+        check(c, ref, t, "fprop, partial last wave")
+    elif layout == "dgrad":
+        dY, W = bf((M, K), 1e-3, 93), bf((N, K), 0.02, 94)          # W: N x K codes read along N
+        qd, qw = fq.quantize_1x128(dY.cuda()), fq.quantize_128x128(W.cuda())
+        c = fq.gemm(qd["q_row"], qw["q"], fq.FP8Q_BLOCKWISE, fq.FP8Q_DGRAD, a_scale=qd["s_row"], b_scale=qw["s"],
+                    ld_sb=N // 128)
+        od, osd = Q.quantize_1x128_rowwise(workloads.bf16_bits(dY))
+        ow, _, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+        ref, t = G.reference(G.dequant_a_1x128(od, osd), G.dequant_b_blockwise(ow, osw, G.DGRAD))
+        check(c, ref, t, "dgrad, partial last wave")
+    else:
+        X, dY = bf((K, M), 1.0, 95, 1e-3, 50.0), bf((K, N), 1e-3, 96)   # K tokens
+        qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
+        qd = fq.quantize_1x128(dY.cuda(), rowwise=False, colwise=True)
+        ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
+        od, osd = Q.quantize_1x128_colwise(workloads.bf16_bits(dY))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od, osd, G.WGRAD))
+        if layout == "wgrad":
+            c = fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                        b_scale=qd["s_col"])
+            check(c, ref, t, "wgrad, partial last wave")
+        else:
+            c_in = torch.full((M, N), 0.5, dtype=torch.float32)
+            c = c_in.cuda()
+            fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                    b_scale=qd["s_col"], out=c, accumulate_fp32=True)
+            got = host(c).astype(np.float64)
+            excess = G.tolerance_violation(got - 0.5, ref, t) - np.abs(got) * 2.0 ** -24
+            assert float(excess.max()) <= 0, f"{int((excess > 0).sum())} elements outside tolerance"
+    assert fq.device_status() == 0
+
+
 def test_blockwise_more_tiles_than_sms(cuda_lib):
     """2048 x 4096 output = 256 tiles: every CTA runs the persistent loop more than once."""
     fq = cuda_lib
