@@ -1,9 +1,26 @@
-"""Pins for Philox (statistical here; bit-exact against cuRAND in the GPU tests) and for the
-random Hadamard transform (Sylvester Hadamard matrix from SciPy, orthogonality)."""
+"""Pins for Philox (the generator's published known-answer vectors, statistics here;
+bit-exact against cuRAND in the GPU tests) and for the random Hadamard transform (Sylvester
+Hadamard matrix from SciPy, orthogonality)."""
+import os
+
 import numpy as np
 import scipy.linalg
 
 from oracle import philox, rht
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def test_philox_known_answer_vectors():
+    """tests/golden/philox4x32_10_kat.txt: counter, key -> output words published with the
+    generator's reference implementation."""
+    rows = [line.split() for line in open(os.path.join(GOLDEN, "philox4x32_10_kat.txt"))
+            if line.strip() and not line.startswith("#")]
+    assert len(rows) == 3
+    for r in rows:
+        w = [int(x, 16) for x in r]
+        out = philox.philox4x32_10(np.array([w[0:4]], dtype=np.uint32), np.array(w[4:6], dtype=np.uint32))
+        assert [int(x) for x in np.asarray(out).ravel()] == w[6:10]
 
 
 def test_philox_deterministic_and_key_sensitive():
