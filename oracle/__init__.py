@@ -9,14 +9,16 @@ none of the method's arithmetic.
 
 The oracle is written in NumPy from the definitions:
 
-* ``formats``  E4M3 / E8M0 / E2M1 / BF16 codecs from their bit definitions
-  (OCP 8-bit floating point spec for E4M3, OCP MX spec v1.0 for E8M0 and E2M1).
+* ``formats``  E4M3 / E5M2 / E8M0 / E2M1 / BF16 codecs from their bit definitions
+  (OCP 8-bit floating point spec for E4M3 and E5M2, OCP MX spec v1.0 for E8M0 and E2M1).
 * ``philox``   Philox4x32-10, the counter-based generator of Salmon, Moraes, Dror and
-  Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11).
+  Shaw, "Parallel Random Numbers: As Easy as 1, 2, 3" (SC'11), pinned by the generator's
+  published known-answer vectors (``tests/golden/philox4x32_10_kat.txt``).
 * ``rht``      the 16x16 random Hadamard transform used on gradient inputs.
 * ``quant``    the quantizers: 1x128 tiles, 128x128 blocks, MX (32-element blocks,
-  E8M0 scales), per-tensor current scaling, NVFP4 (E2M1 values, per-16 E4M3 scales,
-  a per-tensor FP32 scale, optional RHT and stochastic rounding).
+  E8M0 scales), per-tensor current and delayed scaling (E4M3 or E5M2), NVFP4 (E2M1
+  values, per-16 E4M3 scales, a per-tensor FP32 scale, optional RHT and stochastic
+  rounding; 16x16 blocks for weights).
 * ``gemm``     dequantization and the FP64 reference product with the tolerance check.
 
 The pages the method comes from (cited by title in every module):
