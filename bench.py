@@ -796,16 +796,24 @@ class ClockSampler:
             self.proc.wait(timeout=5)
         except subprocess.TimeoutExpired:
             self.proc.kill()
-        rows = []
         with open(self.path) as f:
-            for line in f:
-                parts = [p.strip() for p in line.split(",")]
-                if len(parts) == 7:
-                    try:
-                        rows.append((float(parts[0]), float(parts[1]), parts[3:]))
-                    except ValueError:
-                        pass
+            lines = f.readlines()
         os.unlink(self.path)
+        return self.summarize(lines)
+
+    @staticmethod
+    def summarize(lines):
+        """nvidia-smi CSV lines (the fields of Q, no header, no units) -> median SM clock,
+        maximum SM clock, throttle reasons seen Active in any sample, sample count.  Lines
+        that do not parse (a partial last line when the sampler is stopped) are skipped."""
+        rows = []
+        for line in lines:
+            parts = [p.strip() for p in line.split(",")]
+            if len(parts) == 7:
+                try:
+                    rows.append((float(parts[0]), float(parts[1]), parts[3:]))
+                except ValueError:
+                    pass
         names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
         reasons = sorted({names[i] for _, _, r in rows for i, v in enumerate(r) if v.lower() == "active"})
         if not rows:
