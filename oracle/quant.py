@@ -237,7 +237,10 @@ def nvfp4_global_scale(G):
 
 
 def sr_words(idx, tag, sr_seed):
-    """Philox word for each linear output index idx (int64 array)."""
+    """Philox word for each linear output index idx (int64 array): word idx & 3 of the call
+    at counter (idx >> 2, 0, tag).  Pinned statistically (the words of the four elements of
+    one call, and of neighbouring calls, give uncorrelated decisions; tags 0 and 1 give
+    uncorrelated streams) and by element-wise brute force over output indices."""
     idx = np.asarray(idx, dtype=np.int64)
     blk = (idx >> 2).astype(np.uint64)
     ctr = np.stack([(blk & np.uint64(0xFFFFFFFF)).astype(np.uint32),
@@ -251,7 +254,8 @@ def sr_words(idx, tag, sr_seed):
 def e2m1_encode_sr(y, words):
     """Stochastic rounding of float32 y to E2M1 with one random 32-bit word per element.
 
-    Parity unpinned for the word -> uniform mapping; unbiasedness is pinned statistically.
+    The word -> uniform mapping (top 24 bits, round up iff u < p) is a reading: it is pinned
+    for unbiasedness over 10^6 draws; which word an element takes is pinned in sr_words.
     """
     y = np.asarray(y, dtype=np.float32)
     a = np.abs(y)

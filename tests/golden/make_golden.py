@@ -35,6 +35,16 @@ def small_input():
     return F.f32_to_bf16_bits(x)
 
 
+def nvfp4_input():
+    """The same input without its near-maximum value (row 1 holds 96.0 there instead).  NVFP4
+    scales every 16-block against the tensor amax, so with 3e38 in the tensor every other
+    block scale would round to zero; here most blocks get a non-zero E4M3 scale and the
+    stochastic-rounding and transform entries make real decisions."""
+    x = small_input().copy()
+    x[1, 17] = F.f32_to_bf16_bits(np.array([96.0], np.float32))[0]
+    return x
+
+
 def hexes(a, width):
     """One hex string per row (each element `width` hex digits)."""
     a = np.atleast_2d(np.asarray(a))
@@ -50,14 +60,16 @@ def build():
     q1, s1 = Q.quantize_1x128_rowwise(x)
     qm, em = Q.quantize_mx_rowwise(x)
     qt, st = Q.quantize_tensor(x)
-    n_q, n_s, n_g = Q.quantize_nvfp4_rowwise(x)
-    r_q, r_s, r_g = Q.quantize_nvfp4_rowwise(x, rht=True, rht_seed=5, sr=True, sr_seed=6)
-    c_q, c_s, c_g = Q.quantize_nvfp4_colwise(x, rht=True, rht_seed=5, sr=True, sr_seed=6)
-    w_row, w_sr, w_col, w_sc, w_g = Q.quantize_nvfp4_2d(x)
+    x4 = nvfp4_input()
+    n_q, n_s, n_g = Q.quantize_nvfp4_rowwise(x4)
+    r_q, r_s, r_g = Q.quantize_nvfp4_rowwise(x4, rht=True, rht_seed=5, sr=True, sr_seed=6)
+    c_q, c_s, c_g = Q.quantize_nvfp4_colwise(x4, rht=True, rht_seed=5, sr=True, sr_seed=6)
+    w_row, w_sr, w_col, w_sc, w_g = Q.quantize_nvfp4_2d(x4)
     return {
         "source": "tests/golden/make_golden.py (oracle/ only)",
         "shape": [16, 128],
         "x_bf16": hexes(x, 4),
+        "x_nvfp4_bf16": hexes(x4, 4),
         "1x128_rowwise": {"cite": "Can you explain the role of FP8 precision in DeepSeek-V3 training, "
                                   "Fine-grained quantization / Online quantization",
                           "q": hexes(q1, 2), "s": f32hex(s1)},

@@ -217,6 +217,93 @@ def test_nvfp4_sr_is_unbiased_and_picks_neighbours():
     assert np.array_equal(q, q2) and not np.array_equal(q, q3)
 
 
+def _sr_pattern(R, C):
+    """R x C values whose NVFP4 quantization leaves one fair coin per element: each 16-group
+    holds one anchor 6.0 (the block and tensor amax, so S_g = 448, the block scale is 448 and
+    the encode scale is exactly 1) and fifteen 1.25s, which sit halfway between the E2M1
+    values 1.0 (code 2) and 1.5 (code 3).  With p = 1/2 the reading's rule rounds up iff the
+    element's 32-bit Philox word is below 2^31."""
+    x = np.full((R, C), 1.25, np.float32)
+    x[:, 0::16] = 6.0
+    return x
+
+
+def _up(q_packed):
+    """Rounding decisions (True = up to 1.5) of a quantized _sr_pattern, as a code matrix."""
+    codes = F.unpack_e2m1(q_packed)
+    fair = codes != 7
+    assert set(np.unique(codes[fair])) <= {2, 3}
+    return codes == 3
+
+
+def _corr(a, b):
+    a = a.astype(np.float64) - a.mean()
+    b = b.astype(np.float64) - b.mean()
+    return float((a * b).sum() / np.sqrt((a * a).sum() * (b * b).sum()))
+
+
+def test_nvfp4_sr_words_are_independent_within_and_across_philox_blocks():
+    """Reading: element idx of an output takes word (idx & 3) of the Philox call at counter
+    idx >> 2.  Over ~10^6 fair coins the decisions of the four elements sharing one call,
+    and of the same element slot in neighbouring calls, must be uncorrelated (|r| < 4/sqrt(n)):
+    a word mapping that reuses one word for several elements (e.g. always word 0, or word
+    (idx >> 2) & 3) makes them identical."""
+    R, C = 1024, 1088
+    x = _sr_pattern(R, C)
+    for name, (q, _, _) in (("rowwise", Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=6)),
+                            ("colwise", Q.quantize_nvfp4_colwise(np.ascontiguousarray(x.T), sr=True, sr_seed=6))):
+        d = _up(q).reshape(-1, 16)[:, 4:].reshape(-1, 3, 4)    # Philox blocks 1..3 of each group
+        n = d.shape[0]
+        assert 3 * 4 * n >= 1_000_000 - 200_000 and abs(d.mean() - 0.5) < 4 * 0.5 / np.sqrt(d.size)
+        bound = 4.0 / np.sqrt(n)
+        for blk in range(3):
+            for i in range(4):
+                for j in range(i + 1, 4):
+                    r = _corr(d[:, blk, i], d[:, blk, j])
+                    assert abs(r) < bound, (name, "same call", blk, i, j, r)
+        for blk in range(2):
+            for i in range(4):
+                r = _corr(d[:, blk, i], d[:, blk + 1, i])
+                assert abs(r) < bound, (name, "neighbouring calls", blk, i, r)
+
+
+def test_nvfp4_sr_rowwise_and_colwise_outputs_draw_from_different_streams():
+    """The two outputs of one tensor use tags 0 and 1: at the same output index their fair
+    coins must be uncorrelated (one stream for both would make them identical)."""
+    x = _sr_pattern(1024, 1024)
+    q_row, _, _ = Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=11)
+    q_col, _, _ = Q.quantize_nvfp4_colwise(np.ascontiguousarray(x.T), sr=True, sr_seed=11)
+    a, b = _up(q_row).ravel(), _up(q_col).ravel()
+    keep = (np.arange(a.size) % 16) != 0
+    assert abs(_corr(a[keep], b[keep])) < 4.0 / np.sqrt(keep.sum())
+
+
+def test_nvfp4_sr_decisions_match_brute_force_over_output_indices():
+    """Brute force on a small non-square input: every fair coin of the rowwise output (R x C,
+    tag 0) and of the colwise output (C x R, transposed, tag 1) is recomputed element by
+    element from one scalar call of the generator (pinned by its published known-answer
+    vectors) at counter (idx >> 2, 0, 0, tag), word idx & 3, idx the element's position in
+    that output.  A colwise output indexed by the input position, a wrong word or a wrong
+    counter split fails here."""
+    from oracle.philox import philox4x32_10, seed_to_key
+    R, C = 48, 32
+    x = _sr_pattern(R, C)                       # rowwise coins along rows
+    xc = np.ascontiguousarray(_sr_pattern(C, R).T)   # R x C; colwise coins along columns
+    key = seed_to_key(0x1234_5678_9ABC)
+    cases = ((Q.quantize_nvfp4_rowwise(x, sr=True, sr_seed=0x1234_5678_9ABC)[0], 0, (R, C)),
+             (Q.quantize_nvfp4_colwise(xc, sr=True, sr_seed=0x1234_5678_9ABC)[0], 1, (C, R)))
+    for q, tag, (orows, ocols) in cases:
+        up = _up(q)
+        assert up.shape == (orows, ocols)
+        for r in range(orows):
+            for c in range(ocols):
+                if c % 16 == 0:
+                    continue
+                idx = r * ocols + c
+                w = philox4x32_10(np.array([idx >> 2, 0, 0, tag], np.uint32), key)[idx & 3]
+                assert bool(up[r, c]) == (int(w) < (1 << 31)), (tag, r, c)
+
+
 def test_nvfp4_rht_roundtrip_close_and_orthogonal_gemm():
     rng = np.random.default_rng(8)
     A = rng.standard_normal((32, 256)).astype(np.float32)
