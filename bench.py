@@ -11,8 +11,11 @@ Metric: block-scaled GEMM TFLOP/s (the step's GEMM FLOPs over the whole step's d
 quantization included) with per-kernel TFLOP/s and GB/s as fractions of the roofline.
 
 Contract: python bench.py --gpus N --steps K --warmup W [--impl ours|reference]
-  * N > 1 runs under torch.distributed.run, one rank per GPU; every rank runs the step on
-    its own tokens (weak scaling, no data-path collective); timing is the max over ranks.
+  * N > 1: one rank per GPU under torch.distributed.run.  Launched without a WORLD_SIZE in
+    the environment, bench.py starts torch.distributed.run itself with N ranks; launched
+    by torch.distributed.run, it checks that WORLD_SIZE == N.  Every rank runs the step on
+    its own tokens (weak scaling, no data-path collective); timing is the max over ranks
+    (an all-reduce MAX over the NCCL group), and the line reports the group's size.
   * Inputs live in HBM before the timed region; the L2 is flushed between steps (a 256 MiB
     write, then a 256 MiB read so no dirty lines remain), outside the per-step events.
   * --impl reference times the CPU oracle (rank 0 only) on a bounded sample of the step.
@@ -169,21 +172,43 @@ class LlamaStep:
                           "quantized by the oracle from the BF16 inputs, FP64 reference product")
 
 
+def _llama_cpu_quant_sample(self):
+    """Oracle quantizers on the step's full X (1x128 rowwise and colwise) and W (128x128,
+    both layouts): algorithmic bytes, seconds, description (single-threaded NumPy)."""
+    from oracle import quant as Q
+    if not hasattr(self, "_host_bits"):
+        self._host_bits = tuple(workloads.bf16_bits(t) for t in (self.X, self.W, self.dY))
+    Xb, Wb, _ = self._host_bits
+    M, K, N = self.M, self.K, self.N
+    t0 = time.perf_counter()
+    Q.quantize_1x128_rowwise(Xb)
+    Q.quantize_1x128_colwise(Xb)
+    Q.quantize_128x128(Wb)
+    dt = time.perf_counter() - t0
+    return (b_1x128_fused(M, K) + b_128(K, N), dt,
+            f"1x128 rowwise+colwise of the full X ({M}x{K}) and 128x128 both layouts of the full W ({K}x{N})")
+
+
+LlamaStep.cpu_quant_sample = _llama_cpu_quant_sample
+
+
 class TinyStep(LlamaStep):
     name = "tiny"
     workload = "tiny blockwise fprop: A 256x512, B 512x256"
 
-    def __init__(self, fq, rank):
+    def __init__(self, fq, rank, device="cuda"):
         self.fq = fq
-        d = workloads.tiny(device="cuda")
+        d = workloads.tiny(device=device)
         self.A, self.B = d["A"], d["B"]
+        self.gemm_flop = 2.0 * 256 * 256 * 512
+        if device == "cpu":          # host inputs only: the oracle's sample needs nothing else
+            return
         dev = self.A.device
         self.qa = torch.empty((256, 512), dtype=torch.uint8, device=dev)
         self.sa = torch.empty((4, 256), dtype=torch.float32, device=dev)
         self.qbt = torch.empty((256, 512), dtype=torch.uint8, device=dev)
         self.sb = torch.empty((2, 4), dtype=torch.float32, device=dev)
         self.C = torch.empty((256, 256), dtype=torch.bfloat16, device=dev)
-        self.gemm_flop = 2.0 * 256 * 256 * 512
 
     def inputs(self):
         return [self.A, self.B]
@@ -971,7 +996,7 @@ def measure_e2e(step, launches, stream, args, make_step, world):
     h_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs[0]]
     bi = sum(t.numel() * t.element_size() for t in ins[0])
     bo = sum(t.numel() * t.element_size() for t in outs[0])
-    reps = max(4, min(args.steps, 8))
+    reps = max(4, args.steps)
     s_in, s_out = torch.cuda.Stream(), torch.cuda.Stream()
     ev_in = [torch.cuda.Event() for _ in range(2)]
     ev_c = [torch.cuda.Event() for _ in range(2)]
@@ -1027,6 +1052,17 @@ def cpu_cores():
         return int(torch.get_num_threads())
 
 
+def cpu_model():
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return None
+
+
 def cpu_baseline(step):
     blas = cpu_cores()
     # a bounded sample of about 12 s of CPU work: time one sampled tile per GEMM, then size
@@ -1034,19 +1070,31 @@ def cpu_baseline(step):
     _, dt1, _ = step.cpu_sample(tiles=1)
     tiles = max(1, min(64, int(12.0 / max(dt1, 1e-3))))
     flop, dt, what = step.cpu_sample(tiles=tiles)
-    return {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": int(blas), "kind": "oracle",
-            "sample": what, "seconds": round(dt, 2)}
+    out = {"value": round(flop / dt / 1e12, 6), "unit": "TFLOP/s", "cores": int(blas), "kind": "oracle",
+           "sample": what, "seconds": round(dt, 2), "cpu_model": cpu_model(), "host_threads": os.cpu_count()}
+    if hasattr(step, "cpu_quant_sample"):
+        # the quantizers' oracle: elementwise NumPy, one thread whatever the BLAS thread count
+        nbytes, qdt, qwhat = step.cpu_quant_sample()
+        out["quantize"] = {"value": round(nbytes / qdt / 1e9, 4), "unit": "GB/s", "cores": 1, "kind": "oracle",
+                           "sample": qwhat, "seconds": round(qdt, 2)}
+    return out
 
 
 def run_reference(args, rank, world):
-    """The CPU oracle as it stands, timed on the host cores on a bounded sample per step."""
+    """The CPU oracle as it stands, timed on the host cores on a bounded sample per step.
+    Rank 0 alone runs it; the other ranks do no work."""
     if rank != 0:
         return None
-    torch.cuda.set_device(0) if torch.cuda.is_available() else None
+    cuda = torch.cuda.is_available()
+    if cuda:
+        torch.cuda.set_device(0)
     import fp4_precision_gemm_b200 as fq
-    step = STEPS[args.workload](fq, 0) if torch.cuda.is_available() else None
-    if step is None:
-        return {"impl": "reference", "unavailable": "the oracle's inputs are generated on a CUDA device"}
+    if cuda:
+        step = STEPS[args.workload](fq, 0)
+    elif args.workload == "tiny":
+        step = TinyStep(fq, 0, device="cpu")     # inputs drawn on the host (same recipe, CPU generator)
+    else:
+        return {"impl": "reference", "unavailable": "no CUDA device: the inputs of this workload are drawn on the GPU"}
     for _ in range(args.warmup):
         step.cpu_sample()
     flops, secs = 0.0, 0.0
@@ -1067,6 +1115,41 @@ def run_reference(args, rank, world):
             "e2e": {"value": round(value, 6), "unit": "TFLOP/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
 
 
+def free_port():
+    import socket
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        return sk.getsockname()[1]
+
+
+def spawn_ranks(n, argv, timeout_s=None):
+    """Runs this script as n ranks under torch.distributed.run on 127.0.0.1 (one node) and
+    returns its exit code; each rank sees RANK / LOCAL_RANK / WORLD_SIZE in its environment."""
+    cmd = [sys.executable, "-m", "torch.distributed.run", "--nnodes", "1", "--nproc-per-node", str(n),
+           "--master-addr", "127.0.0.1", "--master-port", str(free_port()), os.path.abspath(__file__)] + list(argv)
+    return subprocess.call(cmd, timeout=timeout_s)
+
+
+def init_ranks(n_expected, backend):
+    """Reads the launcher's environment, checks that it started n_expected ranks, and joins
+    the process group (short timeout, so ranks that wait for a lost peer end with an error).
+    Returns (rank, world, local_rank)."""
+    import datetime
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+    if world != n_expected:
+        raise SystemExit(f"bench.py: --gpus {n_expected} but the launcher started WORLD_SIZE={world} ranks")
+    if world > 1:
+        kw = {}
+        if backend == "nccl":
+            torch.cuda.set_device(local_rank)
+            kw["device_id"] = torch.device("cuda", local_rank)
+        torch.distributed.init_process_group(backend, timeout=datetime.timedelta(seconds=600 if backend == "gloo"
+                                                                                  else 120), **kw)
+    return rank, world, local_rank
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -1082,15 +1165,16 @@ def main():
     args.warmup = max(args.warmup, 3)
     if args.tokens and args.workload != "llama8b":
         ap.error("--tokens applies to the llama8b workload only")
+    if args.gpus < 1:
+        ap.error("--gpus must be >= 1")
+    if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
+        sys.exit(spawn_ranks(args.gpus, sys.argv[1:]))
 
-    world = int(os.environ.get("WORLD_SIZE", "1"))
-    rank = int(os.environ.get("RANK", "0"))
-    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
-    if world > 1 and args.impl == "ours":
-        import datetime
-        torch.cuda.set_device(local_rank)
-        torch.distributed.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
-                                             device_id=torch.device("cuda", local_rank))
+    backend = "nccl" if (args.impl == "ours" and torch.cuda.is_available()) else "gloo"
+    rank, world, local_rank = init_ranks(args.gpus, backend)
+    comm = None
+    if world > 1:
+        comm = {"backend": torch.distributed.get_backend(), "world_size": torch.distributed.get_world_size()}
     names = sorted(STEPS) if args.workload == "all" else [args.workload]
     for name in names:
         args.workload = name
@@ -1099,8 +1183,11 @@ def main():
         else:
             out = run_ours(args, rank, world, local_rank)
         if rank == 0 and out is not None:
+            if comm is not None and "unavailable" not in out:
+                out["comm"] = comm
             print(json.dumps(out), flush=True)
-    if world > 1 and args.impl == "ours":
+    if world > 1:
+        torch.distributed.barrier()
         torch.distributed.destroy_process_group()
 
 

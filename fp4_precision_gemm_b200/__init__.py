@@ -29,6 +29,7 @@ __all__ = [
 
 FP8Q_OK = 0
 FP8Q_ERR_NULL, FP8Q_ERR_SHAPE, FP8Q_ERR_ALIGN, FP8Q_ERR_UNSUPPORTED, FP8Q_ERR_CUDA, FP8Q_ERR_TIMEOUT = 1, 2, 3, 4, 5, 6
+FP8Q_ERR_DEVICE_ARG = 7
 FP8Q_BLOCKWISE, FP8Q_MXFP8, FP8Q_PERTENSOR, FP8Q_NVFP4 = 0, 1, 2, 3
 FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD = 0, 1, 2
 FP8Q_SF_ROWMAJOR, FP8Q_SF_MMA_TILED = 0, 1

@@ -19,7 +19,9 @@ constexpr int kMaxDevices = 64;
 constexpr int kAmaxSlots = 1024;  // rotating 8-byte slots for global amax words
 
 struct DeviceScratch {
-  uint32_t* base = nullptr;  // [0] status word, [64 + 2*i] amax slot i
+  // [0] status word, [64 + 2*i] amax slot i.  Published with release order after num_sms
+  // is set, read with acquire order, so a thread that sees the pointer sees the pool whole.
+  std::atomic<uint32_t*> base{nullptr};
   std::atomic<uint32_t> next{0};
   int num_sms = 0;
 };
@@ -36,9 +38,9 @@ fp8q_status scratch(DeviceScratch** out) {
   int dev = 0;
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
   DeviceScratch& d = g_scratch[dev];
-  if (d.base == nullptr) {
+  if (d.base.load(std::memory_order_acquire) == nullptr) {
     std::lock_guard<std::mutex> lock(g_mutex);
-    if (d.base == nullptr) {
+    if (d.base.load(std::memory_order_relaxed) == nullptr) {
       int sms = 0;
       if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) return FP8Q_ERR_CUDA;
       void* p = nullptr;
@@ -46,7 +48,7 @@ fp8q_status scratch(DeviceScratch** out) {
       if (cudaMalloc(&p, bytes) != cudaSuccess) return FP8Q_ERR_CUDA;
       if (cudaMemset(p, 0, bytes) != cudaSuccess) return FP8Q_ERR_CUDA;
       d.num_sms = sms;
-      d.base = static_cast<uint32_t*>(p);
+      d.base.store(static_cast<uint32_t*>(p), std::memory_order_release);
     }
   }
   *out = &d;
@@ -56,7 +58,7 @@ fp8q_status scratch(DeviceScratch** out) {
 // Next pair of amax words, zeroed on `stream` before use.
 fp8q_status amax_slot(DeviceScratch* d, cudaStream_t s, uint32_t** out) {
   const uint32_t i = d->next.fetch_add(1) % kAmaxSlots;
-  uint32_t* p = d->base + 64 + 2 * i;
+  uint32_t* p = d->base.load(std::memory_order_acquire) + 64 + 2 * i;
   if (cudaMemsetAsync(p, 0, 2 * sizeof(uint32_t), s) != cudaSuccess) return FP8Q_ERR_CUDA;
   *out = p;
   return FP8Q_OK;
@@ -106,6 +108,7 @@ const char* fp8q_status_string(fp8q_status s) {
     case FP8Q_ERR_UNSUPPORTED: return "unsupported combination";
     case FP8Q_ERR_CUDA: return "CUDA runtime/driver error";
     case FP8Q_ERR_TIMEOUT: return "a kernel's bounded wait ran out";
+    case FP8Q_ERR_DEVICE_ARG: return "an argument read on the device was out of range (clamped)";
   }
   return "unknown status";
 }
@@ -125,8 +128,9 @@ fp8q_status fp8q_get_device_status(void* stream) {
   if (st != FP8Q_OK) return st;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t word = 0;
-  if (cudaMemcpyAsync(&word, d->base, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FP8Q_ERR_CUDA;
-  if (cudaMemsetAsync(d->base, 0, sizeof(uint32_t), s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  uint32_t* base = d->base.load(std::memory_order_acquire);
+  if (cudaMemcpyAsync(&word, base, sizeof(word), cudaMemcpyDeviceToHost, s) != cudaSuccess) return FP8Q_ERR_CUDA;
+  if (cudaMemsetAsync(base, 0, sizeof(uint32_t), s) != cudaSuccess) return FP8Q_ERR_CUDA;
   if (cudaStreamSynchronize(s) != cudaSuccess) return FP8Q_ERR_CUDA;
   return word == 0 ? FP8Q_OK : static_cast<fp8q_status>(word);
 }
@@ -136,7 +140,8 @@ fp8q_status fp8q_selftest_bounded_wait(uint64_t limit_ns, void* stream) {
   DeviceScratch* d = nullptr;
   fp8q_status st = scratch(&d);
   if (st != FP8Q_OK) return st;
-  return from_cuda(launch_selftest_wait(d->base, limit_ns, static_cast<cudaStream_t>(stream)));
+  return from_cuda(launch_selftest_wait(d->base.load(std::memory_order_acquire), limit_ns,
+                                       static_cast<cudaStream_t>(stream)));
 }
 
 fp8q_status fp8q_release_scratch(void) {
@@ -144,10 +149,11 @@ fp8q_status fp8q_release_scratch(void) {
   if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) return FP8Q_ERR_CUDA;
   std::lock_guard<std::mutex> lock(g_mutex);
   DeviceScratch& d = g_scratch[dev];
-  if (d.base) {
+  uint32_t* base = d.base.load(std::memory_order_acquire);
+  if (base) {
     if (cudaDeviceSynchronize() != cudaSuccess) return FP8Q_ERR_CUDA;
-    if (cudaFree(d.base) != cudaSuccess) return FP8Q_ERR_CUDA;
-    d.base = nullptr;
+    d.base.store(nullptr, std::memory_order_release);
+    if (cudaFree(base) != cudaSuccess) return FP8Q_ERR_CUDA;
   }
   return FP8Q_OK;
 }
@@ -251,12 +257,8 @@ fp8q_status fp8q_quantize_tensor(const void* x, int64_t rows, int64_t cols, int6
   if ((st = scratch(&d)) != FP8Q_OK) return st;
   uint32_t* amax = nullptr;
   if ((st = amax_slot(d, s, &amax)) != FP8Q_OK) return st;
-  if (rows == 0 || cols == 0) {
-    // empty tensor: amax 0 -> sf 1 -> decode scale 1
-    const float one = 1.0f;
-    return from_cuda(cudaMemcpyAsync(s_dec, &one, sizeof(float), cudaMemcpyHostToDevice, s) == cudaSuccess
-                         ? cudaStreamSynchronize(s) : cudaErrorUnknown);
-  }
+  if (rows == 0 || cols == 0)   // empty tensor: amax 0 -> sf 1 -> decode scale 1, written on `stream`
+    return from_cuda(launch_fill_f32(s_dec, 1.0f, s));
   cudaError_t e = launch_tensor_amax(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax, s);
   if (e == cudaSuccess) e = launch_tensor_cast(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax, q, s_dec, s);
   return from_cuda(e);
@@ -456,7 +458,7 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   DeviceScratch* d = nullptr;
   fp8q_status st = scratch(&d);
   if (st != FP8Q_OK) return st;
-  p.status = d->base;
+  p.status = d->base.load(std::memory_order_acquire);
 
   CUtensorMap ma, mb, msb;
   const int64_t b_rows = grouped ? (int64_t)a->num_groups * a->N : a->N;

@@ -9,6 +9,7 @@ namespace fp8q {
 
 // Status word codes written by kernels (match fp8q_status).
 constexpr uint32_t kDevTimeout = 6;
+constexpr uint32_t kDevBadArg = 7;
 
 // ------------------------------------------------------------------ BF16
 // A 32-bit word holds two BF16 values, the lower-addressed one in bits 0..15.

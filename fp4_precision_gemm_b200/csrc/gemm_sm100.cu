@@ -462,11 +462,21 @@ __device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row
   return T;
 }
 
+// Expert row offsets into shared memory, clamped to [previous offset, M] so that no tile
+// reaches outside C even when the caller's offsets break their rule (the clamp is recorded
+// in the status word), and the prefix count of 256-row pair tiles per expert.
 __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefix, int* offs, int lane) {
   for (int g = lane; g <= p.num_groups; g += 32) offs[g] = p.m_offsets[g];
   __syncwarp();
   if (lane == 0) {
-    int acc = 0;
+    int acc = 0, prev = 0;
+    bool bad = false;
+    for (int g = 0; g <= p.num_groups; ++g) {
+      const int v = offs[g], c = min(max(v, prev), p.M);
+      bad |= (c != v);
+      offs[g] = prev = c;
+    }
+    if (bad && blockIdx.x == 0) atomicExch(p.status, kDevBadArg);
     for (int g = 0; g < p.num_groups; ++g) {
       prefix[g] = acc;
       acc += (offs[g + 1] - offs[g] + kBwPairM - 1) / kBwPairM;

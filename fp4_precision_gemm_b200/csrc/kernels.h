@@ -51,6 +51,9 @@ struct Fp4QuantParams {
   uint32_t* amax_bits;  // [0]: rowwise output's global amax, [1]: colwise output's
 };
 
+// One float written on the stream (the decode scale of an empty tensor), no host sync.
+cudaError_t launch_fill_f32(float* dst, float v, cudaStream_t s);
+
 cudaError_t launch_tensor_delayed(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x, float* hist,
                                   int hlen, int pos, bool e5m2, uint8_t* q, float* s_dec, uint32_t* amax_bits,
                                   cudaStream_t s);

@@ -78,6 +78,13 @@ cudaError_t launch_tensor_cast(const uint16_t* x, int64_t rows, int64_t cols, in
   return cudaGetLastError();
 }
 
+__global__ void fill_f32_kernel(float* dst, float v) { *dst = v; }
+
+cudaError_t launch_fill_f32(float* dst, float v, cudaStream_t s) {
+  fill_f32_kernel<<<1, 1, 0, s>>>(dst, v);
+  return cudaGetLastError();
+}
+
 // ------------------------------------------------------------------ delayed scaling
 // One pass: the scale comes from the largest amax of earlier iterations (the history), so
 // every CTA can cast as it reads; the tensor's own amax is reduced on the way (one
@@ -199,11 +206,8 @@ extern "C" fp8q_status fp8q_quantize_tensor_noalloc(const void* x, int64_t rows,
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   uint32_t* amax = nullptr;
   if (noalloc_scratch(&amax) != cudaSuccess) return FP8Q_ERR_CUDA;
-  if (rows == 0 || cols == 0) {
-    const float one = 1.0f;  // empty tensor: amax 0 -> sf 1 -> decode scale 1
-    if (cudaMemcpyAsync(s_dec, &one, sizeof(float), cudaMemcpyHostToDevice, s) != cudaSuccess) return FP8Q_ERR_CUDA;
-    return cudaStreamSynchronize(s) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
-  }
+  if (rows == 0 || cols == 0)   // empty tensor: amax 0 -> sf 1 -> decode scale 1, written on `stream`
+    return launch_fill_f32(s_dec, 1.0f, s) == cudaSuccess ? FP8Q_OK : FP8Q_ERR_CUDA;
   // the array keeps the previous call's amax: clear the word before this call's reduction
   if (cudaMemsetAsync(amax, 0, kWordsNeeded * sizeof(uint32_t), s) != cudaSuccess) return FP8Q_ERR_CUDA;
   cudaError_t e = launch_tensor_amax(static_cast<const uint16_t*>(x), rows, cols, ld_x, amax, s);

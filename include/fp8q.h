@@ -52,7 +52,9 @@ typedef enum {
   FP8Q_ERR_ALIGN = 3,       /* a pointer or leading dimension is not 16-byte aligned  */
   FP8Q_ERR_UNSUPPORTED = 4, /* valid request this build does not implement            */
   FP8Q_ERR_CUDA = 5,        /* a CUDA runtime/driver call or kernel launch failed     */
-  FP8Q_ERR_TIMEOUT = 6      /* (device status) a bounded wait inside a kernel ran out */
+  FP8Q_ERR_TIMEOUT = 6,     /* (device status) a bounded wait inside a kernel ran out */
+  FP8Q_ERR_DEVICE_ARG = 7   /* (device status) an argument read on the device was out of
+                               range (grouped GEMM offsets); the kernel clamped it        */
 } fp8q_status;
 
 /* Byte layout of MX (E8M0) and NVFP4 (E4M3) scale factors. */
@@ -236,20 +238,26 @@ fp8q_status fp4q_quantize_2d16(const void* x, int64_t rows, int64_t cols, int64_
  *       C[m,n] = bf16( sum_kb sa[kb * ld_sa + m] * sb(kb, n) * partial_kb[m,n] ),
  *     sb by `layout`.  K % 128 == 0.  a_scale/b_scale are float*.
  *   MXFP8: codes E4M3, scales E8M0 in FP8Q_SF_MMA_TILED layout for (M, K/32) and
- *     (N, K/32), applied by the hardware.  K % 32 == 0.
+ *     (N, K/32), applied by the hardware.  K % 128 == 0.
  *   PERTENSOR: codes E4M3, or E5M2 per operand (a_format / b_format, e.g. an E5M2
  *     gradient times E4M3 weights in dgrad); C = (*a_global) * (*b_global) * (A . B^T).
- *     K % 16 == 0.
+ *     K % 128 == 0.
  *   NVFP4: packed E2M1 (lda/ldb in BYTES, K/2 bytes per row), E4M3 scales in
  *     FP8Q_SF_MMA_TILED layout for (M, K/16) and (N, K/16), C scaled by
- *     (*a_global) * (*b_global).  K % 32 == 0.
+ *     (*a_global) * (*b_global).  K % 256 == 0.
+ *   The K rules come from the kernels' pipeline: every stage moves 128 bytes of K per row
+ *   (128 FP8 or 256 FP4 values) and there is no partial last stage; a K that breaks the
+ *   rule returns FP8Q_ERR_SHAPE.  K == 0 is allowed (C = 0, or unchanged when
+ *   accumulating).
  * lda/ldb: row strides in bytes (% 16 == 0).  a/b 16-byte aligned.
  * Grouped (MoE, BLOCKWISE/FPROP only) when num_groups > 0: m_offsets[0..G] (device int32,
  *   non-decreasing, m_offsets[0] == 0, m_offsets[G] == M) delimit each expert's rows of A
  *   and C; B is [G][N][K] (expert g at b + g * N * ldb) and b_scale [G][N/128][K/128]
  *   (expert g at g * (N/128) * ld_sb floats).  The kernel reads the offsets on the device
  *   and builds its tile schedule there (at most M/128 + G row tiles), so the host needs
- *   no copy of them.
+ *   no copy of them.  Offsets that break the rule are clamped on the device to
+ *   [previous offset, M] (no row outside C is ever written) and the device status word
+ *   records FP8Q_ERR_DEVICE_ARG (read it with fp8q_get_device_status).
  * M, N >= 0 arbitrary (tails masked at the store).
  * c_fp32_accumulate (BLOCKWISE only; 0 for the other recipes): C is an FP32 row-major
  *   matrix (ldc % 4 == 0, c 16-byte aligned) that is updated in place,
@@ -307,7 +315,9 @@ fp8q_status fp8q_get_device_status(void* stream);
  * fp8q_get_device_status(). */
 fp8q_status fp8q_selftest_bounded_wait(uint64_t limit_ns, void* stream);
 
-/* Frees the current device's scratch pool (after a device sync).  Optional. */
+/* Frees the current device's scratch pool (after a device sync).  Optional.  Must not
+ * overlap any other fp8q call on that device (from another host thread): a call that
+ * already holds the pool's address would use freed memory. */
 fp8q_status fp8q_release_scratch(void);
 
 const char* fp8q_status_string(fp8q_status s);

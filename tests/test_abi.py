@@ -132,6 +132,34 @@ def test_gemm_validation_codes(L):
     assert fq.fp8q_gemm_blockscaled(_args(N=0), s) == 0
 
 
+@pytest.mark.parametrize("recipe,unit", [("FP8Q_BLOCKWISE", 128), ("FP8Q_MXFP8", 128), ("FP8Q_PERTENSOR", 128),
+                                         ("FP8Q_NVFP4", 256)])
+def test_gemm_k_rule_per_recipe(L, recipe, unit):
+    """The header's K rule for each recipe: the smallest accepted K passes validation (on a
+    machine without a GPU the call then fails at the first CUDA call, FP8Q_ERR_CUDA, never
+    FP8Q_ERR_SHAPE); K one block smaller than the unit, or not a multiple of it, is
+    FP8Q_ERR_SHAPE."""
+    r = getattr(fq, recipe)
+    fp4 = r == fq.FP8Q_NVFP4
+
+    def call(K):
+        kb = K // 2 if fp4 else K
+        ld = max(16, (kb + 15) // 16 * 16)
+        kw = dict(recipe=r, K=K, lda=ld, ldb=ld, ld_sb=max(1, K // 128))
+        if r in (fq.FP8Q_PERTENSOR, fq.FP8Q_NVFP4):
+            kw.update(a_global=0x10000, b_global=0x10000)
+        return fq.fp8q_gemm_blockscaled(_args(**kw), P(0))
+
+    import torch
+    accepted = fq.FP8Q_OK if torch.cuda.is_available() else fq.FP8Q_ERR_CUDA
+    if not torch.cuda.is_available():
+        assert call(unit) == accepted
+        assert call(3 * unit) == accepted
+    assert call(unit // 2) == fq.FP8Q_ERR_SHAPE
+    assert call(unit + unit // 4) == fq.FP8Q_ERR_SHAPE
+    assert call(unit + 16) == fq.FP8Q_ERR_SHAPE
+
+
 def test_product_path_has_no_cpu_fallback():
     """The binding must raise when the library is absent instead of computing on the host."""
     import importlib

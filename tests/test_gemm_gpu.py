@@ -302,6 +302,39 @@ def test_grouped_fprop_ragged_experts(cuda_lib):
         check(got[r0:r1], ref, t, f"grouped expert {g}")
 
 
+@pytest.mark.parametrize("offs,clamped", [([0, 130, 130, 500], [0, 130, 130, 300]),
+                                          ([0, 200, 100, 300], [0, 200, 200, 300])])
+def test_grouped_offsets_out_of_rule_are_clamped_on_the_device(cuda_lib, offs, clamped):
+    """Expert offsets past M or decreasing: the kernel clamps each to [previous, M], writes
+    no row outside C (guard rows below C keep their sentinel), computes the clamped
+    experts, and records FP8Q_ERR_DEVICE_ARG in the device status word."""
+    fq = cuda_lib
+    M, K, N, Gn = 300, 384, 256, 3
+    A = bf((M, K), 1.0, 61)
+    Ws = [bf((K, N), 0.006, 70 + g) for g in range(Gn)]
+    qa = fq.quantize_1x128(A.cuda())
+    qws = [fq.quantize_128x128(w.cuda()) for w in Ws]
+    B = torch.stack([q["q_t"] for q in qws])
+    SB = torch.stack([q["s"] for q in qws])
+    assert fq.device_status() == fq.FP8Q_OK
+    big = torch.full((M + 256, N), 7.0, dtype=torch.bfloat16, device="cuda")
+    fq.gemm(qa["q_row"], B, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qa["s_row"], b_scale=SB,
+            ld_sb=K // 128, m_offsets=torch.tensor(offs, dtype=torch.int32, device="cuda"), out=big[:M])
+    assert fq.device_status() == fq.FP8Q_ERR_DEVICE_ARG
+    assert fq.device_status() == fq.FP8Q_OK                     # reading the status cleared it
+    assert bool((big[M:] == 7.0).all())
+    oa, osa = Q.quantize_1x128_rowwise(workloads.bf16_bits(A))
+    got = host(big[:M].float()).astype(np.float64)
+    for g in range(Gn):
+        r0, r1 = clamped[g], clamped[g + 1]
+        if r1 == r0:
+            continue
+        _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(Ws[g]))
+        rows = np.arange(r0, r1)
+        ref, t = G.reference(G.dequant_a_1x128(oa, osa, rows=rows), G.dequant_b_blockwise(owt, osw, G.FPROP))
+        check(got[r0:r1], ref, t, f"clamped expert {g}")
+
+
 # ----------------------------------------------------------------------------- other recipes
 @pytest.mark.parametrize("M,K,N", [(300, 512, 400), (256, 1024, 256)])
 def test_mxfp8(cuda_lib, M, K, N):

@@ -124,6 +124,24 @@ def test_per_tensor_parity(cuda_lib, R, C):
     assert f32bits(host(out["s_dec"]))[0] == f32bits(np.float32([s]))[0]
 
 
+def test_per_tensor_empty_writes_unit_scale_on_the_stream(cuda_lib):
+    """An empty tensor: amax 0 -> scale 1 -> decode scale 1.0, written by a kernel on the
+    caller's stream (no host synchronization), for both per-tensor entry points."""
+    import ctypes
+    fq = cuda_lib
+    L = fq.lib()
+    x = torch.empty((0, 64), dtype=torch.bfloat16, device="cuda")
+    q = torch.empty((16,), dtype=torch.uint8, device="cuda")
+    for fn in (L.fp8q_quantize_tensor, L.fp8q_quantize_tensor_noalloc):
+        s = torch.full((1,), -3.0, dtype=torch.float32, device="cuda")
+        side = torch.cuda.Stream()
+        with torch.cuda.stream(side):
+            assert fn(ctypes.c_void_p(x.data_ptr()), 0, 64, 64, ctypes.c_void_p(q.data_ptr()),
+                      ctypes.c_void_p(s.data_ptr()), ctypes.c_void_p(side.cuda_stream)) == 0
+        side.synchronize()
+        assert float(s.item()) == 1.0
+
+
 # ----------------------------------------------------------------------------- NVFP4
 NV_CASES = [
     # R, C, row, col, rht, sr
