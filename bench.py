@@ -1160,11 +1160,11 @@ def main():
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
-                    help="llama8b only: token count M (default 8192); smaller cases for profiler captures")
+                    help="llama8b / nvfp4: token count M (default 8192); smaller cases for profiler captures")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
-    if args.tokens and args.workload != "llama8b":
-        ap.error("--tokens applies to the llama8b workload only")
+    if args.tokens and args.workload not in ("llama8b", "nvfp4", "nvfp4_train"):
+        ap.error("--tokens applies to the llama8b and nvfp4 workloads only")
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:

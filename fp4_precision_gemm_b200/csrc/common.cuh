@@ -94,19 +94,21 @@ __device__ __forceinline__ float pow2_neg(int e) {
 // Magnitude grid {0, 0.5, 1, 1.5, 2, 3, 4, 6}; code index = grid index, bit 3 = sign.
 // Stochastic rounding with one 32-bit random word: up iff (word >> 8) * 2^-24 < p,
 // p = (|y| - lo) / (hi - lo).  The gaps of the E2M1 grid are powers of two, so p is a
-// fixed-point fraction of |y|'s own mantissa bits and the decision is an exact integer
-// compare against the 24-bit random value u24 = word >> 8:
-//   |y| in [1, 6):   lo has |y|'s exponent and top mantissa bit, p = (low 22 bits) / 2^22,
-//                    floor code = 2 + 2*(exponent) + top bit = (bits >> 22) - 252;
-//   |y| in [0.5, 1): lo = 0.5, gap 0.5, p = (23 mantissa bits) / 2^23, floor code 1;
-//   |y| < 0.5:       lo = 0, gap 0.5, p = 2|y| (compared in FP32, exact), floor code 0;
-//   |y| >= 6:        code 7 (saturation, no rounding).
+// fixed-point fraction of |y|'s own mantissa bits and the decision is exact in integers:
+//   |y| in [1, 6):   lo keeps |y|'s exponent and top mantissa bit, p = (low 22 bits) / 2^22,
+//                    and "up" is the carry out of those 22 bits when 2^22 - 1 - (u24 >> 2)
+//                    is added to them; the code is then (bits >> 22) - 252, capped at 7
+//                    (|y| >= 6 saturates, no rounding);
+//   |y| in [0.5, 1): lo = 0.5, gap 0.5, p = (23 mantissa bits) / 2^23: the carry out of the
+//                    23 bits when 2^23 - 1 - (u24 >> 1) is added, code (bits >> 23) - 125;
+//   |y| < 0.5:       lo = 0, gap 0.5, p = 2|y|: up iff u24 * 2^-25 < |y| (exact in FP32).
+// (u < p with u = u24 / 2^24 and p = L / 2^22 is u24 < 4L, i.e. (u24 >> 2) < L.)
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t word) {
-  const uint32_t b = __float_as_uint(y), ab = b & 0x7FFFFFFFu, u24 = word >> 8;
-  const uint32_t c_hi = (ab >> 22) - 252u + (u24 < ((ab & 0x3FFFFFu) << 2) ? 1u : 0u);
-  const uint32_t c_mid = 1u + (u24 < ((ab & 0x7FFFFFu) << 1) ? 1u : 0u);
-  const uint32_t c_lo = (__fmul_rn((float)u24, 5.9604644775390625e-08f) < __fmul_rn(__uint_as_float(ab), 2.0f)) ? 1u : 0u;
-  const uint32_t code = ab >= 0x40C00000u ? 7u : ab >= 0x3F800000u ? c_hi : ab >= 0x3F000000u ? c_mid : c_lo;
+  const uint32_t b = __float_as_uint(y), ab = b & 0x7FFFFFFFu;
+  const uint32_t c_hi = min((ab + (0x3FFFFFu - (word >> 10)) - (252u << 22)) >> 22, 7u);
+  const uint32_t c_mid = (ab + (0x7FFFFFu - (word >> 9)) - (125u << 23)) >> 23;
+  const uint32_t c_lo = __fmul_rn((float)(word >> 8), 2.98023223876953125e-08f) < __uint_as_float(ab) ? 1u : 0u;
+  const uint32_t code = ab >= 0x3F800000u ? c_hi : ab >= 0x3F000000u ? c_mid : c_lo;
   return code | ((b >> 28) & 8u);
 }
 

@@ -391,6 +391,8 @@ namespace {
 
 constexpr int kBwPairM = 2 * kBM;               // 256 output rows per pair tile
 constexpr int kBwSb = 10;                       // scale ring: chunks of A/B scales staged ahead
+constexpr int kBwGo = 10;                       // MMA go barriers: a multiple of both the stage count
+                                                // and the two TMEM partial buffers
 
 // Pair tile shape: 256 x 256 outputs, 16 promotion warps.
 struct BwCfg {
@@ -423,7 +425,8 @@ struct BwSmem {
   static constexpr uint32_t stage_c = 32 * epi_cols * 2;
   static constexpr uint32_t cst = ring + kBwSb * slot_bytes;
   static constexpr uint32_t bars = cst + C::EpiWarps * stage_c;
-  static constexpr uint32_t n_bars = 2 * stages + 2 + 2 * kBwSb + 1 + C::EpiWarps / 2;
+  static constexpr uint32_t n_bars = kBwGo + stages + 2 * kBwSb + 1 + C::EpiWarps / 2;
+  static_assert(kBwGo % stages == 0 && kBwGo % 2 == 0, "go slots must cycle with the stages and TMEM buffers");
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t groups = misc + 16;
   // fused output quantization: each promotion warp's 32 row amaxes, read by its partner warp
@@ -501,10 +504,12 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
   constexpr int kStages = S::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint64_t* full = reinterpret_cast<uint64_t*>(smem + S::bars);   // leader: both halves landed
-  uint64_t* empty = full + kStages;    // both CTAs: the stage's MMAs are done (partial ready)
-  uint64_t* pempty = empty + kStages;  // leader: [2] TMEM buffer b drained by both CTAs
-  uint64_t* sfull = pempty + 2;          // local scale ring: slot filled
+  // go[c % kBwGo] (leader): chunk c may be issued - both CTAs' A/B halves for c have landed
+  // and both CTAs' promotion warps have drained chunk c - 2 from its TMEM buffer.  One barrier
+  // per chunk keeps the MMA issuer to a single wait per chunk.
+  uint64_t* go = reinterpret_cast<uint64_t*>(smem + S::bars);
+  uint64_t* empty = go + kBwGo;        // both CTAs: the stage's MMAs are done (partial ready)
+  uint64_t* sfull = empty + kStages;     // local scale ring: slot filled
   uint64_t* sempty = sfull + kBwSb;      // local scale ring: slot read by every promotion warp
   uint64_t* final_bar = sempty + kBwSb;
   uint64_t* xbar = final_bar + 1;        // [EpiWarps/2] fused quantization: partner warps' amaxes
@@ -519,11 +524,9 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
   const int KB = p.K / kBKB;
 
   if (threadIdx.x == 0) {
-    for (int i = 0; i < kStages; ++i) {
-      mbar_init(&full[i], 1);
-      mbar_init(&empty[i], 1);
-    }
-    for (int i = 0; i < 2; ++i) mbar_init(&pempty[i], 2 * kBwEpiWarps);  // per promotion warp, both CTAs
+    // go: the leader producer's expect-tx arrival + one per promotion warp of both CTAs
+    for (int i = 0; i < kBwGo; ++i) mbar_init(&go[i], 1 + 2 * kBwEpiWarps);
+    for (int i = 0; i < kStages; ++i) mbar_init(&empty[i], 1);
     for (int i = 0; i < kBwSb; ++i) {
       mbar_init(&sfull[i], 33);  // lane 0's expect-tx arrival + 32 cp.async arrivals
       mbar_init(&sempty[i], kBwEpiWarps);
@@ -532,6 +535,9 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
     for (int i = 0; i < kBwEpiWarps / 2; ++i) mbar_init(&xbar[i], 2);
     *abort_flag = 0;
     fence_barrier_init();
+    // chunks 0 and 1 have no earlier chunk to drain from their TMEM buffers
+    mbar_arrive_count(&go[0], 2 * kBwEpiWarps);
+    mbar_arrive_count(&go[1], 2 * kBwEpiWarps);
   }
   if (GROUPED && warp == kBwProducerWarp) load_pair_groups(p, prefix, offs, lane);
   if (warp == kBwMmaWarp) {
@@ -566,17 +572,18 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
             ok = false;
             break;
           }
-          if (leader) mbar_arrive_expect_tx(&full[s], 2 * (kAStage + kBwBStage));
-          const uint32_t bar = mapa_shared(smem_u32(&full[s]), 0);
+          const uint32_t g = it % kBwGo;
+          if (leader) mbar_arrive_expect_tx(&go[g], 2 * (kAStage + kBwBStage));
+          const uint32_t bar = mapa_shared(smem_u32(&go[g]), 0);
           tma_load_2d_pair(smem + S::a + s * kAStage, &tma_a, bar, kb * kBKB, T.m0);
           tma_load_2d_pair(smem + S::b + s * kBwBStage, &tma_b, bar, kb * kBKB, b_row);
         }
       }
-      if (leader) {  // the leader's barriers see both halves: wait for the copies in flight
+      if (leader) {  // the leader's go barriers see both halves: wait for the copies in flight
         const uint32_t inflight = it < (uint32_t)kStages ? it : (uint32_t)kStages;
         for (uint32_t j = 0; j < inflight; ++j) {
           const uint32_t i2 = it - 1 - j;
-          mbar_wait_drain(&full[i2 % kStages], (i2 / kStages) & 1, kWaitLimitNs);
+          mbar_wait_drain(&go[i2 % kBwGo], (i2 / kBwGo) & 1, kWaitLimitNs);
         }
       }
     }
@@ -636,9 +643,8 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
         for (int kb = 0; kb < KB; ++kb, ++it) {
-          const uint32_t s = it % kStages, ph = (it / kStages) & 1, pb = it & 1;
-          if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimitNs) ||
-              !mbar_wait(&pempty[pb], ((it >> 1) & 1) ^ 1, abort_flag, kWaitLimitNs)) {
+          const uint32_t s = it % kStages, pb = it & 1;
+          if (!mbar_wait(&go[it % kBwGo], (it / kBwGo) & 1, abort_flag, kWaitLimitNs)) {
             raise_timeout(p, abort_flag);
             ok = false;
             break;
@@ -661,8 +667,7 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
     const int q = warp & 3, cgp = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cgp * 64);
     const int rloc = q * 32 + lane;
-    const uint32_t pempty_leader0 = mapa_shared(smem_u32(&pempty[0]), 0);
-    const uint32_t pempty_leader1 = mapa_shared(smem_u32(&pempty[1]), 0);
+    const uint32_t go_leader = mapa_shared(smem_u32(&go[0]), 0);   // the leader's go[0]
     uint32_t chunk = 0, tile_it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters, ++tile_it) {
@@ -714,7 +719,8 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) {
-          mbar_arrive_cluster_relaxed(pb ? pempty_leader1 : pempty_leader0);
+          // chunk + 2 reuses this TMEM buffer: release it on that chunk's go barrier
+          mbar_arrive_cluster_relaxed(go_leader + 8u * ((chunk + 2) % kBwGo));
           mbar_arrive_relaxed(&sempty[rs]);
         }
         ++chunk;

@@ -21,7 +21,7 @@
 //     two upper butterfly stages when the rowwise transform is on);
 //   * one Philox call yields the 4 words of 4 consecutive output elements.
 // The transposed colwise codes are staged in shared memory and stored as 64-byte rows.
-// With both outputs requested the rowwise and colwise quantization run as separate kernels.
+// With both outputs requested one kernel makes both from a single read of each tile.
 #include "common.cuh"
 #include "kernels.h"
 
@@ -208,8 +208,82 @@ __global__ void __launch_bounds__(256, 3) fp4_amax_kernel(const __grid_constant_
   if (COL) block_max_atomic(m_col, P.amax_bits + 1);
 }
 
-// Colwise output (16-element groups along rows): the 16x4-per-thread tile mapping keeps each
-// group, its transform and its block amax in-thread.
+// Colwise output of one 128x128 tile (16-element groups along rows), from the thread's 16x4
+// sub-block: each column's group, its transform and its block amax are in-thread.  The
+// transposed codes are staged in `tq` (128 x 64 bytes, 8-byte chunks XOR-swizzled) and
+// stored as 64-byte rows; the caller synchronizes the CTA between the two halves.
+template <bool SR>
+__device__ __forceinline__ void col_codes_to_stage(const Fp4QuantParams& P, const Tile& T, const float (&x)[16][4],
+                                                   uint32_t signs, const float* enc_tab, float S_g, uint8_t* tq) {
+  const int64_t nsf = P.rows >> 4, s4 = (nsf + 3) >> 2;
+  const int64_t kr = (T.r0 >> 4) + T.w;
+#pragma unroll
+  for (int j = 0; j < 4; ++j) {
+    const int64_t cg = T.col + j;
+    float e[16];
+#pragma unroll
+    for (int i = 0; i < 16; ++i) e[i] = P.rht_col ? flip(x[i][j], signs, i) : x[i][j];
+    if (P.rht_col) fwht16(e);
+    float m = 0.0f;
+#pragma unroll
+    for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+    uint32_t sb;
+    float enc;
+    block_scale(m, S_g, enc_tab, sb, enc);
+    uint32_t lo = 0, hi = 0;
+#pragma unroll
+    for (int q = 0; q < 4; ++q) {
+      uint32_t c4;
+      if (SR) {
+        const uint64_t blk = (uint64_t)(cg * P.rows + T.r0 + T.w * 16 + 4 * q) >> 2;
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 1u), P.sr_k0, P.sr_k1);
+        c4 = e2m1_sr(__fmul_rn(e[4 * q], enc), r.x) | (e2m1_sr(__fmul_rn(e[4 * q + 1], enc), r.y) << 4) |
+             (e2m1_sr(__fmul_rn(e[4 * q + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[4 * q + 3], enc), r.w) << 12);
+      } else {
+        c4 = e2m1x2_rne(__fmul_rn(e[4 * q + 1], enc), __fmul_rn(e[4 * q], enc)) |
+             (e2m1x2_rne(__fmul_rn(e[4 * q + 3], enc), __fmul_rn(e[4 * q + 2], enc)) << 8);
+      }
+      if (q < 2) lo |= c4 << (16 * q);
+      else hi |= c4 << (16 * (q - 2));
+    }
+    const int c = T.lane * 4 + j;
+    *(uint2*)&tq[c * 64 + ((T.w ^ ((c >> 2) & 7)) * 8)] = make_uint2(lo, hi);
+    if (P.sf_tiled) {
+      if (kr < s4 * 4) P.sf_col[sf_tiled_offset(cg, kr, s4)] = (uint8_t)sb;
+    } else if (cg < P.cols && kr < nsf) {
+      P.sf_col[cg * nsf + kr] = (uint8_t)sb;
+    }
+  }
+}
+
+// Stores the staged transposed codes of one tile (after a CTA barrier): 64-byte rows,
+// 16-byte stores when the transposed row stride (rows / 2 bytes) allows.
+__device__ __forceinline__ void col_stage_store(const Fp4QuantParams& P, const Tile& T, const uint8_t* tq) {
+#pragma unroll
+  for (int pass = 0; pass < 2; ++pass) {
+    const int c = pass * 64 + (threadIdx.x >> 2), h = threadIdx.x & 3;
+    const int64_t cg = T.c0 + c, rg = T.r0 + 32 * h;
+    const uint2 a = *(const uint2*)&tq[c * 64 + (((2 * h) ^ ((c >> 2) & 7)) * 8)];
+    const uint2 b = *(const uint2*)&tq[c * 64 + (((2 * h + 1) ^ ((c >> 2) & 7)) * 8)];
+    uint8_t* dst = P.q_col + cg * (P.rows >> 1) + (rg >> 1);
+    // the transposed row stride is rows/2 bytes: 16-byte aligned only when rows % 32 == 0
+    if (cg < P.cols) {
+      if (rg + 32 <= P.rows) {
+        if (((P.rows >> 1) & 15) == 0) {
+          *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
+        } else {
+          *(uint2*)dst = a;
+          *(uint2*)(dst + 8) = b;
+        }
+      } else if (rg + 16 <= P.rows) {
+        *(uint2*)dst = a;
+      }
+    }
+  }
+}
+
+// Colwise output alone.
+template <bool SR>
 __global__ void __launch_bounds__(256, 3) fp4_quant_col_kernel(const __grid_constant__ Fp4QuantParams P) {
   __shared__ __align__(16) uint8_t tq[128 * 64];
   __shared__ float enc_tab[128];
@@ -217,76 +291,75 @@ __global__ void __launch_bounds__(256, 3) fp4_quant_col_kernel(const __grid_cons
   float x[16][4];
   load16x4(P, T, x);
   const uint32_t signs = P.rht_col ? rht_signs(P) : 0u;
-  if (threadIdx.x < 128) fill_enc_tab(enc_tab, global_scale(P.amax_bits[1]));
+  const float S_g = global_scale(P.amax_bits[1]);
+  if (threadIdx.x < 128) fill_enc_tab(enc_tab, S_g);
+  if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_col = __frcp_rn(S_g);
+  __syncthreads();
+  col_codes_to_stage<SR>(P, T, x, signs, enc_tab, S_g, tq);
+  __syncthreads();
+  col_stage_store(P, T, tq);
+}
+
+// Both outputs from one read of the tile.  The colwise half is the kernel above; the
+// rowwise 16-element groups are the 16x4 sub-blocks of 4 consecutive lanes: the group amax
+// (and, with the rowwise transform, its two upper butterfly stages) takes two xor-shuffles,
+// and each lane's 4 values of a row are 4 consecutive output elements, i.e. one Philox call.
+// A warp stores 64 contiguous bytes of each of its 16 rows.  With the MMA-tiled scale layout
+// the tiles also cover the image's padding rows and scale columns (their data reads as zero,
+// so their scale code is 0).
+template <bool SR_ROW, bool SR_COL>
+__global__ void __launch_bounds__(256, 2) fp4_quant_rowcol_kernel(const __grid_constant__ Fp4QuantParams P) {
+  __shared__ __align__(16) uint8_t tq[128 * 64];
+  __shared__ float enc_tab[2][128];
+  const Tile T = tile_coords(P, blockIdx.x);
+  float x[16][4];
+  load16x4(P, T, x);
+  const uint32_t signs = (P.rht_row || P.rht_col) ? rht_signs(P) : 0u;
+  const float S_row = global_scale(P.amax_bits[0]), S_col = global_scale(P.amax_bits[1]);
+  fill_enc_tab(enc_tab[threadIdx.x >> 7], threadIdx.x < 128 ? S_row : S_col);
+  if (blockIdx.x == 0 && threadIdx.x == 0) {
+    *P.g_row = __frcp_rn(S_row);
+    *P.g_col = __frcp_rn(S_col);
+  }
   __syncthreads();
 
+  // rowwise output
   {
-    const float S_g = global_scale(P.amax_bits[1]);
-    if (blockIdx.x == 0 && threadIdx.x == 0) *P.g_col = __frcp_rn(S_g);
-    const int64_t nsf = P.rows >> 4, s4 = (nsf + 3) >> 2;
-    const int64_t kr = (T.r0 >> 4) + T.w;
+    const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
+    const int64_t kc = (T.c0 >> 4) + (T.lane >> 2);
+    const bool sf_writer = (T.lane & 3) == 0 && (P.sf_tiled ? kc < s4 * 4 : kc < nsf);
 #pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int64_t cg = T.col + j;
-      float e[16];
-#pragma unroll
-      for (int i = 0; i < 16; ++i) e[i] = P.rht_col ? flip(x[i][j], signs, i) : x[i][j];
-      if (P.rht_col) fwht16(e);
-      float m = 0.0f;
-#pragma unroll
-      for (int i = 0; i < 16; ++i) m = fmaxf(m, fabsf(e[i]));
+    for (int i = 0; i < 16; ++i) {
+      const int64_t row = T.r0 + T.w * 16 + i;
+      float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
+      if (P.rht_row) rht_row4(e, signs, T.lane);
+      float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
+      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
       uint32_t sb;
       float enc;
-      block_scale(m, S_g, enc_tab, sb, enc);
-      uint32_t lo = 0, hi = 0;
-#pragma unroll
-      for (int q = 0; q < 4; ++q) {
-        uint32_t c4;
-        if (P.sr_col) {
-          const uint64_t blk = (uint64_t)(cg * P.rows + T.r0 + T.w * 16 + 4 * q) >> 2;
-          const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 1u),
-                                        P.sr_k0, P.sr_k1);
-          c4 = e2m1_sr(__fmul_rn(e[4 * q], enc), r.x) | (e2m1_sr(__fmul_rn(e[4 * q + 1], enc), r.y) << 4) |
-               (e2m1_sr(__fmul_rn(e[4 * q + 2], enc), r.z) << 8) |
-               (e2m1_sr(__fmul_rn(e[4 * q + 3], enc), r.w) << 12);
-        } else {
-          c4 = e2m1x2_rne(__fmul_rn(e[4 * q + 1], enc), __fmul_rn(e[4 * q], enc)) |
-               (e2m1x2_rne(__fmul_rn(e[4 * q + 3], enc), __fmul_rn(e[4 * q + 2], enc)) << 8);
-        }
-        if (q < 2) lo |= c4 << (16 * q);
-        else hi |= c4 << (16 * (q - 2));
+      block_scale(m, S_row, enc_tab[0], sb, enc);
+      uint32_t c4;
+      if (SR_ROW) {
+        const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
+        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
+        c4 = e2m1_sr(__fmul_rn(e[0], enc), r.x) | (e2m1_sr(__fmul_rn(e[1], enc), r.y) << 4) |
+             (e2m1_sr(__fmul_rn(e[2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[3], enc), r.w) << 12);
+      } else {
+        c4 = e2m1x2_rne(__fmul_rn(e[1], enc), __fmul_rn(e[0], enc)) |
+             (e2m1x2_rne(__fmul_rn(e[3], enc), __fmul_rn(e[2], enc)) << 8);
       }
-      const int c = T.lane * 4 + j;
-      *(uint2*)&tq[c * 64 + ((T.w ^ ((c >> 2) & 7)) * 8)] = make_uint2(lo, hi);
-      if (P.sf_tiled) {
-        if (kr < s4 * 4) P.sf_col[sf_tiled_offset(cg, kr, s4)] = (uint8_t)sb;
-      } else if (cg < P.cols && kr < nsf) {
-        P.sf_col[cg * nsf + kr] = (uint8_t)sb;
-      }
-    }
-    __syncthreads();
-#pragma unroll
-    for (int pass = 0; pass < 2; ++pass) {
-      const int c = pass * 64 + (threadIdx.x >> 2), h = threadIdx.x & 3;
-      const int64_t cg = T.c0 + c, rg = T.r0 + 32 * h;
-      const uint2 a = *(const uint2*)&tq[c * 64 + (((2 * h) ^ ((c >> 2) & 7)) * 8)];
-      const uint2 b = *(const uint2*)&tq[c * 64 + (((2 * h + 1) ^ ((c >> 2) & 7)) * 8)];
-      uint8_t* dst = P.q_col + cg * (P.rows >> 1) + (rg >> 1);
-      // the transposed row stride is rows/2 bytes: 16-byte aligned only when rows % 32 == 0
-      if (cg < P.cols) {
-        if (rg + 32 <= P.rows) {
-          if (((P.rows >> 1) & 15) == 0) {
-            *(uint4*)dst = make_uint4(a.x, a.y, b.x, b.y);
-          } else {
-            *(uint2*)dst = a;
-            *(uint2*)(dst + 8) = b;
-          }
-        } else if (rg + 16 <= P.rows) {
-          *(uint2*)dst = a;
-        }
+      if (T.cok && row < P.rows) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)c4;
+      if (sf_writer) {
+        if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+        else if (row < P.rows) P.sf_row[row * nsf + kc] = (uint8_t)sb;
       }
     }
   }
+
+  col_codes_to_stage<SR_COL>(P, T, x, signs, enc_tab[1], S_col, tq);
+  __syncthreads();
+  col_stage_store(P, T, tq);
 }
 
 // ------------------------------------------------------------------ 16x16 weight blocks
@@ -512,15 +585,23 @@ cudaError_t launch_fp4_quant_2d(const Fp4QuantParams& p, int64_t tiles, cudaStre
 
 cudaError_t launch_fp4_quant(const Fp4QuantParams& p, int64_t tiles, cudaStream_t s) {
   const bool row = p.q_row != nullptr, col = p.q_col != nullptr;
-  // Both outputs: the rowwise pass and the colwise pass run as separate kernels (one extra
-  // read of the input); each is ALU-bound with stochastic rounding, and apart they keep far
-  // more threads resident than the combined 16x4 kernel.
+  const unsigned grid = (unsigned)tiles;
+  if (row && col) {   // both outputs from one read of each tile
+    if (p.sr_row && p.sr_col) fp4_quant_rowcol_kernel<true, true><<<grid, 256, 0, s>>>(p);
+    else if (p.sr_row) fp4_quant_rowcol_kernel<true, false><<<grid, 256, 0, s>>>(p);
+    else if (p.sr_col) fp4_quant_rowcol_kernel<false, true><<<grid, 256, 0, s>>>(p);
+    else fp4_quant_rowcol_kernel<false, false><<<grid, 256, 0, s>>>(p);
+    return cudaGetLastError();
+  }
   if (row) {
     const int64_t nsf = p.cols >> 4, kdom = p.sf_tiled ? (nsf + 3) / 4 * 4 : nsf;
     const int64_t rdom = p.sf_tiled ? (p.rows + 127) / 128 * 128 : p.rows;
     fp4_quant_row_kernel<<<blocks_for(rdom * kdom), 256, 0, s>>>(p);
   }
-  if (col) fp4_quant_col_kernel<<<(unsigned)tiles, 256, 0, s>>>(p);
+  if (col) {
+    if (p.sr_col) fp4_quant_col_kernel<true><<<grid, 256, 0, s>>>(p);
+    else fp4_quant_col_kernel<false><<<grid, 256, 0, s>>>(p);
+  }
   return cudaGetLastError();
 }
 

@@ -39,6 +39,10 @@ __device__ __forceinline__ void cp_async_4(void* dst, const void* src, uint32_t 
   asm volatile("cp.async.ca.shared.global [%0], [%1], 4, %2;" ::"r"(smem_u32(dst)), "l"(src), "r"(src_bytes)
                : "memory");
 }
+// `count` arrivals at once (e.g. arrivals that an earlier pipeline stage will never make).
+__device__ __forceinline__ void mbar_arrive_count(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
 // Arrives on the barrier once every cp.async this thread issued before it has landed; the
 // barrier's expected count includes this arrival.
 __device__ __forceinline__ void cp_async_arrive_noinc(uint64_t* bar) {
