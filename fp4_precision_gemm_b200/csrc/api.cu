@@ -316,6 +316,10 @@ fp8q_status fp4q_rht16_quantize_sr(const void* x, int64_t rows, int64_t cols, in
   p.rht_k1 = (uint32_t)(rht_seed >> 32);
   p.sr_k0 = (uint32_t)sr_seed;
   p.sr_k1 = (uint32_t)(sr_seed >> 32);
+  for (int r = 0; r < 10; ++r) {   // Philox4x32-10 key schedule (Weyl sequence of the key)
+    p.sr_rk[2 * r] = p.sr_k0 + (uint32_t)r * 0x9E3779B9u;
+    p.sr_rk[2 * r + 1] = p.sr_k1 + (uint32_t)r * 0xBB67AE85u;
+  }
   p.q_row = row ? q_row : nullptr;
   p.sf_row = sf_row;
   p.g_row = g_dec_row;
@@ -355,6 +359,7 @@ fp8q_status fp4q_quantize_2d16(const void* x, int64_t rows, int64_t cols, int64_
   p.ld_x = ld_x;
   p.rht_row = p.rht_col = p.sr_row = p.sr_col = 0;
   p.rht_k0 = p.rht_k1 = p.sr_k0 = p.sr_k1 = 0;
+  for (int r = 0; r < 20; ++r) p.sr_rk[r] = 0;
   p.q_row = row ? q_row : nullptr;
   p.sf_row = sf_row;
   p.g_row = g_dec;

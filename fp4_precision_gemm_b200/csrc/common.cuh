@@ -99,17 +99,15 @@ __device__ __forceinline__ float pow2_neg(int e) {
 //                    and "up" is the carry out of those 22 bits when 2^22 - 1 - (u24 >> 2)
 //                    is added to them; the code is then (bits >> 22) - 252, capped at 7
 //                    (|y| >= 6 saturates, no rounding);
-//   |y| in [0.5, 1): lo = 0.5, gap 0.5, p = (23 mantissa bits) / 2^23: the carry out of the
-//                    23 bits when 2^23 - 1 - (u24 >> 1) is added, code (bits >> 23) - 125;
-//   |y| < 0.5:       lo = 0, gap 0.5, p = 2|y|: up iff u24 * 2^-25 < |y| (exact in FP32).
+//   |y| < 1:         the grid step is 0.5 throughout, so with F = |y| * 2^25 (exact) the
+//                    floor code is F >> 24 and "up" is u24 < F mod 2^24; both are the carry
+//                    of ceil(F) + (2^24 - 1 - u24) into bit 24 (u24 < F <=> u24 < ceil(F)).
 // (u < p with u = u24 / 2^24 and p = L / 2^22 is u24 < 4L, i.e. (u24 >> 2) < L.)
 __device__ __forceinline__ uint32_t e2m1_sr(float y, uint32_t word) {
   const uint32_t b = __float_as_uint(y), ab = b & 0x7FFFFFFFu;
   const uint32_t c_hi = min((ab + (0x3FFFFFu - (word >> 10)) - (252u << 22)) >> 22, 7u);
-  const uint32_t c_mid = (ab + (0x7FFFFFu - (word >> 9)) - (125u << 23)) >> 23;
-  const uint32_t c_lo = __fmul_rn((float)(word >> 8), 2.98023223876953125e-08f) < __uint_as_float(ab) ? 1u : 0u;
-  const uint32_t code = ab >= 0x3F800000u ? c_hi : ab >= 0x3F000000u ? c_mid : c_lo;
-  return code | ((b >> 28) & 8u);
+  const uint32_t c_lo = (__float2uint_ru(__fmul_rn(__uint_as_float(ab), 33554432.0f)) + (0xFFFFFFu - (word >> 8))) >> 24;
+  return (ab >= 0x3F800000u ? c_hi : c_lo) | ((b >> 28) & 8u);
 }
 
 // Two values to E2M1 by round-to-nearest-even with saturation at 6 (hardware conversion):
@@ -134,6 +132,20 @@ __device__ __forceinline__ uint4 philox4x32_10(uint4 c, uint32_t k0, uint32_t k1
     const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
     const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
     c = make_uint4(hi1 ^ c.y ^ k0, lo1, hi0 ^ c.w ^ k1, lo0);
+  }
+  return c;
+}
+
+// The same generator with the key schedule precomputed: rk[2r], rk[2r + 1] are the key words
+// of round r (k0 + r * 0x9E3779B9, k1 + r * 0xBB67AE85), e.g. kernel parameters, so a round is
+// two wide multiplies and two three-way xors.
+__device__ __forceinline__ uint4 philox4x32_10_rk(uint4 c, const uint32_t (&rk)[20]) {
+#pragma unroll
+  for (int r = 0; r < 10; ++r) {
+    const uint64_t p0 = (uint64_t)c.x * 0xD2511F53u, p1 = (uint64_t)c.z * 0xCD9E8D57u;
+    const uint32_t hi0 = (uint32_t)(p0 >> 32), lo0 = (uint32_t)p0;
+    const uint32_t hi1 = (uint32_t)(p1 >> 32), lo1 = (uint32_t)p1;
+    c = make_uint4(hi1 ^ c.y ^ rk[2 * r], lo1, hi0 ^ c.w ^ rk[2 * r + 1], lo0);
   }
   return c;
 }

@@ -49,6 +49,7 @@ struct Fp4QuantParams {
   int sf_tiled;
   int tiles_c;
   uint32_t* amax_bits;  // [0]: rowwise output's global amax, [1]: colwise output's
+  uint32_t sr_rk[20];   // Philox key schedule of the stochastic-rounding key (sr_k0, sr_k1)
 };
 
 // One float written on the stream (the decode scale of an empty tensor), no host sync.

@@ -95,10 +95,23 @@ __device__ __forceinline__ float global_scale(uint32_t amax_bits) {
   return (s > FLT_MAX) ? FLT_MAX : s;
 }
 
+// fp32(m / 6), correctly rounded.  For m in [2^-125, FLT_MAX] one FMA correction of
+// m * fp32(1/6) gives the correctly rounded quotient (checked on the CPU for every FP32
+// significand over the binades where an intermediate can be subnormal, and on whole binades
+// above, where all steps scale exactly); zero, tiny and non-finite m take the IEEE division.
+__device__ __forceinline__ float div6_rn(float m) {
+  constexpr float kSixth = 0.16666667163372039794921875f;   // fp32(1/6) = 0x3E2AAAAB
+  if (m >= 0x1p-125f && m <= FLT_MAX) {
+    const float q0 = __fmul_rn(m, kSixth);
+    return __fmaf_rn(__fmaf_rn(-6.0f, q0, m), kSixth, q0);
+  }
+  return __fdiv_rn(m, 6.0f);
+}
+
 // E4M3 block scale and the matching encode scale S_g / decode(sb) for block amax `m`; the
 // encode scales of all 128 non-negative codes are tabulated once per CTA (enc_tab).
 __device__ __forceinline__ void block_scale(float m, float S_g, const float* enc_tab, uint32_t& sb, float& enc) {
-  const float t = __fmul_rn(__fdiv_rn(m, 6.0f), S_g);
+  const float t = __fmul_rn(div6_rn(m), S_g);
   sb = cvt_e4m3x2(t, 0.0f) & 0xFFu;
   enc = enc_tab[sb & 0x7Fu];
 }
@@ -236,7 +249,7 @@ __device__ __forceinline__ void col_codes_to_stage(const Fp4QuantParams& P, cons
       uint32_t c4;
       if (SR) {
         const uint64_t blk = (uint64_t)(cg * P.rows + T.r0 + T.w * 16 + 4 * q) >> 2;
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 1u), P.sr_k0, P.sr_k1);
+        const uint4 r = philox4x32_10_rk(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 1u), P.sr_rk);
         c4 = e2m1_sr(__fmul_rn(e[4 * q], enc), r.x) | (e2m1_sr(__fmul_rn(e[4 * q + 1], enc), r.y) << 4) |
              (e2m1_sr(__fmul_rn(e[4 * q + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[4 * q + 3], enc), r.w) << 12);
       } else {
@@ -323,36 +336,50 @@ __global__ void __launch_bounds__(256, 2) fp4_quant_rowcol_kernel(const __grid_c
   }
   __syncthreads();
 
-  // rowwise output
+  // rowwise output, four rows at a time: lane l & 3 of each 4-lane group makes the block
+  // scale (and writes the scale byte) of row i0 + (l & 3); the encode scales are shuffled out
   {
     const int64_t nsf = P.cols >> 4, s4 = (nsf + 3) >> 2;
     const int64_t kc = (T.c0 >> 4) + (T.lane >> 2);
-    const bool sf_writer = (T.lane & 3) == 0 && (P.sf_tiled ? kc < s4 * 4 : kc < nsf);
+    const int jj = T.lane & 3, grp = T.lane & ~3;
+    const bool kc_ok = P.sf_tiled ? kc < s4 * 4 : kc < nsf;
 #pragma unroll
-    for (int i = 0; i < 16; ++i) {
-      const int64_t row = T.r0 + T.w * 16 + i;
-      float e[4] = {x[i][0], x[i][1], x[i][2], x[i][3]};
-      if (P.rht_row) rht_row4(e, signs, T.lane);
-      float m = fmaxf(fmaxf(fabsf(e[0]), fabsf(e[1])), fmaxf(fabsf(e[2]), fabsf(e[3])));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 1));
-      m = fmaxf(m, __shfl_xor_sync(0xFFFFFFFFu, m, 2));
-      uint32_t sb;
-      float enc;
-      block_scale(m, S_row, enc_tab[0], sb, enc);
-      uint32_t c4;
-      if (SR_ROW) {
-        const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
-        const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
-        c4 = e2m1_sr(__fmul_rn(e[0], enc), r.x) | (e2m1_sr(__fmul_rn(e[1], enc), r.y) << 4) |
-             (e2m1_sr(__fmul_rn(e[2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[3], enc), r.w) << 12);
-      } else {
-        c4 = e2m1x2_rne(__fmul_rn(e[1], enc), __fmul_rn(e[0], enc)) |
-             (e2m1x2_rne(__fmul_rn(e[3], enc), __fmul_rn(e[2], enc)) << 8);
+    for (int i0 = 0; i0 < 16; i0 += 4) {
+      float e[4][4], m[4];
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+#pragma unroll
+        for (int k = 0; k < 4; ++k) e[j][k] = x[i0 + j][k];
+        if (P.rht_row) rht_row4(e[j], signs, T.lane);
+        m[j] = fmaxf(fmaxf(fabsf(e[j][0]), fabsf(e[j][1])), fmaxf(fabsf(e[j][2]), fabsf(e[j][3])));
+        m[j] = fmaxf(m[j], __shfl_xor_sync(0xFFFFFFFFu, m[j], 1));
+        m[j] = fmaxf(m[j], __shfl_xor_sync(0xFFFFFFFFu, m[j], 2));
       }
-      if (T.cok && row < P.rows) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)c4;
-      if (sf_writer) {
-        if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
-        else if (row < P.rows) P.sf_row[row * nsf + kc] = (uint8_t)sb;
+      uint32_t sb;
+      float enc_own;
+      block_scale(jj == 0 ? m[0] : jj == 1 ? m[1] : jj == 2 ? m[2] : m[3], S_row, enc_tab[0], sb, enc_own);
+      {
+        const int64_t row = T.r0 + T.w * 16 + i0 + jj;
+        if (kc_ok) {
+          if (P.sf_tiled) P.sf_row[sf_tiled_offset(row, kc, s4)] = (uint8_t)sb;
+          else if (row < P.rows) P.sf_row[row * nsf + kc] = (uint8_t)sb;
+        }
+      }
+#pragma unroll
+      for (int j = 0; j < 4; ++j) {
+        const int64_t row = T.r0 + T.w * 16 + i0 + j;
+        const float enc = __shfl_sync(0xFFFFFFFFu, enc_own, grp | j);
+        uint32_t c4;
+        if (SR_ROW) {
+          const uint64_t blk = (uint64_t)(row * P.cols + T.col) >> 2;
+          const uint4 r = philox4x32_10_rk(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_rk);
+          c4 = e2m1_sr(__fmul_rn(e[j][0], enc), r.x) | (e2m1_sr(__fmul_rn(e[j][1], enc), r.y) << 4) |
+               (e2m1_sr(__fmul_rn(e[j][2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[j][3], enc), r.w) << 12);
+        } else {
+          c4 = e2m1x2_rne(__fmul_rn(e[j][1], enc), __fmul_rn(e[j][0], enc)) |
+               (e2m1x2_rne(__fmul_rn(e[j][3], enc), __fmul_rn(e[j][2], enc)) << 8);
+        }
+        if (T.cok && row < P.rows) *(uint16_t*)(P.q_row + row * (P.cols >> 1) + (T.col >> 1)) = (uint16_t)c4;
       }
     }
   }
@@ -544,7 +571,7 @@ __global__ void __launch_bounds__(256) fp4_quant_row_kernel(const __grid_constan
           uint32_t c4;
           if (P.sr_row) {
             const uint64_t blk = (uint64_t)(row * P.cols + c + j) >> 2;
-            const uint4 r = philox4x32_10(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_k0, P.sr_k1);
+            const uint4 r = philox4x32_10_rk(make_uint4((uint32_t)blk, (uint32_t)(blk >> 32), 0u, 0u), P.sr_rk);
             c4 = e2m1_sr(__fmul_rn(e[j], enc), r.x) | (e2m1_sr(__fmul_rn(e[j + 1], enc), r.y) << 4) |
                  (e2m1_sr(__fmul_rn(e[j + 2], enc), r.z) << 8) | (e2m1_sr(__fmul_rn(e[j + 3], enc), r.w) << 12);
           } else {
