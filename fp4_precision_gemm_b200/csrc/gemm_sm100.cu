@@ -45,15 +45,35 @@ struct Tile {
   int m0, mend, n0, g;
 };
 
-// Tile t of the rasterized order (groups of p.group_m row tiles, column-major inside a group)
-// for output tiles `bn` columns wide.  Grouped GEMMs enumerate each expert's row tiles.
+// Position (row tile, column tile) of tile t in the rasterized order.  Row-grouped
+// (p.group_n == 0): groups of p.group_m row tiles, column-major inside a group, so the
+// group's A rows stay in L2 while B streams.  Column-grouped (p.group_n > 0): groups of
+// p.group_n column tiles, row-major inside a group, so the group's B rows stay in L2 while
+// A streams.
+__device__ __forceinline__ void raster_pos(int t, const GemmParams& p, int row_tiles, int& rt, int& nt) {
+  if (p.group_n > 0) {
+    const int per = p.group_n * row_tiles;
+    const int grp = t / per, first = grp * p.group_n;
+    const int gsz = min(p.tiles_n - first, p.group_n);
+    const int local = t - grp * per;
+    nt = first + local % gsz;
+    rt = local / gsz;
+  } else {
+    const int per = p.group_m * p.tiles_n;
+    const int grp = t / per, first = grp * p.group_m;
+    const int gsz = min(row_tiles - first, p.group_m);
+    const int local = t - grp * per;
+    rt = first + local % gsz;
+    nt = local / gsz;
+  }
+}
+
+// Tile t of the rasterized order for output tiles `bn` columns wide.  Grouped GEMMs
+// enumerate each expert's row tiles.
 __device__ __forceinline__ Tile tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
                                         const int* offs, int bn) {
-  const int per = p.group_m * p.tiles_n;
-  const int grp = t / per, first = grp * p.group_m;
-  const int gsz = min(row_tiles - first, p.group_m);
-  const int local = t - grp * per;
-  const int rt = first + local % gsz, nt = local / gsz;
+  int rt, nt;
+  raster_pos(t, p, row_tiles, rt, nt);
   Tile T;
   T.n0 = nt * bn;
   if (p.num_groups > 0) {
@@ -441,11 +461,8 @@ struct BwSmem {
 template <int BN>
 __device__ __forceinline__ Tile pair_tile_of(int t, const GemmParams& p, int row_tiles, const int* prefix,
                                              const int* offs, uint32_t rank) {
-  const int per = p.group_m * p.tiles_n;
-  const int grp = t / per, first = grp * p.group_m;
-  const int gsz = min(row_tiles - first, p.group_m);
-  const int local = t - grp * per;
-  const int rt = first + local % gsz, nt = local / gsz;
+  int rt, nt;
+  raster_pos(t, p, row_tiles, rt, nt);
   Tile T;
   T.n0 = nt * BN;
   int end;
@@ -830,19 +847,27 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
   }
 }
 
-// Raster group (row tiles per column sweep).  Concurrent tiles should share operands in L2
-// and the operand that is re-read across sweeps should stay resident: when A is the
-// smaller operand (M <= N) a group spans all row tiles (A stays resident, B streams through
-// once), capped at about 40 MB of A; otherwise tiles go row-major (group of one row tile),
-// so each row band of A streams through once against a resident B.  Grouped (expert)
+// Raster (which operand stays in L2).  Concurrent tiles should share operands in L2 and the
+// operand that is re-read across sweeps should stay resident.  When A is the smaller operand
+// (M <= N) groups of row tiles (about 40 MB of A) sweep all column tiles: A stays resident,
+// B streams through once per group.  Otherwise groups of column tiles (about 40 MB of B)
+// sweep all row tiles: B stays resident, A streams through once per group.  Grouped (expert)
 // GEMMs keep groups of kGroupM row tiles.
-static int raster_group(const GemmParams& p, int row_tiles, int tile_m) {
-  if (p.num_groups > 0) return kGroupM;
-  if (p.M > p.N) return 1;
-  const int64_t slab = (int64_t)tile_m * (p.recipe == kNvfp4 ? p.K / 2 : p.K);   // bytes of A per row tile
-  int64_t g = (40ll << 20) / (slab > 0 ? slab : 1);
-  if (g < 1) g = 1;
-  return (int)(g < row_tiles ? g : row_tiles);
+static void raster(GemmParams& q, int row_tiles, int tile_m, int tile_n) {
+  q.group_n = 0;
+  if (q.num_groups > 0) {
+    q.group_m = kGroupM;
+    return;
+  }
+  const int64_t kbytes = q.recipe == kNvfp4 ? q.K / 2 : q.K;
+  if (q.M <= q.N) {
+    int64_t g = (40ll << 20) / max((int64_t)tile_m * kbytes, (int64_t)1);
+    q.group_m = (int)max((int64_t)1, min(g, (int64_t)row_tiles));
+  } else {
+    q.group_m = 1;
+    int64_t g = (40ll << 20) / max((int64_t)tile_n * kbytes, (int64_t)1);
+    q.group_n = (int)max((int64_t)1, min(g, (int64_t)q.tiles_n));
+  }
 }
 
 template <int L, bool G, int EPI = kEpiBf16>
@@ -856,7 +881,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   GemmParams q = p;
   q.tiles_n = (p.N + kBwBN - 1) / kBwBN;
   q.tiles_m = G ? (p.M + kBwPairM - 1) / kBwPairM + p.num_groups : (p.M + kBwPairM - 1) / kBwPairM;
-  q.group_m = raster_group(q, q.tiles_m, kBwPairM);
+  raster(q, q.tiles_m, kBwPairM, kBwBN);
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
@@ -890,7 +915,7 @@ static cudaError_t launch_scaled(const GemmParams& p, const CUtensorMap& a, cons
   if (e != cudaSuccess) return e;
   GemmParams q = p;
   q.tiles_n = (p.N + kBN - 1) / kBN;
-  q.group_m = raster_group(q, q.tiles_m, kBM);
+  raster(q, q.tiles_m, kBM, kBN);
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   int grid = (int)(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;

@@ -90,6 +90,7 @@ struct GemmParams {
   int num_groups;
   int tiles_m, tiles_n;    // output tile grid (non-grouped)
   int group_m;             // raster: row tiles per column sweep (set by the launcher)
+  int group_n;             // raster: > 0 -> column tiles per row sweep instead (set by the launcher)
   int a_fmt, b_fmt;        // PERTENSOR: element format of A / B (0 E4M3, 1 E5M2)
   uint8_t* q_out;          // BLOCKWISE, optional: 1x128 E4M3 codes of the BF16 output (along N)
   float* s_out;            //   and their decode scales, s_out[(n / 128) * ld_s_out + m]
