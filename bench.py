@@ -480,11 +480,13 @@ class MxStep:
     name = "mxfp8"
     workload = "MXFP8 (and per-tensor) GEMMs (M,K,N) = (8192,4096,4096), (8192,4096,14336), (8192,14336,4096)"
 
-    def __init__(self, fq, rank):
+    def __init__(self, fq, rank, which=None):
         self.fq = fq
-        d = workloads.mxfp8(device="cuda")
+        d = workloads.mxfp8(device="cuda", which=which)
         self.items = []
         for i, (M, K, N) in enumerate(workloads.MXFP8_GEMMS):
+            if which is not None and i not in which:
+                continue
             A, W = d[f"A{i}"], d[f"W{i}"]
             dev = A.device
             it = {"M": M, "K": K, "N": N, "A": A, "W": W, "Wt": W.t().contiguous(),
@@ -864,11 +866,21 @@ def job_tflops(flop_per_rank, world, ms):
     return world * flop_per_rank / (ms * 1e-3) / 1e12
 
 
+def step_kwargs(args):
+    """Constructor arguments of the step for the smaller profiler cases (--tokens, --mx-shapes)."""
+    kw = {}
+    if args.tokens:
+        kw["M"] = args.tokens
+    if args.mx_shapes:
+        kw["which"] = tuple(int(v) for v in args.mx_shapes.split(","))
+    return kw
+
+
 def run_ours(args, rank, world, local_rank):
     import fp4_precision_gemm_b200 as fq
     torch.cuda.set_device(local_rank)
     fq.lib()
-    step = STEPS[args.workload](fq, rank, **({"M": args.tokens} if args.tokens else {}))
+    step = STEPS[args.workload](fq, rank, **step_kwargs(args))
     launches = step.launches()
     n_launch = getattr(step, "launch_count", lambda: len(launches))()
     flush = torch.empty(256 << 20, dtype=torch.uint8, device="cuda")
@@ -947,9 +959,9 @@ def run_ours(args, rank, world, local_rank):
         ach = f["bytes"] / (f["ms"] * 1e-3) / 1e9
         roof = {"kernel": dom, "bound": "hbm", "achieved": round(ach, 1), "peak": peaks["hbm_gbs"], "unit": "GB/s",
                 "frac": round(ach / peaks["hbm_gbs"], 3), "traffic": None, "peak_source": f"{src}: hbm_gbs"}
-    roof["traffic"] = traffic_for(dom, args.workload) if not args.tokens else None
+    roof["traffic"] = traffic_for(dom, args.workload) if not (args.tokens or args.mx_shapes) else None
 
-    make_step = lambda: STEPS[args.workload](fq, rank, **({"M": args.tokens} if args.tokens else {}))  # noqa: E731
+    make_step = lambda: STEPS[args.workload](fq, rank, **step_kwargs(args))  # noqa: E731
     e2e = measure_e2e(step, launches, stream, args, make_step, world) if (not args.no_e2e) else None
     value = job_tflops(step.gemm_flop, world, ms)
     out = {
@@ -1161,10 +1173,14 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="llama8b / nvfp4: token count M (default 8192); smaller cases for profiler captures")
+    ap.add_argument("--mx-shapes", default=None,
+                    help="mxfp8 only: comma list of its GEMM shapes to run (0, 1, 2); smaller profiler cases")
     args = ap.parse_args()
     args.warmup = max(args.warmup, 3)
     if args.tokens and args.workload not in ("llama8b", "nvfp4", "nvfp4_train"):
         ap.error("--tokens applies to the llama8b and nvfp4 workloads only")
+    if args.mx_shapes and args.workload != "mxfp8":
+        ap.error("--mx-shapes applies to the mxfp8 workload only")
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:
