@@ -399,10 +399,12 @@ __global__ void __launch_bounds__(kThreads, 1)
 // In each CTA warps 0-15 promote (warp w: TMEM lanes 32*(w%4).., columns 64*(w/4)..), warp
 // 16 drives the A/B TMA, warp 17 owns TMEM (and, in the leader, issues the MMAs) and warp 18
 // stages each chunk's scales in a shared-memory ring.  Every promotion thread keeps its 64
-// FP32 accumulators in registers for the whole tile; 19 warps leave it 96 registers, so the
-// partials come out of TMEM 16 columns at a time and wgrad's column scales are read from
-// shared memory just before their use.  Two 256-column TMEM partial buffers (all 512
-// columns) alternate per K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted;
+// FP32 accumulators in registers for the whole tile, and wgrad's column scales are read from
+// shared memory just before their use.  With 19 warps a thread has 96 registers, so fprop and
+// dgrad take the partial out of TMEM 16 columns per load and wait; wgrad adds warp 19 to
+// complete the helper warpgroup, which hands registers to the promotion warps (112 each) so
+// that the next 16-column load is in flight under the current FMAs.  Two 256-column TMEM
+// partial buffers (all 512 columns) alternate per K chunk, so the MMAs of chunk k + 1 run while chunk k is promoted;
 // the stage's single commit tells both the producers (stage free) and the promotion warps
 // (partial complete) of both CTAs.  The per-chunk hand-off between the MMA issuer and the
 // promotion warps costs about the same for any tile width, so the widest tile does the most
@@ -414,13 +416,27 @@ constexpr int kBwSb = 10;                       // scale ring: chunks of A/B sca
 constexpr int kBwGo = 10;                       // MMA go barriers: a multiple of both the stage count
                                                 // and the two TMEM partial buffers
 
-// Pair tile shape: 256 x 256 outputs, 16 promotion warps.
+// Pair tile shape: 256 x 256 outputs, 16 promotion warps.  wgrad (two FP32 operations per
+// element and chunk: the column scale, then the row scale) moves registers from the helper
+// warpgroup to the promotion warps so that each keeps a TMEM load in flight under its FMAs;
+// fprop and dgrad measured faster without the move (their single FMA per element leaves the
+// load latency mostly hidden by the other warps).
+template <int L>
 struct BwCfg {
   static constexpr int BN = (int)kBlockwiseTileN;       // output columns per pair tile
   static constexpr int HalfBN = BN / 2;                 // B rows loaded by each CTA
   static constexpr int EpiWarps = 4 * (BN / 64);        // 32 rows x 64 columns each
   static constexpr int ProducerWarp = EpiWarps, MmaWarp = EpiWarps + 1, ScaleWarp = EpiWarps + 2;
-  static constexpr int Threads = (EpiWarps + 3) * 32;
+  static constexpr bool Split = (L == kWgrad);           // register reallocation
+  static constexpr int IdleWarp = EpiWarps + 3;          // completes the helper warpgroup
+  static constexpr int Threads = (EpiWarps + (Split ? 4 : 3)) * 32;
+  // Registers per thread: 96 at launch (640 threads, one CTA per SM); the helper warpgroup
+  // gives 64 of each thread's back and the promotion warps take 16 more each.
+  static constexpr int RegsLaunch = 96, RegsPromo = 112, RegsHelper = 32;
+  static_assert(!Split || EpiWarps * 32 * RegsPromo + 128 * RegsHelper <= Threads * RegsLaunch,
+                "register shares exceed the launch pool");
+  static_assert(ProducerWarp % 4 == 0 && IdleWarp == ProducerWarp + 3,
+                "the helper warps form one warpgroup");
   static constexpr uint32_t BStage = HalfBN * kBKB;    // 16 KB
 };
 
@@ -430,7 +446,7 @@ struct BwCfg {
 // fprop/dgrad: [A scales][the B scales of the tile's four 64-column groups].
 template <int L>
 struct BwSmem {
-  using C = BwCfg;
+  using C = BwCfg<L>;
   static constexpr bool wg = (L == kWgrad);
   static constexpr int stages = 5;
   static constexpr uint32_t slot_sbw = 0;
@@ -508,16 +524,17 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 }  // namespace
 
 template <int L, bool GROUPED, int EPI>
-__global__ void __launch_bounds__(BwCfg::Threads, 1)
+__global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
-  constexpr int kBwBN = BwCfg::BN, kBwHalfBN = BwCfg::HalfBN, kBwEpiWarps = BwCfg::EpiWarps;
-  constexpr int kBwProducerWarp = BwCfg::ProducerWarp, kBwMmaWarp = BwCfg::MmaWarp;
-  constexpr int kBwScaleWarp = BwCfg::ScaleWarp;
-  constexpr uint32_t kBwBStage = BwCfg::BStage;
+  using C = BwCfg<L>;
+  constexpr int kBwBN = C::BN, kBwHalfBN = C::HalfBN, kBwEpiWarps = C::EpiWarps;
+  constexpr int kBwProducerWarp = C::ProducerWarp, kBwMmaWarp = C::MmaWarp;
+  constexpr int kBwScaleWarp = C::ScaleWarp;
+  constexpr uint32_t kBwBStage = C::BStage;
   constexpr int kStages = S::stages;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -570,6 +587,9 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
   const int total = row_tiles * p.tiles_n;
   const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
 
+  if (warp >= kBwEpiWarps) {
+  // wgrad: the helper warpgroup (warps 16-19) gives registers to the promotion warps
+  if constexpr (C::Split) reg_dealloc<C::RegsHelper>();
   if (warp == kBwProducerWarp) {
     // ------------------------------------------------------------------ A / B producer
     // One thread: wait for a free stage, arm the leader's barrier, issue the two TMA loads.
@@ -679,8 +699,11 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
       mma_commit_pair(final_bar, 0x1);
       mbar_wait_drain(final_bar, 0, kWaitLimitNs);
     }
+  }  // wgrad: warp 19 only completes the helper warpgroup
   } else {
     // ------------------------------------------------------------------ promotion warps 0-15
+    // wgrad: 64 accumulators plus two 16-column partials in flight
+    if constexpr (C::Split) reg_alloc<C::RegsPromo>();
     const int q = warp & 3, cgp = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(cgp * 64);
     const int rloc = q * 32 + lane;
@@ -706,40 +729,51 @@ __global__ void __launch_bounds__(BwCfg::Threads, 1)
         tc_fence_after();
         const float scale = kWg ? sa : __fmul_rn(sa, sbv);
         const float2 s2 = make_float2(scale, scale);
-        if constexpr (!kWg) {
+        // 16-column group h of the partial, times the chunk's scales, into the accumulators
+        // (wgrad also scales each column: its B scales are per column and chunk)
+        auto fma16 = [&](const uint32_t (&r)[16], int h) {
 #pragma unroll
-          for (int h = 0; h < 4; ++h) {
-            uint32_t r[16];
-            tmem_ld_32x32b_x16(t_lane + pb * kBwBN + h * 16, r);
-            tmem_ld_wait(r);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              const float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-              acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
-            }
+          for (int i = 0; i < 8; ++i) {
+            float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            if constexpr (kWg) pr = __fmul2_rn(pr, ld_shared_f2(sbw + h * 16 + 2 * i));
+            acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
           }
+        };
+        const uint32_t tb = t_lane + pb * kBwBN;
+        const uint32_t go_rel = go_leader + 8u * ((chunk + 2) % kBwGo);  // chunk + 2 reuses pb
+        if constexpr (C::Split) {
+          // the next group's load is in flight while a group's FMAs run; once the last group
+          // is in registers the TMEM buffer goes back to the MMA issuer, before its FMAs
+          uint32_t ra[16], rb[16];
+          tmem_ld_32x32b_x16(tb, ra);
+          tmem_ld_wait(ra);
+          tmem_ld_32x32b_x16(tb + 16, rb);
+          fma16(ra, 0);
+          tmem_ld_wait(rb);
+          tmem_ld_32x32b_x16(tb + 32, ra);
+          fma16(rb, 1);
+          tmem_ld_wait(ra);
+          tmem_ld_32x32b_x16(tb + 48, rb);
+          fma16(ra, 2);
+          tmem_ld_wait(rb);
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(go_rel);
+          fma16(rb, 3);
         } else {
-          // wgrad also scales each column (its B scales are per column and chunk)
 #pragma unroll
           for (int h = 0; h < 4; ++h) {
             uint32_t r[16];
-            tmem_ld_32x32b_x16(t_lane + pb * kBwBN + h * 16, r);
+            tmem_ld_32x32b_x16(tb + h * 16, r);
             tmem_ld_wait(r);
-#pragma unroll
-            for (int i = 0; i < 8; ++i) {
-              float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-              pr = __fmul2_rn(pr, ld_shared_f2(sbw + h * 16 + 2 * i));
-              acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
-            }
+            fma16(r, h);
           }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive_cluster_relaxed(go_rel);
         }
-        tc_fence_before();
         __syncwarp();
-        if (lane == 0) {
-          // chunk + 2 reuses this TMEM buffer: release it on that chunk's go barrier
-          mbar_arrive_cluster_relaxed(go_leader + 8u * ((chunk + 2) % kBwGo));
-          mbar_arrive_relaxed(&sempty[rs]);
-        }
+        if (lane == 0) mbar_arrive_relaxed(&sempty[rs]);   // the chunk's scales are read
         ++chunk;
       }
       if (!ok) break;
@@ -874,7 +908,17 @@ template <int L, bool G, int EPI = kEpiBf16>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
                                     const CUtensorMap& sb, int num_sms, cudaStream_t s) {
   auto kern = gemm_blockwise_kernel<L, G, EPI>;
-  constexpr int kBwBN = BwCfg::BN;
+  using C = BwCfg<L>;
+  constexpr int kBwBN = C::BN;
+  // The register reallocation inside the wgrad kernel adds up to exactly the launch pool at
+  // 96 registers per thread; with any other count an increase could wait forever, so refuse.
+  if constexpr (C::Split) {
+    static const int regs = [] {
+      cudaFuncAttributes fa{};
+      return cudaFuncGetAttributes(&fa, gemm_blockwise_kernel<L, G, EPI>) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (regs != C::RegsLaunch) return cudaErrorInvalidConfiguration;
+  }
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
@@ -885,7 +929,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
-  cfg.blockDim = dim3(BwCfg::Threads);
+  cfg.blockDim = dim3(C::Threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
   cudaLaunchAttribute attr[1];
