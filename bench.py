@@ -80,8 +80,10 @@ class LlamaStep:
     name = "llama8b"
     workload = "llama3-8b up-proj blockwise fwd+bwd: X 8192x4096, W 4096x14336, dY 8192x14336"
 
-    def __init__(self, fq, rank, M=8192, K=4096, N=14336):
+    def __init__(self, fq, rank, M=8192, K=4096, N=14336, separate_quant=False):
         self.fq, self.M, self.K, self.N = fq, M, K, N
+        # the three tensors' quantizations as one multi-tensor launch (default) or three calls
+        self.separate_quant = separate_quant
         self.workload = f"llama3-8b up-proj blockwise fwd+bwd: X {M}x{K}, W {K}x{N}, dY {M}x{N}"
         d = workloads.llama8b(device="cuda", M=M, K=K, N=N)
         if rank:   # other ranks: their own tokens, the same weights
@@ -118,8 +120,25 @@ class LlamaStep:
                 assert st == 0, st
             return f
 
+        # X (1x128, both outputs), W (128x128, both layouts) and dY (1x128, both outputs) in one
+        # multi-tensor launch: one ramp and one partial last wave for the three tensors
+        items = (fq.QuantItem * 3)()
+        for it, x, (R, C) in zip(items, (self.X, self.W, self.dY), ((M, K), (K, N), (M, N))):
+            it.x, it.rows, it.cols, it.ld_x = P(x), R, C, C
+        items[0].kind = items[2].kind = fq.FP8Q_ITEM_1X128
+        for it, (qr, sr, qc, sc) in ((items[0], (self.qx_r, self.sx_r, self.qx_c, self.sx_c)),
+                                     (items[2], (self.qd_r, self.sd_r, self.qd_c, self.sd_c))):
+            it.q_row, it.s_row, it.ld_s_row = P(qr), P(sr), sr.shape[1]
+            it.q_col, it.s_col, it.ld_s_col = P(qc), P(sc), sc.shape[1]
+        items[1].kind = fq.FP8Q_ITEM_128X128
+        items[1].q_t, items[1].q, items[1].s = P(self.qw_t), P(self.qw), P(self.sw)
+
         def q128():
             st = fq.fp8q_quantize_128x128(P(self.W), K, N, N, P(self.qw_t), P(self.qw), P(self.sw), fq._stream())
+            assert st == 0, st
+
+        def qall():
+            st = fq.fp8q_quantize_multi(items, 3, fq._stream())
             assert st == 0, st
 
         def gemm(a, b, layout, sa, sb, ld_sb, c):
@@ -127,12 +146,17 @@ class LlamaStep:
                 fq.gemm(a, b, fq.FP8Q_BLOCKWISE, layout, a_scale=sa, b_scale=sb, ld_sb=ld_sb, out=c)
             return f
 
-        return [
-            Launch("quantize_1x128 X (row+col)", q1x128(self.X, self.qx_r, self.sx_r, self.qx_c, self.sx_c, M, K),
-                   "quantize", bytes_=b_1x128_fused(M, K)),
-            Launch("quantize_128x128 W (both layouts)", q128, "quantize", bytes_=b_128(K, N)),
-            Launch("quantize_1x128 dY (row+col)", q1x128(self.dY, self.qd_r, self.sd_r, self.qd_c, self.sd_c, M, N),
-                   "quantize", bytes_=b_1x128_fused(M, N)),
+        if self.separate_quant:
+            quant = [
+                Launch("quantize_1x128 X (row+col)", q1x128(self.X, self.qx_r, self.sx_r, self.qx_c, self.sx_c, M, K),
+                       "quantize", bytes_=b_1x128_fused(M, K)),
+                Launch("quantize_128x128 W (both layouts)", q128, "quantize", bytes_=b_128(K, N)),
+                Launch("quantize_1x128 dY (row+col)", q1x128(self.dY, self.qd_r, self.sd_r, self.qd_c, self.sd_c, M, N),
+                       "quantize", bytes_=b_1x128_fused(M, N))]
+        else:
+            quant = [Launch("quantize X 1x128 (row+col), W 128x128 (both layouts), dY 1x128 (row+col): one launch",
+                            qall, "quantize", bytes_=b_1x128_fused(M, K) + b_128(K, N) + b_1x128_fused(M, N))]
+        return quant + [
             Launch("gemm blockwise fprop", gemm(self.qx_r, self.qw_t, fq.FP8Q_FPROP, self.sx_r, self.sw, K // 128, self.Y),
                    "gemm_blockwise", flop=2.0 * M * N * K),
             Launch("gemm blockwise dgrad", gemm(self.qd_r, self.qw, fq.FP8Q_DGRAD, self.sd_r, self.sw, K // 128, self.dX),
@@ -873,6 +897,8 @@ def step_kwargs(args):
         kw["M"] = args.tokens
     if args.mx_shapes:
         kw["which"] = tuple(int(v) for v in args.mx_shapes.split(","))
+    if args.separate_quant:
+        kw["separate_quant"] = True
     return kw
 
 
@@ -971,7 +997,9 @@ def run_ours(args, rank, world, local_rank):
         "data": "synthetic (seeded normal BF16 with outliers; see workloads.py)",
         "config": {"workload": step.workload, "l2": "flushed between steps (256 MiB write, then 256 MiB read)",
                    "gemm_tflop_per_step": round(step.gemm_flop / 1e12, 4),
-                   "parallelism": f"dp{world} (independent replicas, no collective)"},
+                   "parallelism": f"dp{world} (independent replicas, no collective)",
+                   **({"quantize_launch": "three calls" if step.separate_quant else "one multi-tensor launch"}
+                      if hasattr(step, "separate_quant") else {})},
         "roofline": roof, "kernels": kern, "gpu_launches": n_launch * args.steps,
         "clocks": clocks, "e2e": e2e, "device_status": status, "wall_s_timed_region": round(t_wall, 3),
     }
@@ -1173,6 +1201,8 @@ def main():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--tokens", type=int, default=None,
                     help="llama8b / nvfp4: token count M (default 8192); smaller cases for profiler captures")
+    ap.add_argument("--separate-quant", action="store_true",
+                    help="llama8b only: quantize X, W and dY with three calls instead of one multi-tensor launch")
     ap.add_argument("--mx-shapes", default=None,
                     help="mxfp8 only: comma list of its GEMM shapes to run (0, 1, 2); smaller profiler cases")
     args = ap.parse_args()
@@ -1181,6 +1211,8 @@ def main():
         ap.error("--tokens applies to the llama8b and nvfp4 workloads only")
     if args.mx_shapes and args.workload != "mxfp8":
         ap.error("--mx-shapes applies to the mxfp8 workload only")
+    if args.separate_quant and args.workload != "llama8b":
+        ap.error("--separate-quant applies to the llama8b workload only")
     if args.gpus < 1:
         ap.error("--gpus must be >= 1")
     if args.gpus > 1 and "WORLD_SIZE" not in os.environ:

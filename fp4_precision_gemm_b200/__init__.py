@@ -25,6 +25,8 @@ __all__ = [
     "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
     "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_tensor_delayed", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
     "quantize_nvfp4_2d16", "gemm", "device_status", "EXPORTED_SYMBOLS",
+    "fp8q_quantize_multi", "QuantItem", "FP8Q_ITEM_1X128", "FP8Q_ITEM_128X128", "FP8Q_MAX_QUANT_ITEMS",
+    "quantize_multi",
 ]
 
 FP8Q_OK = 0
@@ -35,13 +37,15 @@ FP8Q_FPROP, FP8Q_DGRAD, FP8Q_WGRAD = 0, 1, 2
 FP8Q_SF_ROWMAJOR, FP8Q_SF_MMA_TILED = 0, 1
 FP4Q_ROW, FP4Q_COL = 1, 2
 FP8Q_E4M3, FP8Q_E5M2 = 0, 1
+FP8Q_ITEM_1X128, FP8Q_ITEM_128X128 = 0, 1
+FP8Q_MAX_QUANT_ITEMS = 8
 
 EXPORTED_SYMBOLS = [
     "fp8q_quantize_1x128", "fp8q_quantize_128x128", "fp8q_quantize_mx32", "fp8q_quantize_tensor",
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
-    "fp4q_quantize_2d16",
+    "fp4q_quantize_2d16", "fp8q_quantize_multi",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -51,6 +55,17 @@ class Fp8qError(RuntimeError):
     def __init__(self, status, where):
         self.status = status
         super().__init__(f"{where}: status {status} ({_status_str(status)})")
+
+
+class QuantItem(ctypes.Structure):
+    """Mirror of fp8q_quant_item (field order and types as in include/fp8q.h)."""
+    _fields_ = [
+        ("kind", ctypes.c_int32), ("x", ctypes.c_void_p),
+        ("rows", ctypes.c_int64), ("cols", ctypes.c_int64), ("ld_x", ctypes.c_int64),
+        ("q_row", ctypes.c_void_p), ("s_row", ctypes.c_void_p), ("ld_s_row", ctypes.c_int64),
+        ("q_col", ctypes.c_void_p), ("s_col", ctypes.c_void_p), ("ld_s_col", ctypes.c_int64),
+        ("q_t", ctypes.c_void_p), ("q", ctypes.c_void_p), ("s", ctypes.c_void_p),
+    ]
 
 
 class GemmArgs(ctypes.Structure):
@@ -94,6 +109,7 @@ def lib():
                                              _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp4q_quantize_2d16.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
+        L.fp8q_quantize_multi.argtypes = [ctypes.POINTER(QuantItem), ctypes.c_int32, _vp]
         L.fp8q_sf_bytes.argtypes = [_int, _i64, _i64, _int]
         L.fp8q_sf_bytes.restype = ctypes.c_size_t
         L.fp8q_get_device_status.argtypes = [_vp]
@@ -110,7 +126,8 @@ def lib():
                                                      "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled",
                                                      "fp8q_get_device_status", "fp8q_release_scratch",
                                                      "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped",
-                                                     "fp8q_quantize_tensor_delayed", "fp4q_quantize_2d16"):
+                                                     "fp8q_quantize_tensor_delayed", "fp4q_quantize_2d16",
+                                                     "fp8q_quantize_multi"):
                 f.restype = ctypes.c_int
         _LIB = L
     return _LIB
@@ -145,6 +162,11 @@ def fp8q_quantize_1x128(x, rows, cols, ld_x, q_row, s_row, ld_s_row, q_col, s_co
 
 def fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream):
     return lib().fp8q_quantize_128x128(w, K, N, ld_w, q_t, q, s, stream)
+
+
+def fp8q_quantize_multi(items, n_items, stream):
+    """items: a ctypes array of QuantItem (or None with n_items == 0)."""
+    return lib().fp8q_quantize_multi(items, n_items, stream)
 
 
 def fp8q_quantize_128x128_grouped(w, groups, K, N, ld_w, q_t, q, s, stream):
@@ -243,6 +265,50 @@ def quantize_128x128(w, transposed=True, plain=True, stream=None):
                                _ptr(out["s"]), _stream(stream))
     _check(st, "fp8q_quantize_128x128")
     return out
+
+
+def quantize_multi(specs, stream=None):
+    """Several quantizations in one launch.  specs: a list of ("1x128", x, rowwise, colwise)
+    and ("128x128", w, transposed, plain) tuples.  Returns one output dict per spec, laid
+    out exactly as quantize_1x128 / quantize_128x128 return them."""
+    items = (QuantItem * max(len(specs), 1))()
+    outs = []
+    n = 0
+    for spec in specs:
+        kind, x, a, b = spec
+        _check_bf16(x)
+        R, C = x.shape
+        dev = x.device
+        it = items[n] if x.numel() else QuantItem()   # an empty tensor has nothing to launch
+        n += 1 if x.numel() else 0
+        it.x, it.rows, it.cols, it.ld_x = x.data_ptr(), R, C, x.stride(0)
+        out = {}
+        if kind == "1x128":
+            it.kind = FP8Q_ITEM_1X128
+            if a:
+                out["q_row"] = torch.empty((R, C), dtype=torch.uint8, device=dev)
+                out["s_row"] = torch.empty((C // 128, max(R, 1) + (-max(R, 1)) % 4), dtype=torch.float32, device=dev)
+                it.q_row, it.s_row, it.ld_s_row = out["q_row"].data_ptr(), out["s_row"].data_ptr(), out["s_row"].shape[1]
+            if b:
+                out["q_col"] = torch.empty((C, R), dtype=torch.uint8, device=dev)
+                out["s_col"] = torch.empty((R // 128, C + (-C) % 4), dtype=torch.float32, device=dev)
+                it.q_col, it.s_col, it.ld_s_col = out["q_col"].data_ptr(), out["s_col"].data_ptr(), out["s_col"].shape[1]
+        elif kind == "128x128":
+            it.kind = FP8Q_ITEM_128X128
+            out["s"] = torch.empty((C // 128, R // 128), dtype=torch.float32, device=dev)
+            it.s = out["s"].data_ptr()
+            if a:
+                out["q_t"] = torch.empty((C, R), dtype=torch.uint8, device=dev)
+                it.q_t = out["q_t"].data_ptr()
+            if b:
+                out["q"] = torch.empty((R, C), dtype=torch.uint8, device=dev)
+                it.q = out["q"].data_ptr()
+        else:
+            raise ValueError(f"unknown quantization kind {kind!r}")
+        outs.append(out)
+    st = fp8q_quantize_multi(items, n, _stream(stream))
+    _check(st, "fp8q_quantize_multi")
+    return outs
 
 
 def quantize_128x128_grouped(w, transposed=True, plain=True, stream=None):

@@ -172,35 +172,104 @@ static fp8q_status check_input(const void* x, int64_t rows, int64_t cols, int64_
 
 static int64_t tiles_of(int64_t rows, int64_t cols) { return ((rows + 127) / 128) * ((cols + 127) / 128); }
 
-fp8q_status fp8q_quantize_1x128(const void* x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t* q_row,
-                                float* s_row, int64_t ld_s_row, uint8_t* q_col, float* s_col, int64_t ld_s_col,
-                                void* stream) {
+}  // extern "C"
+
+namespace {
+
+// Validation and launch parameters of one 1x128 quantization (the rules of
+// fp8q_quantize_1x128); `tiles` is 0 when there is nothing to do.
+fp8q_status plan_1x128(const void* x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t* q_row, float* s_row,
+                       int64_t ld_s_row, uint8_t* q_col, float* s_col, int64_t ld_s_col, TileQuantParams& p,
+                       bool& row, bool& col, int64_t& tiles) {
   fp8q_status st = check_input(x, rows, cols, ld_x);
   if (st != FP8Q_OK) return st;
-  const bool row = q_row || s_row, col = q_col || s_col;
+  row = q_row || s_row;
+  col = q_col || s_col;
   if (!row && !col) return FP8Q_ERR_NULL;
   if ((row && (!q_row || !s_row)) || (col && (!q_col || !s_col))) return FP8Q_ERR_NULL;
   if (row && (cols % 128 != 0 || ld_s_row < rows || ld_s_row % 4 != 0)) return FP8Q_ERR_SHAPE;
   if (col && (rows % 128 != 0 || cols % 16 != 0 || ld_s_col < cols || ld_s_col % 4 != 0)) return FP8Q_ERR_SHAPE;
   if ((row && !aligned16(q_row)) || (col && !aligned16(q_col))) return FP8Q_ERR_ALIGN;
-  if (rows == 0 || cols == 0) return FP8Q_OK;
-  TileQuantParams p{static_cast<const uint16_t*>(x), rows, cols, ld_x, q_row, s_row, ld_s_row,
-                    q_col, s_col, ld_s_col, (int)((cols + 127) / 128), 0};
-  return from_cuda(launch_tile_quant(kTile1x128, row, col, p, tiles_of(rows, cols), static_cast<cudaStream_t>(stream)));
+  p = TileQuantParams{static_cast<const uint16_t*>(x), rows, cols, ld_x, q_row, s_row, ld_s_row,
+                      q_col, s_col, ld_s_col, (int)((cols + 127) / 128), 0};
+  tiles = (rows == 0 || cols == 0) ? 0 : tiles_of(rows, cols);
+  return FP8Q_OK;
 }
 
-fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t ld_w, uint8_t* q_t, uint8_t* q,
-                                  float* s, void* stream) {
+// The same for one 128x128 quantization (the rules of fp8q_quantize_128x128).
+fp8q_status plan_128x128(const void* w, int64_t K, int64_t N, int64_t ld_w, uint8_t* q_t, uint8_t* q, float* s,
+                         TileQuantParams& p, int64_t& tiles) {
   fp8q_status st = check_input(w, K, N, ld_w);
   if (st != FP8Q_OK) return st;
   if (!s) return FP8Q_ERR_NULL;
   if (K % 128 != 0 || N % 128 != 0) return FP8Q_ERR_SHAPE;
   if ((q && !aligned16(q)) || (q_t && !aligned16(q_t))) return FP8Q_ERR_ALIGN;
-  if (K == 0 || N == 0) return FP8Q_OK;
-  TileQuantParams p{static_cast<const uint16_t*>(w), K, N, ld_w, q, s, K / 128, q_t, nullptr, 0,
-                    (int)(N / 128), 0};
-  return from_cuda(launch_tile_quant(kTile128, q != nullptr, q_t != nullptr, p, tiles_of(K, N),
+  p = TileQuantParams{static_cast<const uint16_t*>(w), K, N, ld_w, q, s, K / 128, q_t, nullptr, 0,
+                      (int)(N / 128), 0};
+  tiles = (K == 0 || N == 0) ? 0 : tiles_of(K, N);
+  return FP8Q_OK;
+}
+
+}  // namespace
+
+extern "C" {
+
+fp8q_status fp8q_quantize_1x128(const void* x, int64_t rows, int64_t cols, int64_t ld_x, uint8_t* q_row,
+                                float* s_row, int64_t ld_s_row, uint8_t* q_col, float* s_col, int64_t ld_s_col,
+                                void* stream) {
+  TileQuantParams p{};
+  bool row = false, col = false;
+  int64_t tiles = 0;
+  fp8q_status st = plan_1x128(x, rows, cols, ld_x, q_row, s_row, ld_s_row, q_col, s_col, ld_s_col, p, row, col, tiles);
+  if (st != FP8Q_OK || tiles == 0) return st;
+  return from_cuda(launch_tile_quant(kTile1x128, row, col, p, tiles, static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t ld_w, uint8_t* q_t, uint8_t* q,
+                                  float* s, void* stream) {
+  TileQuantParams p{};
+  int64_t tiles = 0;
+  fp8q_status st = plan_128x128(w, K, N, ld_w, q_t, q, s, p, tiles);
+  if (st != FP8Q_OK || tiles == 0) return st;
+  return from_cuda(launch_tile_quant(kTile128, q != nullptr, q_t != nullptr, p, tiles,
                                      static_cast<cudaStream_t>(stream)));
+}
+
+fp8q_status fp8q_quantize_multi(const fp8q_quant_item* items, int32_t n_items, void* stream) {
+  if (n_items < 0 || n_items > FP8Q_MAX_QUANT_ITEMS) return FP8Q_ERR_SHAPE;
+  if (n_items > 0 && !items) return FP8Q_ERR_NULL;
+  TileQuantMulti m{};
+  int64_t tiles = 0;
+  for (int i = 0; i < n_items; ++i) {   // every item is checked before anything is launched
+    const fp8q_quant_item& it = items[i];
+    TileQuantParams p{};
+    int64_t t = 0;
+    int kind;
+    fp8q_status st;
+    if (it.kind == FP8Q_ITEM_1X128) {
+      bool row = false, col = false;
+      st = plan_1x128(it.x, it.rows, it.cols, it.ld_x, it.q_row, it.s_row, it.ld_s_row, it.q_col, it.s_col,
+                      it.ld_s_col, p, row, col, t);
+      kind = row && col ? kMulti1x128Both : row ? kMulti1x128Row : kMulti1x128Col;
+    } else if (it.kind == FP8Q_ITEM_128X128) {
+      st = plan_128x128(it.x, it.rows, it.cols, it.ld_x, it.q_t, it.q, it.s, p, t);
+      kind = it.q && it.q_t ? kMulti128Both : it.q ? kMulti128Row : kMulti128Col;
+      if (st == FP8Q_OK && !it.q && !it.q_t) st = FP8Q_ERR_NULL;
+    } else {
+      return FP8Q_ERR_UNSUPPORTED;
+    }
+    if (st != FP8Q_OK) return st;
+    if (t == 0) continue;
+    m.kind[m.n] = kind;
+    m.item[m.n] = p;
+    m.tile_begin[m.n] = tiles;
+    ++m.n;
+    tiles += t;
+  }
+  if (tiles == 0) return FP8Q_OK;
+  if (tiles >= (1ll << 31)) return FP8Q_ERR_SHAPE;
+  m.tile_begin[m.n] = tiles;
+  return from_cuda(launch_tile_quant_multi(m, tiles, static_cast<cudaStream_t>(stream)));
 }
 
 fp8q_status fp8q_quantize_128x128_grouped(const void* w, int64_t groups, int64_t K, int64_t N, int64_t ld_w,

@@ -28,6 +28,20 @@ struct TileQuantParams {
 cudaError_t launch_tile_quant(int mode, bool row, bool col, const TileQuantParams& p,
                               int64_t tiles, cudaStream_t s);
 
+// Multi-tensor launch: up to kMaxMultiItems tensors, each a 1x128 (rowwise, colwise or both)
+// or a 128x128 (either or both layouts) quantization; item i owns the launch's tiles
+// [tile_begin[i], tile_begin[i + 1]).
+constexpr int kMaxMultiItems = 8;
+enum { kMulti1x128Row = 0, kMulti1x128Col = 1, kMulti1x128Both = 2, kMulti128Row = 3, kMulti128Col = 4,
+       kMulti128Both = 5 };
+struct TileQuantMulti {
+  int n;
+  int kind[kMaxMultiItems];
+  int64_t tile_begin[kMaxMultiItems + 1];
+  TileQuantParams item[kMaxMultiItems];
+};
+cudaError_t launch_tile_quant_multi(const TileQuantMulti& m, int64_t tiles, cudaStream_t s);
+
 // Per-tensor current scaling: amax pass into *amax_bits (zeroed by the caller), then cast.
 cudaError_t launch_tensor_amax(const uint16_t* x, int64_t rows, int64_t cols, int64_t ld_x,
                                uint32_t* amax_bits, cudaStream_t s);

@@ -40,6 +40,15 @@ __device__ __forceinline__ uint32_t word(const uint4& v, int jw) {
 // Physical 8-byte chunk of logical row-chunk k in transposed row c of the staging tile.
 __device__ __forceinline__ int tq_chunk(int c, int k) { return k ^ ((c >> 3) ^ (c & 1)); }
 
+// Shared memory of one tile: reduction slots, column scales / exponents and the transposed
+// staging tile.
+struct TileSmem {
+  uint32_t red[8][64];
+  float colsf[128];
+  uint8_t colexp[128 * 4];
+  __align__(16) uint8_t tq[128 * 128];
+};
+
 }  // namespace
 
 // Resident CTAs per SM: the kernel is latency bound on its loads, so the register budget is
@@ -47,17 +56,18 @@ __device__ __forceinline__ int tq_chunk(int c, int k) { return k ^ ((c >> 3) ^ (
 template <bool ROW, bool COL>
 constexpr int kTileQuantCtas = (ROW && !COL) ? 3 : 4;
 
+// One 128x128 tile (index `tile` of the call, grouped calls counting every matrix's tiles)
+// quantized by the CTA's 256 threads.
 template <int MODE, bool ROW, bool COL>
-__global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kernel(const __grid_constant__ TileQuantParams P) {
-  __shared__ uint32_t red[8][64];
-  __shared__ float colsf[128];
-  __shared__ uint8_t colexp[128 * 4];
-  __shared__ __align__(16) uint8_t tq[COL ? 128 * 128 : 16];
+__device__ __forceinline__ void tile_quant_tile(const TileQuantParams& P, int64_t tile, TileSmem& sm) {
+  auto& red = sm.red;
+  auto& colsf = sm.colsf;
+  auto& colexp = sm.colexp;
+  auto& tq = sm.tq;
 
   const int t = threadIdx.x, warp = t >> 5;
   const int cs = t & 15, rb = t >> 4;
   // grouped calls: CTA -> (matrix b, tile within it); every operand pointer moves by b strides
-  int64_t tile = blockIdx.x;
   const int64_t bidx = P.batch_tiles ? tile / P.batch_tiles : 0;
   tile -= bidx * P.batch_tiles;
   const uint16_t* X = P.x + bidx * P.x_bstride;
@@ -247,6 +257,45 @@ __global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kern
   }
 }
 
+template <int MODE, bool ROW, bool COL>
+__global__ void __launch_bounds__(256, kTileQuantCtas<ROW, COL>) tile_quant_kernel(const __grid_constant__ TileQuantParams P) {
+  __shared__ TileSmem sm;
+  tile_quant_tile<MODE, ROW, COL>(P, blockIdx.x, sm);
+}
+
+// Several tensors in one launch (each its own mode and outputs): CTA b takes tile
+// b - tile_begin[i] of the item i whose range holds b, so the launch pays one ramp and one
+// partial last wave for all of them.  The rowwise-only forms need more registers (3 CTAs
+// per SM); a launch without them is compiled for 4.
+template <bool ROWONLY>
+__global__ void __launch_bounds__(256, ROWONLY ? 3 : 4) tile_quant_multi_kernel(const __grid_constant__ TileQuantMulti M) {
+  __shared__ TileSmem sm;
+  const int64_t b = blockIdx.x;
+  int i = 0;
+  while (i + 1 < M.n && b >= M.tile_begin[i + 1]) ++i;
+  const TileQuantParams& P = M.item[i];
+  const int64_t tile = b - M.tile_begin[i];
+  switch (M.kind[i]) {
+    case kMulti1x128Col: tile_quant_tile<kTile1x128, false, true>(P, tile, sm); break;
+    case kMulti1x128Both: tile_quant_tile<kTile1x128, true, true>(P, tile, sm); break;
+    case kMulti128Col: tile_quant_tile<kTile128, false, true>(P, tile, sm); break;
+    case kMulti128Both: tile_quant_tile<kTile128, true, true>(P, tile, sm); break;
+    default:
+      if constexpr (ROWONLY) {
+        if (M.kind[i] == kMulti1x128Row) tile_quant_tile<kTile1x128, true, false>(P, tile, sm);
+        else tile_quant_tile<kTile128, true, false>(P, tile, sm);
+      }
+      break;
+  }
+}
+
+cudaError_t launch_tile_quant_multi(const TileQuantMulti& m, int64_t tiles, cudaStream_t s) {
+  bool rowonly = false;
+  for (int i = 0; i < m.n; ++i) rowonly |= (m.kind[i] == kMulti1x128Row || m.kind[i] == kMulti128Row);
+  if (rowonly) tile_quant_multi_kernel<true><<<dim3((unsigned)tiles), dim3(256), 0, s>>>(m);
+  else tile_quant_multi_kernel<false><<<dim3((unsigned)tiles), dim3(256), 0, s>>>(m);
+  return cudaGetLastError();
+}
 
 cudaError_t launch_tile_quant(int mode, bool row, bool col, const TileQuantParams& p,
                               int64_t tiles, cudaStream_t s) {

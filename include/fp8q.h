@@ -126,6 +126,35 @@ fp8q_status fp8q_quantize_128x128(const void* w, int64_t K, int64_t N, int64_t l
 fp8q_status fp8q_quantize_128x128_grouped(const void* w, int64_t groups, int64_t K, int64_t N, int64_t ld_w,
                                           uint8_t* q_t, uint8_t* q, float* s, void* stream);
 
+/* [DSV3] "Fine-grained quantization", "Online quantization": several tensors in one launch.
+ * Each item is one fp8q_quantize_1x128 call (kind FP8Q_ITEM_1X128: x is rows x cols, the
+ * q_row / s_row / ld_s_row and q_col / s_col / ld_s_col outputs) or one
+ * fp8q_quantize_128x128 call (kind FP8Q_ITEM_128X128: x is K x N with K = rows, N = cols,
+ * outputs q_t, q and s), with exactly that call's requirements, layouts and results; the
+ * fields of the other kind are ignored.  For 128x128 at least one of q_t and q is required.
+ * Up to FP8Q_MAX_QUANT_ITEMS items; every item is validated before anything is launched
+ * (the first failing item's status is returned and nothing runs).  One kernel quantizes
+ * all items' 128x128 tiles, so the GPU is filled across tensors and the call pays one launch
+ * and one partial last wave.  Items must not overlap each other's outputs.  Items with no
+ * elements are skipped; n_items == 0 -> FP8Q_OK, nothing launched. */
+#define FP8Q_MAX_QUANT_ITEMS 8
+typedef enum { FP8Q_ITEM_1X128 = 0, FP8Q_ITEM_128X128 = 1 } fp8q_item_kind;
+typedef struct fp8q_quant_item {
+  int32_t kind;                   /* fp8q_item_kind */
+  const void* x;                  /* BF16 input */
+  int64_t rows, cols, ld_x;
+  uint8_t* q_row;                 /* FP8Q_ITEM_1X128 outputs */
+  float* s_row;
+  int64_t ld_s_row;
+  uint8_t* q_col;
+  float* s_col;
+  int64_t ld_s_col;
+  uint8_t* q_t;                   /* FP8Q_ITEM_128X128 outputs */
+  uint8_t* q;
+  float* s;
+} fp8q_quant_item;
+fp8q_status fp8q_quantize_multi(const fp8q_quant_item* items, int32_t n_items, void* stream);
+
 /* [NeMo] MXFP8: 32-element blocks, E8M0 scale = smallest e with amax <= 448 * 2^e
  * (amax == 0 -> e = -127; e clamped to [-127, 127]; byte e + 127), codes
  * E4M3(fp32(x * 2^-e)).

@@ -232,3 +232,37 @@ def test_fused_output_quantization_validation(L):
     assert g(_args(**{**base, "ld_q_out": 264}), s) == fq.FP8Q_ERR_SHAPE                    # % 16
     assert g(_args(**{**base, "ld_s_out": 100}), s) == fq.FP8Q_ERR_SHAPE                    # >= M
     assert g(_args(**{**base, "q_out": MISALIGNED.value}), s) == fq.FP8Q_ERR_ALIGN
+
+
+def test_quantize_multi_validates_every_item_before_launching():
+    """Bad items are rejected with their single-call status, before any launch (no GPU
+    here, so a launch would fail with FP8Q_ERR_CUDA instead)."""
+    S = 0x10000                   # never dereferenced: validation fails before any launch
+    def item(kind, rows, cols, **kw):
+        it = fq.QuantItem()
+        it.kind, it.x, it.rows, it.cols, it.ld_x = kind, S, rows, cols, cols
+        for k, v in kw.items():
+            setattr(it, k, v)
+        return it
+    def call(*its):
+        arr = (fq.QuantItem * max(len(its), 1))(*its)
+        return fq.fp8q_quantize_multi(arr, len(its), None)
+    one = dict(q_row=S, s_row=S, ld_s_row=128)
+    w = dict(q_t=S, q=S, s=S)
+    assert call() == fq.FP8Q_OK
+    assert fq.fp8q_quantize_multi(None, 1, None) == fq.FP8Q_ERR_NULL
+    arr = (fq.QuantItem * 9)(*[item(fq.FP8Q_ITEM_1X128, 0, 128, **one) for _ in range(9)])
+    assert fq.fp8q_quantize_multi(arr, 9, None) == fq.FP8Q_ERR_SHAPE             # more than 8 items
+    assert fq.fp8q_quantize_multi(arr, -1, None) == fq.FP8Q_ERR_SHAPE
+    assert call(item(7, 128, 128, **one)) == fq.FP8Q_ERR_UNSUPPORTED              # unknown kind
+    assert call(item(fq.FP8Q_ITEM_1X128, 128, 100, **one)) == fq.FP8Q_ERR_SHAPE  # cols % 128
+    assert call(item(fq.FP8Q_ITEM_1X128, 128, 128)) == fq.FP8Q_ERR_NULL          # no output
+    assert call(item(fq.FP8Q_ITEM_128X128, 128, 128, s=S)) == fq.FP8Q_ERR_NULL   # neither layout
+    assert call(item(fq.FP8Q_ITEM_128X128, 128, 128, q=S)) == fq.FP8Q_ERR_NULL   # no scales
+    assert call(item(fq.FP8Q_ITEM_128X128, 100, 128, **w)) == fq.FP8Q_ERR_SHAPE  # K % 128
+    # a valid item first: the bad second item still stops the call before any launch
+    assert call(item(fq.FP8Q_ITEM_1X128, 128, 128, **one),
+                item(fq.FP8Q_ITEM_1X128, 128, 128, q_row=S + 1, s_row=S, ld_s_row=128)) == fq.FP8Q_ERR_ALIGN
+    # empty items are skipped: nothing to launch
+    assert call(item(fq.FP8Q_ITEM_1X128, 0, 128, **one), item(fq.FP8Q_ITEM_128X128, 128, 0, **w)) == fq.FP8Q_OK
+    assert ctypes.sizeof(fq.QuantItem) == 112

@@ -76,6 +76,65 @@ def test_128x128_parity(cuda_lib, K, N):
     assert np.array_equal(f32bits(host(out["s"])), f32bits(s))
 
 
+# ----------------------------------------------------------------------------- multi-tensor
+def _check_multi_item(spec, out, x):
+    bits = workloads.bf16_bits(x)
+    R, C = x.shape
+    if spec[0] == "1x128":
+        if spec[2]:
+            q, s = Q.quantize_1x128_rowwise(bits)
+            assert np.array_equal(host(out["q_row"]), q)
+            assert np.array_equal(f32bits(host(out["s_row"])[:, :R]), f32bits(s))
+        if spec[3]:
+            q, s = Q.quantize_1x128_colwise(bits)
+            assert np.array_equal(host(out["q_col"]), q)
+            assert np.array_equal(f32bits(host(out["s_col"])[:, :C]), f32bits(s))
+    else:
+        q, qt, s = Q.quantize_128x128(bits)
+        assert np.array_equal(f32bits(host(out["s"])), f32bits(s))
+        if spec[2]:
+            assert np.array_equal(host(out["q_t"]), qt)
+        if spec[3]:
+            assert np.array_equal(host(out["q"]), q)
+
+
+@pytest.mark.parametrize("specs", [
+    # the step's three tensors (activation, weight, gradient): both outputs each
+    [("1x128", (384, 640), True, True), ("128x128", (384, 640), True, True), ("1x128", (256, 896), True, True)],
+    # every item form, rowwise-only among them (the 3-CTA launch), an empty item skipped
+    [("1x128", (300, 640), True, False), ("1x128", (384, 656), False, True), ("128x128", (512, 256), False, True),
+     ("128x128", (256, 384), True, False), ("1x128", (0, 256), True, False), ("1x128", (1, 128), True, False)],
+])
+def test_quantize_multi_matches_the_oracle_per_item(cuda_lib, specs):
+    """One multi-tensor launch gives every item exactly what its own quantizer gives
+    (oracle), codes and scales bit for bit."""
+    fq = cuda_lib
+    xs = [crafted_bf16(max(R, 1), C, seed=31 * i + R + C)[:R] for i, (_, (R, C), _, _) in enumerate(specs)]
+    outs = fq.quantize_multi([(k, x.cuda(), a, b) for (k, _, a, b), x in zip(specs, xs)])
+    torch.cuda.synchronize()
+    assert fq.device_status() == 0
+    for spec, out, x in zip(specs, outs, xs):
+        if x.shape[0] == 0:
+            continue
+        _check_multi_item(spec, out, x)
+
+
+def test_quantize_multi_equals_separate_calls_on_the_llama8b_step(cuda_lib):
+    """The Llama-3-8B step's X (1x128 both), W (128x128 both) and dY (1x128 both) in one
+    launch equal the three separate calls byte for byte."""
+    fq = cuda_lib
+    W = workloads.llama8b(device="cuda")
+    X, Wt, dY = W["X"], W["W"], W["dY"]
+    outs = fq.quantize_multi([("1x128", X, True, True), ("128x128", Wt, True, True), ("1x128", dY, True, True)])
+    ref = [fq.quantize_1x128(X, rowwise=True, colwise=True), fq.quantize_128x128(Wt),
+           fq.quantize_1x128(dY, rowwise=True, colwise=True)]
+    torch.cuda.synchronize()
+    for a, b in zip(outs, ref):
+        assert sorted(a) == sorted(b)
+        for k in a:
+            assert torch.equal(a[k], b[k]), k
+
+
 # ----------------------------------------------------------------------------- MX
 def test_128x128_grouped_matches_each_matrix(cuda_lib):
     """A stack of expert weight matrices quantized in one grouped call equals quantizing
