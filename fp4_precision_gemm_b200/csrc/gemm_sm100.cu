@@ -16,7 +16,8 @@
 //
 // Both kernels are persistent (one CTA per SM) and warp-specialized: one warp drives TMA
 // into a ring of 128B-swizzled K chunks (128 bytes of K per stage), one warp allocates TMEM
-// and a single thread issues tcgen05.mma, the remaining warps drain TMEM.
+// and a single thread issues tcgen05.mma, the remaining warps drain TMEM (and, for MX and
+// NVFP4, four warps store each stage's scale factors into TMEM).
 // Every wait is bounded: a wait that runs out records a timeout in the device status word,
 // raises the CTA's abort flag and the roles wind down (waiting, bounded, for their own
 // copies and MMAs in flight) before TMEM is released.
@@ -139,28 +140,33 @@ __device__ __forceinline__ void add4_f32(const GemmParams& p, int m, int n, uint
 
 // ------------------------------------------------------------------ hardware-scaled kernel
 // MXFP8, NVFP4 and per-tensor: 128 x 256 output tiles accumulated across all of K in TMEM
-// (256 columns per accumulator); the scale factors of MX / NVFP4 stages are copied from
-// shared memory into TMEM with tcgen05.cp and consumed by the block-scaled MMA.  Per-tensor
-// has no scale columns, so it keeps two accumulators and the epilogue of one tile overlaps
-// the MMAs of the next; MX / NVFP4 drain their single accumulator before the next tile.
+// (256 columns per accumulator).  The scale factors of an MX / NVFP4 stage arrive in shared
+// memory with its A/B chunk; four scale warps (one per TMEM lane quadrant) move them into the
+// stage's TMEM scale columns with tcgen05.st and signal the MMA issuer, so the tensor pipe
+// only runs MMAs (a tcgen05.cp per 512-byte atom, issued by the MMA thread, occupied the
+// tensor pipe for about as long as the MMAs of an NVFP4 stage).  Per-tensor has no scale
+// columns, so it keeps two accumulators and the epilogue of one tile overlaps the MMAs of
+// the next; MX / NVFP4 drain their single accumulator before the next tile.
 // The epilogue stages BF16 rows through shared memory (width per recipe, as shared memory
 // allows) so global stores are contiguous row segments.
 constexpr int kBN = 256;
 constexpr int kStages = 4;
 constexpr int kEpiWarps = 8;
-constexpr int kProducerWarp = 8, kMmaWarp = 9;
-constexpr int kThreads = 320;
+constexpr int kProducerWarp = 8, kMmaWarp = 9, kSfWarp0 = 10;   // scale warps 10-13 (MX, NVFP4)
 constexpr uint32_t kBStage = kBN * kBKB;  // 32 KB
 
 template <int R> struct Cfg;
 template <> struct Cfg<kPerTensor> {
   static constexpr uint32_t sfa = 0, sfb = 0, tmem_cols = 512, acc_bufs = 2, epi_cols = 64;
+  static constexpr int threads = 320;
 };
 template <> struct Cfg<kMx> {
   static constexpr uint32_t sfa = 512, sfb = 1024, tmem_cols = 512, sf_cols = 16, acc_bufs = 1, epi_cols = 32;
+  static constexpr int threads = 448;
 };
 template <> struct Cfg<kNvfp4> {
   static constexpr uint32_t sfa = 2048, sfb = 4096, tmem_cols = 512, sf_cols = 64, acc_bufs = 1, epi_cols = 16;
+  static constexpr int threads = 448;
 };
 
 template <int R>
@@ -172,7 +178,7 @@ struct Smem {
   static constexpr uint32_t stage_c = 32 * Cfg<R>::epi_cols * 2;   // per epilogue warp
   static constexpr uint32_t cst = sf + kStages * sf_stage;
   static constexpr uint32_t bars = cst + kEpiWarps * stage_c;
-  static constexpr uint32_t n_bars = 2 * kStages + 2 * Cfg<R>::acc_bufs + 1;
+  static constexpr uint32_t n_bars = 4 * kStages + 2 * Cfg<R>::acc_bufs + 1;
   static constexpr uint32_t misc = bars + n_bars * 8;
   static constexpr uint32_t alloc = misc + 16 + 1024;  // + room to align the base to 1024 bytes
   static_assert(alloc <= 227 * 1024, "shared memory");
@@ -205,7 +211,7 @@ __device__ __forceinline__ void stage_store_rows(uint4* stg, const float* v, con
 }  // namespace
 
 template <int R>
-__global__ void __launch_bounds__(kThreads, 1)
+__global__ void __launch_bounds__(Cfg<R>::threads, 1)
     gemm_scaled_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                        const __grid_constant__ CUtensorMap tma_b) {
   using S = Smem<R>;
@@ -217,6 +223,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* accfull = empty + kStages;   // [kAcc] the tile's accumulator is complete
   uint64_t* accempty = accfull + kAcc;   // [kAcc] the epilogue has drained it
   uint64_t* final_bar = accempty + kAcc; // MMA wind-down
+  uint64_t* sfready = final_bar + 1;     // [kStages] MX / NVFP4: the stage's scales are in TMEM
+  uint64_t* sffull = sfready + kStages;  // [kStages] MX / NVFP4: the stage's scale bytes landed
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + S::misc);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + S::misc + 4);
 
@@ -233,6 +241,10 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&accempty[b], kEpiWarps);  // one arrival per epilogue warp
     }
     mbar_init(final_bar, 1);
+    for (int i = 0; i < kStages; ++i) {
+      mbar_init(&sfready[i], 4);   // one arrival per scale warp
+      mbar_init(&sffull[i], 1);
+    }
     *abort_flag = 0;
     fence_barrier_init();
   }
@@ -258,26 +270,32 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
-          mbar_arrive_expect_tx(&full[s], kAStage + kBStage + Cfg<R>::sfa + Cfg<R>::sfb);
-          tma_load_2d(smem + S::a + s * kAStage, &tma_a, &full[s], kb * kBKB, T.m0);
-          tma_load_2d(smem + S::b + s * kBStage, &tma_b, &full[s], kb * kBKB, T.n0);
-          if constexpr (R == kMx || R == kNvfp4) {
-            // scale atoms: 512 bytes per 128 rows x 4 scale columns; MX: 1 atom per chunk,
-            // NVFP4: 4 atoms per chunk, for A's row band and B's two row bands.  A B band
-            // past the padded buffer end is replaced by band 0 (its columns are never stored).
+          // scale atoms: 512 bytes per 128 rows x 4 scale columns; MX: 1 atom per chunk,
+          // NVFP4: 4 atoms per chunk, for A's row band and B's two row bands.  A B band past
+          // the padded buffer end is replaced by band 0 (its columns are never stored).
+          auto load_scales = [&](uint64_t* bar) {
             constexpr uint32_t apc = Cfg<R>::sfa / 512;
             uint8_t* dst = smem + S::sf + s * S::sf_stage;
             const int band_a = T.m0 / kBM;
-            bulk_load(dst, p.sfa + ((int64_t)band_a * p.sfa_s4 + (int64_t)kb * apc) * 512, Cfg<R>::sfa, &full[s]);
+            bulk_load(dst, p.sfa + ((int64_t)band_a * p.sfa_s4 + (int64_t)kb * apc) * 512, Cfg<R>::sfa, bar);
             const int bands_b = (p.N + kBM - 1) / kBM;
 #pragma unroll
             for (int h = 0; h < 2; ++h) {
               const int band = T.n0 / kBM + h;
               const uint8_t* src = (band < bands_b) ? p.sfb + ((int64_t)band * p.sfb_s4 + (int64_t)kb * apc) * 512
                                                     : p.sfb + ((int64_t)kb * apc) * 512;
-              bulk_load(dst + Cfg<R>::sfa + h * Cfg<R>::sfa, src, Cfg<R>::sfa, &full[s]);
+              bulk_load(dst + Cfg<R>::sfa + h * Cfg<R>::sfa, src, Cfg<R>::sfa, bar);
             }
+          };
+          // the scale bytes first, on their own barrier, so the scale warps move them into
+          // TMEM while the stage's A/B chunk is still in flight
+          if constexpr (R != kPerTensor) {
+            mbar_arrive_expect_tx(&sffull[s], Cfg<R>::sfa + Cfg<R>::sfb);
+            load_scales(&sffull[s]);
           }
+          mbar_arrive_expect_tx(&full[s], kAStage + kBStage);
+          tma_load_2d(smem + S::a + s * kAStage, &tma_a, &full[s], kb * kBKB, T.m0);
+          tma_load_2d(smem + S::b + s * kBStage, &tma_b, &full[s], kb * kBKB, T.n0);
         }
       }
       // wind down: every issued stage's copies must land before the CTA exits
@@ -285,6 +303,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       for (uint32_t j = 0; j < inflight; ++j) {
         const uint32_t i2 = it - 1 - j;
         mbar_wait_drain(&full[i2 % kStages], (i2 / kStages) & 1, kWaitLimitNs);
+        if constexpr (R != kPerTensor) mbar_wait_drain(&sffull[i2 % kStages], (i2 / kStages) & 1, kWaitLimitNs);
       }
     }
   } else if (warp == kMmaWarp) {
@@ -304,6 +323,9 @@ __global__ void __launch_bounds__(kThreads, 1)
         for (int kb = 0; kb < KB; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (!mbar_wait(&full[s], ph, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+          if constexpr (R != kPerTensor) {
+            if (!mbar_wait(&sfready[s], ph, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+          }
           tc_fence_after();
           const uint64_t adesc = smem_desc(smem_u32(smem + S::a + s * kAStage), 16, 1024, 2);
           const uint64_t bdesc = smem_desc(smem_u32(smem + S::b + s * kBStage), 16, 1024, 2);
@@ -314,17 +336,6 @@ __global__ void __launch_bounds__(kThreads, 1)
             const uint32_t sf_col = kBN + s * Cfg<R>::sf_cols;  // this stage's scale columns
             const uint32_t sfa_t = tmem + sf_col;
             const uint32_t sfb_t = tmem + sf_col + Cfg<R>::sfa / 128;
-            const uint32_t sfsm = smem_u32(smem + S::sf + s * S::sf_stage);
-            constexpr uint32_t atoms_a = Cfg<R>::sfa / 512;
-#pragma unroll
-            for (uint32_t a = 0; a < atoms_a; ++a) {
-              // A atom a -> 4 columns; B band h atom a -> 4 columns after A's
-              tmem_cp_32x128b_x4(sfa_t + 4 * a, smem_desc(sfsm + 512 * a, 0, 128, 0));
-#pragma unroll
-              for (uint32_t h = 0; h < 2; ++h)
-                tmem_cp_32x128b_x4(sfb_t + 8 * a + 4 * h,
-                                   smem_desc(sfsm + Cfg<R>::sfa + h * Cfg<R>::sfa + 512 * a, 0, 128, 0));
-            }
 #pragma unroll
             for (uint32_t k = 0; k < 4; ++k) {
               const uint32_t acc = (kb > 0 || k > 0);
@@ -346,6 +357,54 @@ __global__ void __launch_bounds__(kThreads, 1)
       // wind down: all MMAs this thread issued complete before TMEM is released
       mma_commit(final_bar);
       mbar_wait_drain(final_bar, 0, kWaitLimitNs);
+    }
+  } else if (warp >= kSfWarp0) {
+    // ------------------------------------------------------------------ scale warps 10-13
+    // Warp q = warp % 4 writes TMEM lanes 32q..32q+31.  A stage's scales sit in shared memory
+    // as 512-byte atoms (128 rows x 4 scale bytes, row r's 4 bytes at (r%32)*16 + (r/32)*4);
+    // the block-scaled MMA reads, for its K step a, 4 columns per atom in which lane l of
+    // every quadrant holds the atom's 16 bytes l*16..l*16+15.  Each lane therefore stores
+    // the same 16 bytes per atom in all four quadrants: A's atoms in 4 columns each, B's two
+    // row bands per atom in 4 columns each, after A's.
+    if constexpr (R != kPerTensor) {
+      constexpr int apc = (int)(Cfg<R>::sfa / 512);   // atoms per stage (MMAs per chunk for NVFP4)
+      const uint32_t t_q = tmem + ((uint32_t)((warp & 3) * 32) << 16);
+      uint32_t it = 0;
+      bool ok = true;
+      for (int t = blockIdx.x; t < total && ok; t += gridDim.x) {
+        for (int kb = 0; kb < KB; ++kb, ++it) {
+          const uint32_t s = it % kStages, ph = (it / kStages) & 1;
+          // the stage's scale bytes have landed; the MMAs that read this scale slot four
+          // chunks ago completed before the producer refilled the stage
+          if (!mbar_wait(&sffull[s], ph, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
+          tc_fence_after();
+          const uint8_t* sm = smem + S::sf + s * S::sf_stage + lane * 16;
+          const uint32_t sf_col = kBN + s * Cfg<R>::sf_cols;
+          uint32_t va[4 * apc], vb[8 * apc];
+#pragma unroll
+          for (int a = 0; a < apc; ++a) {
+            const uint4 x = *reinterpret_cast<const uint4*>(sm + 512 * a);
+            va[4 * a] = x.x, va[4 * a + 1] = x.y, va[4 * a + 2] = x.z, va[4 * a + 3] = x.w;
+#pragma unroll
+            for (int h = 0; h < 2; ++h) {
+              const uint4 y = *reinterpret_cast<const uint4*>(sm + Cfg<R>::sfa + h * Cfg<R>::sfa + 512 * a);
+              vb[8 * a + 4 * h] = y.x, vb[8 * a + 4 * h + 1] = y.y, vb[8 * a + 4 * h + 2] = y.z,
+              vb[8 * a + 4 * h + 3] = y.w;
+            }
+          }
+          if constexpr (apc == 1) {
+            tmem_st_32x32b_x4(t_q + sf_col, va);
+            tmem_st_32x32b_x8(t_q + sf_col + 4, vb);
+          } else {
+            tmem_st_32x32b_x16(t_q + sf_col, va);
+            tmem_st_32x32b_x32(t_q + sf_col + 16, vb);
+          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&sfready[s]);
+        }
+      }
     }
   } else {
     // ------------------------------------------------------------------ epilogue warps 0-7
@@ -963,7 +1022,7 @@ static cudaError_t launch_scaled(const GemmParams& p, const CUtensorMap& a, cons
   const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
   int grid = (int)(tiles < num_sms ? tiles : num_sms);
   if (grid < 1) grid = 1;
-  kern<<<grid, kThreads, smem, s>>>(q, a, b);
+  kern<<<grid, Cfg<R>::threads, smem, s>>>(q, a, b);
   return cudaGetLastError();
 }
 
