@@ -792,10 +792,16 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
         // (wgrad also scales each column: its B scales are per column and chunk)
         auto fma16 = [&](const uint32_t (&r)[16], int h) {
 #pragma unroll
-          for (int i = 0; i < 8; ++i) {
-            float2 pr = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
-            if constexpr (kWg) pr = __fmul2_rn(pr, ld_shared_f2(sbw + h * 16 + 2 * i));
-            acc[h * 8 + i] = __ffma2_rn(pr, s2, acc[h * 8 + i]);
+          for (int i = 0; i < 8; i += 2) {
+            float2 p0 = make_float2(__uint_as_float(r[2 * i]), __uint_as_float(r[2 * i + 1]));
+            float2 p1 = make_float2(__uint_as_float(r[2 * i + 2]), __uint_as_float(r[2 * i + 3]));
+            if constexpr (kWg) {
+              const float4 c = ld_shared_f4(sbw + h * 16 + 2 * i);
+              p0 = __fmul2_rn(p0, make_float2(c.x, c.y));
+              p1 = __fmul2_rn(p1, make_float2(c.z, c.w));
+            }
+            acc[h * 8 + i] = __ffma2_rn(p0, s2, acc[h * 8 + i]);
+            acc[h * 8 + i + 1] = __ffma2_rn(p1, s2, acc[h * 8 + i + 1]);
           }
         };
         const uint32_t tb = t_lane + pb * kBwBN;
