@@ -156,18 +156,29 @@ constexpr int kProducerWarp = 8, kMmaWarp = 9, kSfWarp0 = 10;   // scale warps 1
 constexpr uint32_t kBStage = kBN * kBKB;  // 32 KB
 
 template <int R> struct Cfg;
+// MX / NVFP4 (single accumulator): 16 warps, 128 registers a thread at launch; the two helper
+// warpgroups (warps 8-15: producer, MMA, four scale warps, two idle) drop to 40 and the two
+// epilogue warpgroups rise to 216, enough to hold a thread's 128 accumulator values, so the
+// epilogue takes the whole accumulator out of TMEM, hands it back to the MMA issuer at once
+// and scales, converts and stores while the next tile's MMAs run.
 template <> struct Cfg<kPerTensor> {
   static constexpr uint32_t sfa = 0, sfb = 0, tmem_cols = 512, acc_bufs = 2, epi_cols = 64;
   static constexpr int threads = 320;
+  static constexpr bool split = false;
 };
 template <> struct Cfg<kMx> {
   static constexpr uint32_t sfa = 512, sfb = 1024, tmem_cols = 512, sf_cols = 16, acc_bufs = 1, epi_cols = 32;
-  static constexpr int threads = 448;
+  static constexpr int threads = 512;
+  static constexpr bool split = true;
 };
 template <> struct Cfg<kNvfp4> {
   static constexpr uint32_t sfa = 2048, sfb = 4096, tmem_cols = 512, sf_cols = 64, acc_bufs = 1, epi_cols = 16;
-  static constexpr int threads = 448;
+  static constexpr int threads = 512;
+  static constexpr bool split = true;
 };
+constexpr int kSplitRegsLaunch = 128, kSplitRegsEpi = 216, kSplitRegsHelper = 40;
+static_assert(2 * 128 * kSplitRegsEpi + 2 * 128 * kSplitRegsHelper <= 512 * kSplitRegsLaunch,
+              "register shares exceed the launch pool");
 
 template <int R>
 struct Smem {
@@ -258,6 +269,9 @@ __global__ void __launch_bounds__(Cfg<R>::threads, 1)
   const uint32_t tmem = *tmem_slot;
   const int total = p.tiles_m * p.tiles_n;
 
+  if (warp >= kEpiWarps) {
+  // helper warpgroups: warps 8-11 and 12-15 (MX / NVFP4) give registers to the epilogue
+  if constexpr (Cfg<R>::split) reg_dealloc<kSplitRegsHelper>();
   if (warp == kProducerWarp) {
     // ------------------------------------------------------------------ TMA producer
     if (lane == 0) {
@@ -358,7 +372,7 @@ __global__ void __launch_bounds__(Cfg<R>::threads, 1)
       mma_commit(final_bar);
       mbar_wait_drain(final_bar, 0, kWaitLimitNs);
     }
-  } else if (warp >= kSfWarp0) {
+  } else if (warp < kSfWarp0 + 4) {
     // ------------------------------------------------------------------ scale warps 10-13
     // Warp q = warp % 4 writes TMEM lanes 32q..32q+31.  A stage's scales sit in shared memory
     // as 512-byte atoms (128 rows x 4 scale bytes, row r's 4 bytes at (r%32)*16 + (r/32)*4);
@@ -380,24 +394,33 @@ __global__ void __launch_bounds__(Cfg<R>::threads, 1)
           tc_fence_after();
           const uint8_t* sm = smem + S::sf + s * S::sf_stage + lane * 16;
           const uint32_t sf_col = kBN + s * Cfg<R>::sf_cols;
-          uint32_t va[4 * apc], vb[8 * apc];
-#pragma unroll
-          for (int a = 0; a < apc; ++a) {
-            const uint4 x = *reinterpret_cast<const uint4*>(sm + 512 * a);
-            va[4 * a] = x.x, va[4 * a + 1] = x.y, va[4 * a + 2] = x.z, va[4 * a + 3] = x.w;
-#pragma unroll
-            for (int h = 0; h < 2; ++h) {
-              const uint4 y = *reinterpret_cast<const uint4*>(sm + Cfg<R>::sfa + h * Cfg<R>::sfa + 512 * a);
-              vb[8 * a + 4 * h] = y.x, vb[8 * a + 4 * h + 1] = y.y, vb[8 * a + 4 * h + 2] = y.z,
-              vb[8 * a + 4 * h + 3] = y.w;
-            }
-          }
+          auto ld16 = [&](uint32_t off, uint32_t* v) {   // 16 bytes of one atom row
+            const uint4 x = *reinterpret_cast<const uint4*>(sm + off);
+            v[0] = x.x, v[1] = x.y, v[2] = x.z, v[3] = x.w;
+          };
           if constexpr (apc == 1) {
+            uint32_t va[4], vb[8];
+            ld16(0, va);
+            ld16(Cfg<R>::sfa, vb);
+            ld16(2 * Cfg<R>::sfa, vb + 4);
             tmem_st_32x32b_x4(t_q + sf_col, va);
             tmem_st_32x32b_x8(t_q + sf_col + 4, vb);
           } else {
-            tmem_st_32x32b_x16(t_q + sf_col, va);
-            tmem_st_32x32b_x32(t_q + sf_col + 16, vb);
+            // 16 columns per store (the warp has 40 registers): A's four atoms, then B's
+            // atoms 0-1 and 2-3 with their two row bands each
+            uint32_t v[16];
+#pragma unroll
+            for (int a = 0; a < 4; ++a) ld16(512 * a, v + 4 * a);
+            tmem_st_32x32b_x16(t_q + sf_col, v);
+#pragma unroll
+            for (int g = 0; g < 2; ++g) {
+              uint32_t w[16];
+#pragma unroll
+              for (int a = 0; a < 2; ++a)
+#pragma unroll
+                for (int h = 0; h < 2; ++h) ld16(Cfg<R>::sfa + h * Cfg<R>::sfa + 512 * (2 * g + a), w + 8 * a + 4 * h);
+              tmem_st_32x32b_x16(t_q + sf_col + 16 + 16 * g, w);
+            }
           }
           tmem_st_wait();
           tc_fence_before();
@@ -406,8 +429,10 @@ __global__ void __launch_bounds__(Cfg<R>::threads, 1)
         }
       }
     }
+  }  // warps 14-15 (MX / NVFP4) only complete the second helper warpgroup
   } else {
     // ------------------------------------------------------------------ epilogue warps 0-7
+    if constexpr (Cfg<R>::split) reg_alloc<kSplitRegsEpi>();
     constexpr int EC = (int)Cfg<R>::epi_cols;
     const int q = warp & 3, wg = warp >> 2;
     const uint32_t t_lane = tmem + ((uint32_t)(q * 32) << 16) + (uint32_t)(wg * 128);
@@ -421,22 +446,42 @@ __global__ void __launch_bounds__(Cfg<R>::threads, 1)
       const int ncol0 = T.n0 + wg * 128;
       if (!mbar_wait(&accfull[ab], (tiles_done / kAcc) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); break; }
       tc_fence_after();
-#pragma unroll 1
-      for (int c = 0; c < 128 / EC; ++c) {
-        float v[EC];
+      if constexpr (Cfg<R>::split) {
+        // the thread's 128 values out of TMEM at once, the accumulator back to the MMA
+        // issuer, then scale, convert and store from registers
+        uint32_t r[8][16];
 #pragma unroll
-        for (int h = 0; h < EC / 16; ++h) {
-          uint32_t r[16];
-          tmem_ld_32x32b_x16(t_lane + ab * (uint32_t)kBN + c * EC + h * 16, r);
-          tmem_ld_wait(r);
+        for (int h = 0; h < 8; ++h) tmem_ld_32x32b_x16(t_lane + ab * (uint32_t)kBN + h * 16, r[h]);
 #pragma unroll
-          for (int i = 0; i < 16; ++i) v[h * 16 + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+        for (int h = 0; h < 8; ++h) tmem_ld_wait(r[h]);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed(&accempty[ab]);
+#pragma unroll
+        for (int c = 0; c < 128 / EC; ++c) {
+          float v[EC];
+#pragma unroll
+          for (int i = 0; i < EC; ++i) v[i] = __fmul_rn(__uint_as_float(r[(c * EC + i) / 16][(c * EC + i) % 16]), alpha);
+          stage_store_rows<EC>(stg, v, p, T.m0 + q * 32, T.mend, ncol0 + c * EC, lane);
         }
-        stage_store_rows<EC>(stg, v, p, T.m0 + q * 32, T.mend, ncol0 + c * EC, lane);
+      } else {
+#pragma unroll 1
+        for (int c = 0; c < 128 / EC; ++c) {
+          float v[EC];
+#pragma unroll
+          for (int h = 0; h < EC / 16; ++h) {
+            uint32_t r[16];
+            tmem_ld_32x32b_x16(t_lane + ab * (uint32_t)kBN + c * EC + h * 16, r);
+            tmem_ld_wait(r);
+#pragma unroll
+            for (int i = 0; i < 16; ++i) v[h * 16 + i] = __fmul_rn(__uint_as_float(r[i]), alpha);
+          }
+          stage_store_rows<EC>(stg, v, p, T.m0 + q * 32, T.mend, ncol0 + c * EC, lane);
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive_relaxed(&accempty[ab]);
       }
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive_relaxed(&accempty[ab]);
     }
   }
 
@@ -1019,6 +1064,15 @@ template <int R>
 static cudaError_t launch_scaled(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b, int num_sms,
                                  cudaStream_t s) {
   auto kern = gemm_scaled_kernel<R>;
+  // The register reallocation of MX / NVFP4 adds up to exactly the launch pool at 128
+  // registers per thread; with any other count an increase could wait forever, so refuse.
+  if constexpr (Cfg<R>::split) {
+    static const int regs = [] {
+      cudaFuncAttributes fa{};
+      return cudaFuncGetAttributes(&fa, gemm_scaled_kernel<R>) == cudaSuccess ? fa.numRegs : -1;
+    }();
+    if (regs != kSplitRegsLaunch) return cudaErrorInvalidConfiguration;
+  }
   const int smem = (int)Smem<R>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
