@@ -563,7 +563,8 @@ struct BwSmem {
   // epilogue staging per promotion warp: 32 rows x epi_cols BF16 (wgrad: half the width)
   static constexpr int epi_cols = 32;
   static constexpr uint32_t stage_c = 32 * epi_cols * 2;
-  static constexpr uint32_t cst = ring + kBwSb * slot_bytes;
+  // staging buffers 1024-byte aligned: the TMA store's 64-byte swizzle follows address bits
+  static constexpr uint32_t cst = ((ring + kBwSb * slot_bytes + 1023) / 1024) * 1024;
   static constexpr uint32_t bars = cst + C::EpiWarps * stage_c;
   static constexpr uint32_t n_bars = kBwGo + stages + 2 * kBwSb + 1 + C::EpiWarps / 2;
   static_assert(kBwGo % stages == 0 && kBwGo % 2 == 0, "go slots must cycle with the stages and TMEM buffers");
@@ -630,7 +631,8 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 template <int L, bool GROUPED, int EPI>
 __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
-                          const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb) {
+                          const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb,
+                          const __grid_constant__ CUtensorMap tma_c) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
@@ -896,13 +898,31 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
       uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
       if constexpr (!ACC32) {
+        // plain BF16 (not grouped): the staged 32 x 32 box goes out by one TMA store and the
+        // warp moves on to the next tile while the copy engine writes it (the swizzled staging
+        // layout is the tensor map's 64-byte swizzle); the box is reused only after the store
+        // has read it.  Grouped and quantizing epilogues store the rows themselves.
+        constexpr bool kTmaStore = (EPI == kEpiBf16) && !GROUPED;
 #pragma unroll
         for (int h = 0; h < 64 / EC; ++h) {
+          if constexpr (kTmaStore) {
+            if (lane == 0) bulk_wait_read();
+            __syncwarp();
+          }
 #pragma unroll
           for (int c = 0; c < CPR; ++c) {
             const float2* a4 = acc + h * (EC / 2) + c * 4;
             stg[lane * CPR + (c ^ swz(lane))] = make_uint4(pack_bf16(a4[0].x, a4[0].y), pack_bf16(a4[1].x, a4[1].y),
                                                            pack_bf16(a4[2].x, a4[2].y), pack_bf16(a4[3].x, a4[3].y));
+          }
+          if constexpr (kTmaStore) {
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_store_2d(&tma_c, stg, ncol0 + h * EC, T.m0 + q * 32);
+              bulk_commit();
+            }
+            continue;
           }
           __syncwarp();
 #pragma unroll
@@ -982,6 +1002,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     }
   }
 
+  if (EPI == kEpiBf16 && !GROUPED && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
   tc_fence_before();
   __syncwarp();     // role loops ran on lane 0 only: reconverge before the aligned barrier
   cluster_sync();   // the leader's MMAs into both TMEMs are complete before either frees
@@ -1016,7 +1037,7 @@ static void raster(GemmParams& q, int row_tiles, int tile_m, int tile_n) {
 
 template <int L, bool G, int EPI = kEpiBf16>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
-                                    const CUtensorMap& sb, int num_sms, cudaStream_t s) {
+                                    const CUtensorMap& sb, const CUtensorMap& c, int num_sms, cudaStream_t s) {
   auto kern = gemm_blockwise_kernel<L, G, EPI>;
   using C = BwCfg<L>;
   constexpr int kBwBN = C::BN;
@@ -1057,7 +1078,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   if (clusters > tiles) clusters = (int)tiles;
   if (clusters < 1) clusters = 1;
   cfg.gridDim = dim3(2 * clusters);
-  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb);
+  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb, c);
 }
 
 template <int R>
@@ -1106,23 +1127,23 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
-                        const CUtensorMap& tma_sb, int num_sms, cudaStream_t s) {
+                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, int num_sms, cudaStream_t s) {
   if (p.recipe == kBlockwise) {
     if (p.c32 != nullptr) {   // FP32 accumulate epilogue: its own instantiations
-      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
     }
     if (p.q_out != nullptr) {  // BF16 output plus its fused 1x128 quantization
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
     }
-    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, num_sms, s);
-    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, num_sms, s);
-    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, num_sms, s);
-    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, num_sms, s);
+    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
   }
   if (p.recipe == kMx) return launch_scaled<kMx>(p, tma_a, tma_b, num_sms, s);
   if (p.recipe == kPerTensor) return launch_scaled<kPerTensor>(p, tma_a, tma_b, num_sms, s);
