@@ -555,7 +555,7 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   }
   // the blockwise plain BF16 epilogue stores its staged 32 x 32 boxes by TMA
   CUtensorMap mc = ma;
-  if (a->recipe == FP8Q_BLOCKWISE && !acc32 && !qout && !grouped && a->M > 0 && a->N > 0) {
+  if (a->recipe == FP8Q_BLOCKWISE && !acc32 && !qout && a->M > 0 && a->N > 0) {
     if (!make_map(&mc, a->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->N, a->M, a->ldc * 2, 32, 32,
                   CU_TENSOR_MAP_SWIZZLE_64B))
       return FP8Q_ERR_CUDA;

@@ -898,14 +898,15 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
       uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
       if constexpr (!ACC32) {
-        // plain BF16 (not grouped): the staged 32 x 32 box goes out by one TMA store and the
-        // warp moves on to the next tile while the copy engine writes it (the swizzled staging
-        // layout is the tensor map's 64-byte swizzle); the box is reused only after the store
-        // has read it.  Grouped and quantizing epilogues store the rows themselves.
-        constexpr bool kTmaStore = (EPI == kEpiBf16) && !GROUPED;
+        // plain BF16: the staged 32 x 32 box goes out by one TMA store and the warp moves on
+        // to the next tile while the copy engine writes it (the swizzled staging layout is the
+        // tensor map's 64-byte swizzle); the box is reused only after the store has read it.
+        // A grouped GEMM's box that would reach past its expert's rows, and the quantizing
+        // epilogue, store the rows themselves.
+        const bool tma_box = (EPI == kEpiBf16) && (!GROUPED || T.m0 + q * 32 + 32 <= T.mend);
 #pragma unroll
         for (int h = 0; h < 64 / EC; ++h) {
-          if constexpr (kTmaStore) {
+          if (EPI == kEpiBf16) {
             if (lane == 0) bulk_wait_read();
             __syncwarp();
           }
@@ -915,7 +916,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
             stg[lane * CPR + (c ^ swz(lane))] = make_uint4(pack_bf16(a4[0].x, a4[0].y), pack_bf16(a4[1].x, a4[1].y),
                                                            pack_bf16(a4[2].x, a4[2].y), pack_bf16(a4[3].x, a4[3].y));
           }
-          if constexpr (kTmaStore) {
+          if (tma_box) {
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
@@ -1002,7 +1003,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     }
   }
 
-  if (EPI == kEpiBf16 && !GROUPED && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
+  if (EPI == kEpiBf16 && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
   tc_fence_before();
   __syncwarp();     // role loops ran on lane 0 only: reconverge before the aligned barrier
   cluster_sync();   // the leader's MMAs into both TMEMs are complete before either frees

@@ -115,7 +115,7 @@ struct GemmParams {
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
 // tma_c: BF16 C (N inner, M outer, 32 x 32 boxes, 64-byte swizzle), used by the blockwise
-// kernel's plain BF16 epilogue when the GEMM is not grouped.
+// kernel's plain BF16 epilogue.
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, const CUtensorMap& tma_c, int num_sms, cudaStream_t s);
 
