@@ -553,14 +553,18 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   } else {
     msb = ma;
   }
-  // the blockwise plain BF16 epilogue stores its staged 32 x 32 boxes by TMA
-  CUtensorMap mc = ma;
-  if (a->recipe == FP8Q_BLOCKWISE && !acc32 && !qout && a->M > 0 && a->N > 0) {
+  // the blockwise BF16 epilogues store their staged 32 x 32 boxes (and the fused
+  // quantization its 32 x 64 code boxes) by TMA
+  CUtensorMap mc = ma, mq = ma;
+  if (a->recipe == FP8Q_BLOCKWISE && !acc32 && a->M > 0 && a->N > 0) {
     if (!make_map(&mc, a->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->N, a->M, a->ldc * 2, 32, 32,
                   CU_TENSOR_MAP_SWIZZLE_64B))
       return FP8Q_ERR_CUDA;
+    if (qout && !make_map(&mq, a->q_out, CU_TENSOR_MAP_DATA_TYPE_UINT8, a->N, a->M, a->ld_q_out, 64, 32,
+                          CU_TENSOR_MAP_SWIZZLE_64B))
+      return FP8Q_ERR_CUDA;
   }
-  return from_cuda(launch_gemm(p, ma, mb, msb, mc, d->num_sms, s));
+  return from_cuda(launch_gemm(p, ma, mb, msb, mc, mq, d->num_sms, s));
 }
 
 }  // extern "C"

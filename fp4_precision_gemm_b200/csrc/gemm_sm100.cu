@@ -632,7 +632,7 @@ template <int L, bool GROUPED, int EPI>
 __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb,
-                          const __grid_constant__ CUtensorMap tma_c) {
+                          const __grid_constant__ CUtensorMap tma_c, const __grid_constant__ CUtensorMap tma_q) {
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
@@ -898,18 +898,15 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
       uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
       if constexpr (!ACC32) {
-        // plain BF16: the staged 32 x 32 box goes out by one TMA store and the warp moves on
-        // to the next tile while the copy engine writes it (the swizzled staging layout is the
-        // tensor map's 64-byte swizzle); the box is reused only after the store has read it.
-        // A grouped GEMM's box that would reach past its expert's rows, and the quantizing
-        // epilogue, store the rows themselves.
-        const bool tma_box = (EPI == kEpiBf16) && (!GROUPED || T.m0 + q * 32 + 32 <= T.mend);
+        // BF16: the staged 32 x 32 box goes out by one TMA store and the warp moves on to the
+        // next tile while the copy engine writes it (the swizzled staging layout is the tensor
+        // map's 64-byte swizzle); the box is reused only after the store has read it.  A
+        // grouped GEMM's box that would reach past its expert's rows is stored by the warp.
+        const bool tma_box = !GROUPED || T.m0 + q * 32 + 32 <= T.mend;
 #pragma unroll
         for (int h = 0; h < 64 / EC; ++h) {
-          if (EPI == kEpiBf16) {
-            if (lane == 0) bulk_wait_read();
-            __syncwarp();
-          }
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < CPR; ++c) {
             const float2* a4 = acc + h * (EC / 2) + c * 4;
@@ -976,6 +973,8 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
         am = fmaxf(am, xch[(warp ^ 4) * 32 + lane]);
         const float sf = e4m3_sf(am);
         const float2 s2 = make_float2(sf, sf);
+        if (lane == 0) bulk_wait_read();     // the BF16 box store has read the buffer
+        __syncwarp();
 #pragma unroll
         for (int c = 0; c < 4; ++c) {        // 16 codes (16 bytes) per chunk of the lane's row
           uint32_t w[4];
@@ -987,15 +986,13 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
           }
           stg[lane * 4 + (c ^ swz(lane))] = make_uint4(w[0], w[1], w[2], w[3]);
         }
+        // the 32 x 64 code box (same 64-byte swizzle) goes out by TMA store as well
+        fence_proxy_async();
         __syncwarp();
-#pragma unroll
-        for (int i = 0; i < 4; ++i) {        // 8 rows x 64 bytes per instruction
-          const int r = i * 8 + lane / 4, c = lane % 4;
-          const uint4 v = stg[r * 4 + (c ^ swz(r))];
-          const int mr = T.m0 + q * 32 + r, n = ncol0 + c * 16;
-          if (mr < T.mend && n < p.N) *reinterpret_cast<uint4*>(p.q_out + (int64_t)mr * p.ld_q_out + n) = v;
+        if (lane == 0) {
+          tma_store_2d(&tma_q, stg, ncol0, T.m0 + q * 32);
+          bulk_commit();
         }
-        __syncwarp();
         const int mrow = T.m0 + q * 32 + lane;
         if ((cgp & 1) == 0 && mrow < T.mend && ncol0 < p.N)
           p.s_out[(int64_t)(ncol0 >> 7) * p.ld_s_out + mrow] = __frcp_rn(sf);
@@ -1003,7 +1000,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     }
   }
 
-  if (EPI == kEpiBf16 && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
+  if (!ACC32 && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
   tc_fence_before();
   __syncwarp();     // role loops ran on lane 0 only: reconverge before the aligned barrier
   cluster_sync();   // the leader's MMAs into both TMEMs are complete before either frees
@@ -1038,7 +1035,8 @@ static void raster(GemmParams& q, int row_tiles, int tile_m, int tile_n) {
 
 template <int L, bool G, int EPI = kEpiBf16>
 static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
-                                    const CUtensorMap& sb, const CUtensorMap& c, int num_sms, cudaStream_t s) {
+                                    const CUtensorMap& sb, const CUtensorMap& c, const CUtensorMap& qm, int num_sms,
+                                    cudaStream_t s) {
   auto kern = gemm_blockwise_kernel<L, G, EPI>;
   using C = BwCfg<L>;
   constexpr int kBwBN = C::BN;
@@ -1079,7 +1077,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   if (clusters > tiles) clusters = (int)tiles;
   if (clusters < 1) clusters = 1;
   cfg.gridDim = dim3(2 * clusters);
-  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb, c);
+  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb, c, qm);
 }
 
 template <int R>
@@ -1128,23 +1126,24 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
-                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, int num_sms, cudaStream_t s) {
+                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q, int num_sms,
+                        cudaStream_t s) {
   if (p.recipe == kBlockwise) {
     if (p.c32 != nullptr) {   // FP32 accumulate epilogue: its own instantiations
-      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
     }
     if (p.q_out != nullptr) {  // BF16 output plus its fused 1x128 quantization
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
     }
-    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
-    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, num_sms, s);
+    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
   }
   if (p.recipe == kMx) return launch_scaled<kMx>(p, tma_a, tma_b, num_sms, s);
   if (p.recipe == kPerTensor) return launch_scaled<kPerTensor>(p, tma_a, tma_b, num_sms, s);

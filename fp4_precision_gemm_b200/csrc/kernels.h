@@ -114,9 +114,11 @@ struct GemmParams {
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
-// tma_c: BF16 C (N inner, M outer, 32 x 32 boxes, 64-byte swizzle), used by the blockwise
-// kernel's plain BF16 epilogue.
+// tma_c: BF16 C (N inner, M outer, 32 x 32 boxes, 64-byte swizzle) and tma_q: the fused
+// quantization's E4M3 codes (N inner, M outer, 64 x 32 boxes, 64-byte swizzle), stored by the
+// blockwise kernel's BF16 epilogues.
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
-                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, int num_sms, cudaStream_t s);
+                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q, int num_sms,
+                        cudaStream_t s);
 
 }  // namespace fp8q
