@@ -553,10 +553,15 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   } else {
     msb = ma;
   }
-  // the blockwise BF16 epilogues store their staged 32 x 32 boxes (and the fused
-  // quantization its 32 x 64 code boxes) by TMA
+  // the blockwise epilogues send their staged boxes by TMA: BF16 32 x 32 boxes (and the fused
+  // quantization's 32 x 64 code boxes) stored, FP32 boxes added
   CUtensorMap mc = ma, mq = ma;
-  if (a->recipe == FP8Q_BLOCKWISE && !acc32 && a->M > 0 && a->N > 0) {
+  if (a->recipe == FP8Q_BLOCKWISE && acc32 && a->M > 0 && a->N > 0) {
+    // FP32 accumulation: 32 x 16 FP32 boxes added into C by TMA reduction
+    if (!make_map(&mc, a->c, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, a->N, a->M, a->ldc * 4, 16, 32,
+                  CU_TENSOR_MAP_SWIZZLE_64B))
+      return FP8Q_ERR_CUDA;
+  } else if (a->recipe == FP8Q_BLOCKWISE && a->M > 0 && a->N > 0) {
     if (!make_map(&mc, a->c, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, a->N, a->M, a->ldc * 2, 32, 32,
                   CU_TENSOR_MAP_SWIZZLE_64B))
       return FP8Q_ERR_CUDA;

@@ -934,13 +934,28 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
         }
       } else {
         constexpr int EC32 = EC / 2;   // FP32 columns per pass (same bytes per row)
+        // the staged 32 x 16 FP32 box is added into C by one TMA reduction (C + S rounded to
+        // FP32 once per element, as below); a grouped box reaching past its expert's rows is
+        // added by the warp
+        const bool tma_box = !GROUPED || T.m0 + q * 32 + 32 <= T.mend;
 #pragma unroll
         for (int h = 0; h < 64 / EC32; ++h) {
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
 #pragma unroll
           for (int c = 0; c < CPR; ++c) {
             const float2* a2 = acc + h * (EC32 / 2) + c * 2;
             stg[lane * CPR + (c ^ swz(lane))] = make_uint4(__float_as_uint(a2[0].x), __float_as_uint(a2[0].y),
                                                            __float_as_uint(a2[1].x), __float_as_uint(a2[1].y));
+          }
+          if (tma_box) {
+            fence_proxy_async();
+            __syncwarp();
+            if (lane == 0) {
+              tma_reduce_add_2d(&tma_c, stg, ncol0 + h * EC32, T.m0 + q * 32);
+              bulk_commit();
+            }
+            continue;
           }
           __syncwarp();
 #pragma unroll
@@ -1000,7 +1015,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     }
   }
 
-  if (!ACC32 && warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // TMA stores done
+  if (warp < kBwEpiWarps && lane == 0) bulk_wait_all();   // the epilogue's TMA stores are done
   tc_fence_before();
   __syncwarp();     // role loops ran on lane 0 only: reconverge before the aligned barrier
   cluster_sync();   // the leader's MMAs into both TMEMs are complete before either frees

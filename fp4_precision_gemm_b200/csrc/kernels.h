@@ -114,9 +114,9 @@ struct GemmParams {
 
 cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream_t s);
 
-// tma_c: BF16 C (N inner, M outer, 32 x 32 boxes, 64-byte swizzle) and tma_q: the fused
-// quantization's E4M3 codes (N inner, M outer, 64 x 32 boxes, 64-byte swizzle), stored by the
-// blockwise kernel's BF16 epilogues.
+// tma_c: C for the blockwise kernel's epilogues, N inner, M outer, 64-byte swizzle: BF16 with
+// 32 x 32 boxes (stored), or FP32 with 16 x 32 boxes (added, FP32 accumulation); tma_q: the
+// fused quantization's E4M3 codes (64 x 32 boxes, stored).
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q, int num_sms,
                         cudaStream_t s);
