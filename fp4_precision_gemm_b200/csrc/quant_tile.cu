@@ -183,6 +183,10 @@ __device__ __forceinline__ void tile_quant_tile(const TileQuantParams& P, int64_
       const int pr = cs & 7;
       const uint32_t w = pr < 2 ? rp[0] : pr < 4 ? rp[1] : pr < 6 ? rp[2] : rp[3];
       sf_own = e4m3_sf(bf16_bits_to_float((pr & 1) ? (w >> 16) : (w & 0xFFFFu)));
+      // lane cs < 8 of the row group also writes row cs's decode scale (one reciprocal per
+      // lane instead of one per row with a single lane active)
+      const int64_t row = r0 + rb * 8 + cs;
+      if (cs < 8 && row < P.rows) ((float*)SR)[(c0 >> 7) * P.ld_s_row + row] = __frcp_rn(sf_own);
     }
 #pragma unroll
     for (int p = 0; p < 8; ++p) {
@@ -208,8 +212,6 @@ __device__ __forceinline__ void tile_quant_tile(const TileQuantParams& P, int64_
         }
         *(uint2*)(QR + row * P.cols + col) = make_uint2(c[0] | (c[1] << 16), c[2] | (c[3] << 16));
       }
-      if (MODE == kTile1x128 && cs == 0 && row < P.rows)
-        ((float*)SR)[(c0 >> 7) * P.ld_s_row + row] = __frcp_rn(sf);
       if (MODE == kTileMX && (cs & 3) == 0) {
         const int64_t kc = (col >> 5);
         uint8_t* dst = SR;
