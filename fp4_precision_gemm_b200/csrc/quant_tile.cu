@@ -275,7 +275,7 @@ __global__ void __launch_bounds__(256, ROWONLY ? 3 : 4) tile_quant_multi_kernel(
   const int64_t b = blockIdx.x;
   int i = 0;
   while (i + 1 < M.n && b >= M.tile_begin[i + 1]) ++i;
-  const TileQuantParams& P = M.item[i];
+  const TileQuantParams P = M.item[i];   // by value: registers, not indexed parameter loads
   const int64_t tile = b - M.tile_begin[i];
   switch (M.kind[i]) {
     case kMulti1x128Col: tile_quant_tile<kTile1x128, false, true>(P, tile, sm); break;
