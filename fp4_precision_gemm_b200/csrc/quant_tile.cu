@@ -130,18 +130,15 @@ __device__ __forceinline__ void tile_quant_tile(const TileQuantParams& P, int64_
     }
     __syncthreads();
     if (MODE == kTile1x128) {
-      if (t < 64) {
-        uint32_t m = red[0][t];
+      if (t < 128) {   // one column per thread: word t/2 holds columns cc and cc + 1
+        const int wd = t >> 1, h = t & 1;
+        uint32_t m = red[0][wd];
 #pragma unroll
-        for (int w = 1; w < 8; ++w) m = max2(m, red[w][t]);
-        const int cc = (t >> 2) * 8 + (t & 3) * 2;
-#pragma unroll
-        for (int h = 0; h < 2; ++h) {
-          const float sf = e4m3_sf(bf16_bits_to_float(h ? (m >> 16) : (m & 0xFFFFu)));
-          colsf[cc + h] = sf;
-          if (c0 + cc + h < P.cols)
-            ((float*)SC)[(r0 >> 7) * P.ld_s_col + c0 + cc + h] = __frcp_rn(sf);
-        }
+        for (int w = 1; w < 8; ++w) m = max2(m, red[w][wd]);
+        const int cc = (wd >> 2) * 8 + (wd & 3) * 2 + h;
+        const float sf = e4m3_sf(bf16_bits_to_float(h ? (m >> 16) : (m & 0xFFFFu)));
+        colsf[cc] = sf;
+        if (c0 + cc < P.cols) ((float*)SC)[(r0 >> 7) * P.ld_s_col + c0 + cc] = __frcp_rn(sf);
       }
       __syncthreads();
     } else {  // MX: 32-row block b = warp / 2 spans warps 2b and 2b+1
