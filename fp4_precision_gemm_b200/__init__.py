@@ -24,8 +24,8 @@ __all__ = [
     "fp4q_rht16_quantize_sr", "fp4q_quantize_2d16", "FP8Q_E4M3", "FP8Q_E5M2", "fp8q_gemm_blockscaled", "fp8q_sf_bytes",
     "fp8q_get_device_status", "fp8q_selftest_bounded_wait", "fp8q_status_string", "fp8q_version", "GemmArgs",
     "quantize_1x128", "quantize_128x128", "quantize_128x128_grouped", "quantize_tensor_delayed", "quantize_mx32", "quantize_tensor", "rht16_quantize_sr",
-    "quantize_nvfp4_2d16", "gemm", "device_status", "EXPORTED_SYMBOLS",
-    "fp8q_quantize_multi", "QuantItem", "FP8Q_ITEM_1X128", "FP8Q_ITEM_128X128", "FP8Q_MAX_QUANT_ITEMS",
+    "quantize_nvfp4_2d16", "gemm", "gemm_workspace_bytes", "device_status", "EXPORTED_SYMBOLS",
+    "fp8q_quantize_multi", "fp8q_gemm_workspace_bytes", "QuantItem", "FP8Q_ITEM_1X128", "FP8Q_ITEM_128X128", "FP8Q_MAX_QUANT_ITEMS",
     "quantize_multi",
 ]
 
@@ -45,7 +45,7 @@ EXPORTED_SYMBOLS = [
     "fp4q_rht16_quantize_sr", "fp8q_gemm_blockscaled", "fp8q_sf_bytes", "fp8q_get_device_status",
     "fp8q_release_scratch", "fp8q_status_string", "fp8q_version", "fp8q_quantize_tensor_noalloc",
     "fp8q_selftest_bounded_wait", "fp8q_quantize_128x128_grouped", "fp8q_quantize_tensor_delayed",
-    "fp4q_quantize_2d16", "fp8q_quantize_multi",
+    "fp4q_quantize_2d16", "fp8q_quantize_multi", "fp8q_gemm_workspace_bytes",
 ]
 
 library_path = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfp8q.so")
@@ -82,6 +82,7 @@ class GemmArgs(ctypes.Structure):
         ("a_format", ctypes.c_int32), ("b_format", ctypes.c_int32),
         ("q_out", ctypes.c_void_p), ("s_out", ctypes.c_void_p),
         ("ld_q_out", ctypes.c_int64), ("ld_s_out", ctypes.c_int64),
+        ("workspace", ctypes.c_void_p), ("workspace_bytes", ctypes.c_int64),
     ]
 
 
@@ -109,6 +110,8 @@ def lib():
                                              _vp, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp4q_quantize_2d16.argtypes = [_vp, _i64, _i64, _i64, _vp, _vp, _vp, _vp, _vp, _int, _vp]
         L.fp8q_gemm_blockscaled.argtypes = [ctypes.POINTER(GemmArgs), _vp]
+        L.fp8q_gemm_workspace_bytes.argtypes = [ctypes.POINTER(GemmArgs)]
+        L.fp8q_gemm_workspace_bytes.restype = ctypes.c_size_t
         L.fp8q_quantize_multi.argtypes = [ctypes.POINTER(QuantItem), ctypes.c_int32, _vp]
         L.fp8q_sf_bytes.argtypes = [_int, _i64, _i64, _int]
         L.fp8q_sf_bytes.restype = ctypes.c_size_t
@@ -203,6 +206,10 @@ def fp4q_quantize_2d16(x, rows, cols, ld_x, q_row, sf_row, q_col, sf_col, g_dec,
 
 def fp8q_gemm_blockscaled(args, stream):
     return lib().fp8q_gemm_blockscaled(ctypes.byref(args), stream)
+
+
+def fp8q_gemm_workspace_bytes(args):
+    return lib().fp8q_gemm_workspace_bytes(ctypes.byref(args))
 
 
 def fp8q_sf_bytes(recipe, outer, inner, layout):
@@ -420,14 +427,9 @@ def quantize_nvfp4_2d16(w, rowwise=True, colwise=True, sf_layout=FP8Q_SF_MMA_TIL
     return out
 
 
-def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
-         a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False,
-         a_format=0, b_format=0, q_out=None, s_out=None, stream=None):
-    """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
-    Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16.
-    accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T.
-    q_out (M, N) uint8 and s_out (N/128, M) float32 (BLOCKWISE): also receive the 1x128
-    rowwise quantization of the BF16 C, made in the GEMM's epilogue."""
+def _gemm_args(a, b, recipe, layout, a_scale, b_scale, ld_sa, ld_sb, a_global, b_global, K, m_offsets, out,
+               accumulate_fp32, a_format, b_format, q_out, s_out):
+    """The C ABI's argument block for gemm() (and the output tensor it writes)."""
     M = a.shape[0]
     grouped = m_offsets is not None
     N = b.shape[1] if grouped else b.shape[0]
@@ -457,8 +459,46 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
         args.s_out = s_out.data_ptr() if s_out is not None else None
         args.ld_q_out = q_out.stride(0) if q_out is not None else 0
         args.ld_s_out = s_out.stride(0) if s_out is not None else 0
+    return args, c
+
+
+def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=None, ld_sa=None, ld_sb=None,
+         a_global=None, b_global=None, K=None, m_offsets=None, out=None, accumulate_fp32=False,
+         a_format=0, b_format=0, q_out=None, s_out=None, stream=None, split_tail=True):
+    """C = A . B^T (BF16).  a: (M, K or K/2) uint8 codes, b: (N, ...) or (G, N, ...) uint8.
+    Scales as the C ABI describes for the recipe.  Returns C (M, N) bf16.
+    accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T.
+    q_out (M, N) uint8 and s_out (N/128, M) float32 (BLOCKWISE): also receive the 1x128
+    rowwise quantization of the BF16 C, made in the GEMM's epilogue.
+    split_tail (BLOCKWISE, BF16 output): give the call the workspace it asks for
+    (fp8q_gemm_workspace_bytes), taken from torch's caching allocator on the call's stream, so
+    that a mostly idle last wave is split into K ranges."""
+    args, c = _gemm_args(a, b, recipe, layout, a_scale, b_scale, ld_sa, ld_sb, a_global, b_global, K, m_offsets,
+                         out, accumulate_fp32, a_format, b_format, q_out, s_out)
+    ws = None
+    if split_tail and recipe == FP8Q_BLOCKWISE:
+        nbytes = fp8q_gemm_workspace_bytes(args)
+        if nbytes > 0:
+            ws = torch.empty(nbytes, dtype=torch.uint8, device=a.device)
+            if stream is not None:
+                ws.record_stream(stream)
+            args.workspace, args.workspace_bytes = ws.data_ptr(), nbytes
     _check(fp8q_gemm_blockscaled(args, _stream(stream)), "fp8q_gemm_blockscaled")
     return c
+
+
+def gemm_workspace_bytes(M, N, K, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, accumulate_fp32=False,
+                         fused_quant=False, grouped=False):
+    """Workspace bytes gemm() gives a call of this kind and size (0: the call launches one
+    kernel; otherwise three: the main tiles, the split last wave, the sum of its ranges)."""
+    args = GemmArgs()
+    args.recipe, args.layout = recipe, layout
+    args.M, args.N, args.K = M, N, K
+    args.c_fp32_accumulate = 1 if accumulate_fp32 else 0
+    args.num_groups = 1 if grouped else 0
+    if fused_quant:
+        args.q_out, args.s_out = 16, 16          # only their presence is read
+    return fp8q_gemm_workspace_bytes(args)
 
 
 def device_status(stream=None):

@@ -497,6 +497,12 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   p.s_out = qout ? a->s_out : nullptr;
   p.ld_q_out = a->ld_q_out;
   p.ld_s_out = a->ld_s_out;
+  if (a->workspace != nullptr && a->workspace_bytes >= 1024 && a->recipe == FP8Q_BLOCKWISE && !acc32 && !qout &&
+      !grouped) {
+    if (!aligned16(a->workspace)) return FP8Q_ERR_ALIGN;
+    p.ws = static_cast<float*>(a->workspace);
+    p.ws_bytes = a->workspace_bytes;
+  }
   p.ldc = a->ldc;
   p.m_offsets = a->m_offsets;
   p.num_groups = a->num_groups;
@@ -569,7 +575,30 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
                           CU_TENSOR_MAP_SWIZZLE_64B))
       return FP8Q_ERR_CUDA;
   }
-  return from_cuda(launch_gemm(p, ma, mb, msb, mc, mq, d->num_sms, s));
+  // the split tail's workspace: FP32 rows of 256 columns, stored in 16 x 32 boxes
+  CUtensorMap mws = ma;
+  if (p.ws != nullptr && !make_map(&mws, p.ws, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, kBlockwiseTileN,
+                                   (uint64_t)p.ws_bytes / (kBlockwiseTileN * 4), kBlockwiseTileN * 4, 16, 32,
+                                   CU_TENSOR_MAP_SWIZZLE_64B))
+    return FP8Q_ERR_CUDA;
+  return from_cuda(launch_gemm(p, ma, mb, msb, mc, mq, mws, d->num_sms, s));
+}
+
+size_t fp8q_gemm_workspace_bytes(const fp8q_gemm_args* a) {
+  if (!a || a->recipe != FP8Q_BLOCKWISE || a->layout < FP8Q_FPROP || a->layout > FP8Q_WGRAD) return 0;
+  if (a->c_fp32_accumulate || a->q_out || a->s_out || a->num_groups != 0) return 0;
+  if (a->M <= 0 || a->N <= 0 || a->K <= 0 || a->K % 128 != 0) return 0;
+  if (a->M >= (1ll << 31) || a->N >= (1ll << 31) || a->K >= (1ll << 31)) return 0;
+  DeviceScratch* d = nullptr;
+  if (scratch(&d) != FP8Q_OK) return 0;
+  GemmParams p;
+  std::memset(&p, 0, sizeof(p));
+  p.recipe = a->recipe;
+  p.layout = a->layout;
+  p.M = (int)a->M;
+  p.N = (int)a->N;
+  p.K = (int)a->K;
+  return blockwise_workspace_bytes(p, d->num_sms);
 }
 
 }  // extern "C"

@@ -626,9 +626,30 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
   }
 }
 
+// Work unit t of a launch: the raster index of its pair tile and its K chunks [kb0, kb1).
+// The main launch's units are whole tiles; a split tail's unit t is K range t % tail_splits
+// of tail tile t / tail_splits (raster index main_tiles + t / tail_splits).
+template <bool TAIL>
+__device__ __forceinline__ int unit_tile(int t, const GemmParams& p) {
+  return TAIL ? p.main_tiles + t / p.tail_splits : t;
+}
+template <bool TAIL>
+__device__ __forceinline__ void unit_chunks(int t, const GemmParams& p, int KB, int& kb0, int& kb1) {
+  if (TAIL) {
+    const int r = t % p.tail_splits;
+    kb0 = r * KB / p.tail_splits;
+    kb1 = (r + 1) * KB / p.tail_splits;
+  } else {
+    kb0 = 0;
+    kb1 = KB;
+  }
+}
+
 }  // namespace
 
-template <int L, bool GROUPED, int EPI>
+// TAIL: a split tail's launch (FP32 epilogue, p.ws through tma_c): unit t's 256 x 256 partial
+// sum over its K range is stored (not added) at workspace rows [256 t, 256 t + 256).
+template <int L, bool GROUPED, int EPI, bool TAIL>
 __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb,
@@ -636,6 +657,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
+  static_assert(!TAIL || (ACC32 && !GROUPED), "a split tail stores FP32 partial sums of whole tiles");
   using C = BwCfg<L>;
   constexpr int kBwBN = C::BN, kBwHalfBN = C::HalfBN, kBwEpiWarps = C::EpiWarps;
   constexpr int kBwProducerWarp = C::ProducerWarp, kBwMmaWarp = C::MmaWarp;
@@ -690,7 +712,9 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   const int row_tiles = GROUPED ? prefix[p.num_groups] : p.tiles_m;
-  const int total = row_tiles * p.tiles_n;
+  const int total = GROUPED ? row_tiles * p.tiles_n
+                    : TAIL  ? (p.tiles_m * p.tiles_n - p.main_tiles) * p.tail_splits
+                            : p.main_tiles;
   const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
 
   if (warp >= kBwEpiWarps) {
@@ -706,9 +730,11 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
-        const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
+        const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
         const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        int kb0, kb1;
+        unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) {
             raise_timeout(p, abort_flag);
@@ -739,9 +765,11 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
-      const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
       const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
-      for (int kb = 0; kb < KB; ++kb, ++it) {
+      int kb0, kb1;
+      unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const uint32_t r = it % kBwSb, rph = (it / kBwSb) & 1;
         int good = 1;
         if (lane == 0) {
@@ -785,7 +813,9 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
-        for (int kb = 0; kb < KB; ++kb, ++it) {
+        int kb0, kb1;
+        unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+        for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % kStages, pb = it & 1;
           if (!mbar_wait(&go[it % kBwGo], (it / kBwGo) & 1, abort_flag, kWaitLimitNs)) {
             raise_timeout(p, abort_flag);
@@ -817,12 +847,14 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     uint32_t chunk = 0, tile_it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters, ++tile_it) {
-      const Tile T = pair_tile_of<kBwBN>(t, p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
       const int ncol0 = T.n0 + cgp * 64;
       float2 acc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
-      for (int kb = 0; kb < KB; ++kb) {
+      int kb0, kb1;
+      unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+      for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t rs = chunk % kBwSb;
         if (!mbar_wait(&sfull[rs], (chunk / kBwSb) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
         const uint8_t* slot = smem + S::ring + rs * S::slot_bytes;
@@ -952,7 +984,10 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
-              tma_reduce_add_2d(&tma_c, stg, ncol0 + h * EC32, T.m0 + q * 32);
+              if constexpr (TAIL)   // this unit's own workspace rows: a store
+                tma_store_2d(&tma_c, stg, cgp * 64 + h * EC32, t * kBwPairM + (int)rank * kBM + q * 32);
+              else
+                tma_reduce_add_2d(&tma_c, stg, ncol0 + h * EC32, T.m0 + q * 32);
               bulk_commit();
             }
             continue;
@@ -1048,51 +1083,153 @@ static void raster(GemmParams& q, int row_tiles, int tile_m, int tile_n) {
   }
 }
 
-template <int L, bool G, int EPI = kEpiBf16>
-static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
-                                    const CUtensorMap& sb, const CUtensorMap& c, const CUtensorMap& qm, int num_sms,
-                                    cudaStream_t s) {
-  auto kern = gemm_blockwise_kernel<L, G, EPI>;
+// Launch configuration of one blockwise instantiation: its shared memory, the register check
+// of the register-moving (wgrad) form, and how many CTA pairs can be resident at once.
+template <int L, bool G, int EPI, bool TAIL>
+static cudaError_t blockwise_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int num_sms, cudaStream_t s,
+                                    int& pairs) {
+  auto kern = gemm_blockwise_kernel<L, G, EPI, TAIL>;
   using C = BwCfg<L>;
-  constexpr int kBwBN = C::BN;
   // The register reallocation inside the wgrad kernel adds up to exactly the launch pool at
   // 96 registers per thread; with any other count an increase could wait forever, so refuse.
   if constexpr (C::Split) {
     static const int regs = [] {
       cudaFuncAttributes fa{};
-      return cudaFuncGetAttributes(&fa, gemm_blockwise_kernel<L, G, EPI>) == cudaSuccess ? fa.numRegs : -1;
+      return cudaFuncGetAttributes(&fa, gemm_blockwise_kernel<L, G, EPI, TAIL>) == cudaSuccess ? fa.numRegs : -1;
     }();
     if (regs != C::RegsLaunch) return cudaErrorInvalidConfiguration;
   }
   const int smem = (int)BwSmem<L>::alloc;
   cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, smem);
   if (e != cudaSuccess) return e;
-  GemmParams q = p;
-  q.tiles_n = (p.N + kBwBN - 1) / kBwBN;
-  q.tiles_m = G ? (p.M + kBwPairM - 1) / kBwPairM + p.num_groups : (p.M + kBwPairM - 1) / kBwPairM;
-  raster(q, q.tiles_m, kBwPairM, kBwBN);
-  const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
-  cudaLaunchConfig_t cfg = {};
+  cfg = cudaLaunchConfig_t{};
   cfg.gridDim = dim3(num_sms - (num_sms & 1));
   cfg.blockDim = dim3(C::Threads);
   cfg.dynamicSmemBytes = smem;
   cfg.stream = s;
-  cudaLaunchAttribute attr[1];
   attr[0].id = cudaLaunchAttributeClusterDimension;
   attr[0].val.clusterDim.x = 2;
   attr[0].val.clusterDim.y = 1;
   attr[0].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  // persistent: as many pairs as can be resident at once (never more than the tiles)
   int resident = 0;
   e = cudaOccupancyMaxActiveClusters(&resident, kern, &cfg);
   if (e != cudaSuccess) return e;
-  int clusters = resident < num_sms / 2 ? resident : num_sms / 2;
-  if (clusters > tiles) clusters = (int)tiles;
-  if (clusters < 1) clusters = 1;
-  cfg.gridDim = dim3(2 * clusters);
-  return cudaLaunchKernelEx(&cfg, kern, q, a, b, sb, c, qm);
+  pairs = resident < num_sms / 2 ? resident : num_sms / 2;
+  if (pairs < 1) pairs = 1;
+  return cudaSuccess;
+}
+
+// Output tiles of a blockwise GEMM (256-row pair tiles x 256 columns) with its raster.
+static void blockwise_grid(GemmParams& q, bool grouped) {
+  q.tiles_n = (q.N + kBlockwiseTileN - 1) / kBlockwiseTileN;
+  q.tiles_m = (q.M + kBwPairM - 1) / kBwPairM + (grouped ? q.num_groups : 0);
+  raster(q, q.tiles_m, kBwPairM, kBlockwiseTileN);
+}
+
+// Split of the last, partial wave: with `pairs` persistent CTA pairs, `tiles` tiles leave
+// tiles % pairs for a last wave in which most pairs are idle for a whole tile.  When that
+// wave is at most half full, its tiles are cut into `splits` K ranges of at least 4 chunks
+// (at most one range per pair), so the wave takes about 1 / splits of a tile's time; the
+// ranges' FP32 partial sums go to a workspace and a small kernel adds them and rounds to
+// BF16.  The second launch, its pipeline fill and the sum cost about as much as 25-30 chunks
+// of a tile (measured on the 256 x 256 tiles: a Llama-3-8B wgrad, 64 chunks cut 9 ways, gains
+// 3-4%; its fprop, 32 chunks cut 4 ways, loses 0.5%), so the split is taken only when it saves
+// at least kTailMinSaved chunks of the last wave.  Returns the workspace bytes (0: no split).
+constexpr int kTailMinSaved = 40;
+static int64_t tail_plan(int64_t tiles, int pairs, int KB, int& tail, int& splits) {
+  tail = (int)(tiles % pairs);
+  splits = 0;
+  if (tail == 0 || 2 * tail > pairs) return 0;
+  const int s = min(pairs / tail, KB / 4);
+  if (s < 2 || KB - (KB + s - 1) / s < kTailMinSaved) return 0;
+  splits = s;
+  return (int64_t)tail * s * kBwPairM * kBlockwiseTileN * (int64_t)sizeof(float);
+}
+
+// Split tail, last step: each thread adds the K-range partial sums of 8 columns of one row of
+// a tail tile in range order (FP32) and stores them as BF16 into C, masked at M and N; a CTA
+// covers 8 rows, 32 CTAs a tile.
+__global__ void __launch_bounds__(256) blockwise_tail_sum_kernel(const __grid_constant__ GemmParams p) {
+  const int u = blockIdx.x >> 5, r = (blockIdx.x & 31) * 8 + (threadIdx.x >> 5);
+  int rt, nt;
+  raster_pos(p.main_tiles + u, p, p.tiles_m, rt, nt);
+  const int c = (threadIdx.x & 31) * 8;
+  const int m = rt * kBwPairM + r, n = nt * (int)kBlockwiseTileN + c;
+  if (m >= p.M || n >= p.N) return;
+  constexpr int64_t kRange = (int64_t)kBwPairM * kBlockwiseTileN / 4;   // float4s per K range
+  const float4* w = reinterpret_cast<const float4*>(p.ws) + (int64_t)u * p.tail_splits * kRange +
+                    ((int64_t)r * kBlockwiseTileN + c) / 4;
+  float4 lo = __ldg(w), hi = __ldg(w + 1);
+#pragma unroll 4
+  for (int k = 1; k < p.tail_splits; ++k) {
+    const float4 a = __ldg(w + k * kRange), b = __ldg(w + k * kRange + 1);
+    lo = make_float4(__fadd_rn(lo.x, a.x), __fadd_rn(lo.y, a.y), __fadd_rn(lo.z, a.z), __fadd_rn(lo.w, a.w));
+    hi = make_float4(__fadd_rn(hi.x, b.x), __fadd_rn(hi.y, b.y), __fadd_rn(hi.z, b.z), __fadd_rn(hi.w, b.w));
+  }
+  store8_bf16(p, m, n, make_uint4(pack_bf16(lo.x, lo.y), pack_bf16(lo.z, lo.w), pack_bf16(hi.x, hi.y),
+                                  pack_bf16(hi.z, hi.w)));
+}
+
+template <int L, bool G, int EPI = kEpiBf16>
+static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, const CUtensorMap& b,
+                                    const CUtensorMap& sb, const CUtensorMap& c, const CUtensorMap& qm,
+                                    const CUtensorMap& ws, int num_sms, cudaStream_t s) {
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  int pairs = 1;
+  cudaError_t e = blockwise_config<L, G, EPI, false>(cfg, attr, num_sms, s, pairs);
+  if (e != cudaSuccess) return e;
+  GemmParams q = p;
+  blockwise_grid(q, G);
+  const int64_t tiles = (int64_t)q.tiles_m * q.tiles_n;
+  if (tiles > (int64_t)INT32_MAX / 2) return cudaErrorInvalidValue;
+  q.main_tiles = (int)tiles;
+  q.tail_splits = 0;
+  int tail = 0, splits = 0;
+  if constexpr (EPI == kEpiBf16 && !G) {
+    const int64_t need = tail_plan(tiles, pairs, p.K / kBKB, tail, splits);
+    if (need > 0 && p.ws != nullptr && p.ws_bytes >= need) q.main_tiles = (int)(tiles - tail);
+    else splits = 0;
+  }
+  if (q.main_tiles > 0) {
+    cfg.gridDim = dim3(2 * (int)min((int64_t)pairs, (int64_t)q.main_tiles));
+    e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<L, G, EPI, false>, q, a, b, sb, c, qm);
+    if (e != cudaSuccess) return e;
+  }
+  if constexpr (EPI == kEpiBf16 && !G) {
+    if (splits > 0) {
+      cudaLaunchConfig_t tcfg;
+      cudaLaunchAttribute tattr[1];
+      int tpairs = 1;
+      e = blockwise_config<L, false, kEpiAcc32, true>(tcfg, tattr, num_sms, s, tpairs);
+      if (e != cudaSuccess) return e;
+      q.tail_splits = splits;
+      tcfg.gridDim = dim3(2 * min(tpairs, tail * splits));
+      e = cudaLaunchKernelEx(&tcfg, gemm_blockwise_kernel<L, false, kEpiAcc32, true>, q, a, b, sb, ws, qm);
+      if (e != cudaSuccess) return e;
+      blockwise_tail_sum_kernel<<<tail * 32, 256, 0, s>>>(q);
+      return cudaGetLastError();
+    }
+  }
+  return cudaSuccess;
+}
+
+size_t blockwise_workspace_bytes(const GemmParams& p, int num_sms) {
+  if (p.recipe != kBlockwise || p.c32 != nullptr || p.q_out != nullptr || p.num_groups > 0) return 0;
+  if (p.M <= 0 || p.N <= 0 || p.K <= 0) return 0;
+  cudaLaunchConfig_t cfg;
+  cudaLaunchAttribute attr[1];
+  int pairs = 1;
+  cudaError_t e = p.layout == kFprop   ? blockwise_config<kFprop, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs)
+                  : p.layout == kDgrad ? blockwise_config<kDgrad, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs)
+                                       : blockwise_config<kWgrad, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs);
+  if (e != cudaSuccess) return 0;
+  GemmParams q = p;
+  blockwise_grid(q, false);
+  int tail = 0, splits = 0;
+  return (size_t)tail_plan((int64_t)q.tiles_m * q.tiles_n, pairs, p.K / kBKB, tail, splits);
 }
 
 template <int R>
@@ -1141,24 +1278,24 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
 }
 
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
-                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q, int num_sms,
-                        cudaStream_t s) {
+                        const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q,
+                        const CUtensorMap& tma_ws, int num_sms, cudaStream_t s) {
   if (p.recipe == kBlockwise) {
     if (p.c32 != nullptr) {   // FP32 accumulate epilogue: its own instantiations
-      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      if (p.num_groups > 0) return launch_blockwise<kFprop, true, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiAcc32>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
     }
     if (p.q_out != nullptr) {  // BF16 output plus its fused 1x128 quantization
-      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+      if (p.layout == kFprop) return launch_blockwise<kFprop, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+      if (p.layout == kDgrad) return launch_blockwise<kDgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+      return launch_blockwise<kWgrad, false, kEpiQuant>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
     }
-    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
-    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, num_sms, s);
+    if (p.num_groups > 0) return launch_blockwise<kFprop, true>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+    if (p.layout == kFprop) return launch_blockwise<kFprop, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+    if (p.layout == kDgrad) return launch_blockwise<kDgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
+    return launch_blockwise<kWgrad, false>(p, tma_a, tma_b, tma_sb, tma_c, tma_q, tma_ws, num_sms, s);
   }
   if (p.recipe == kMx) return launch_scaled<kMx>(p, tma_a, tma_b, num_sms, s);
   if (p.recipe == kPerTensor) return launch_scaled<kPerTensor>(p, tma_a, tma_b, num_sms, s);

@@ -322,9 +322,27 @@ typedef struct {
   uint8_t* q_out;               /* optional fused 1x128 quantization of C (see above) */
   float* s_out;
   int64_t ld_q_out, ld_s_out;
+  void* workspace;              /* optional: split of the last wave (see fp8q_gemm_workspace_bytes) */
+  int64_t workspace_bytes;
 } fp8q_gemm_args;
 
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);
+
+/* Workspace bytes that fp8q_gemm_blockscaled can use for `args` on the current device; 0 when
+ * the call would use none.  Only BLOCKWISE GEMMs with BF16 output, not grouped and without the
+ * fused quantization, use one: their kernel keeps one CTA pair per two SMs and walks the
+ * 256 x 256 output tiles wave by wave, and when the last wave would leave more than half of
+ * the pairs idle for a whole tile, its tiles are cut into K ranges of at least 4 chunks of 128
+ * (one range per pair at most), run as a second launch that stores each range's FP32 partial
+ * sum (the same promoted sum, over the range's chunks only) into the workspace, and a third
+ * small launch adds the ranges in order in FP32 and rounds to BF16 into C.  The result is the
+ * same FP32 sum, grouped by ranges, so it can differ from the unsplit schedule's by FP32
+ * rounding, and it is the same on every run.  workspace (device memory, 16-byte aligned, or
+ * NULL) with workspace_bytes: a NULL workspace, fewer bytes than this function returns, or
+ * any other kind of GEMM keeps the unsplit schedule (no error).  The library only uses the
+ * workspace in kernels enqueued on the call's stream; the caller must not use it
+ * concurrently elsewhere before they complete.  Returns 0 for NULL or invalid arguments. */
+size_t fp8q_gemm_workspace_bytes(const fp8q_gemm_args* args);
 
 /* Bytes of a scale-factor buffer: recipe MXFP8 (inner/32 scale columns) or NVFP4
  * (inner/16), `outer` rows, in `layout`.  Returns 0 for other recipes. */

@@ -266,3 +266,41 @@ def test_quantize_multi_validates_every_item_before_launching():
     # empty items are skipped: nothing to launch
     assert call(item(fq.FP8Q_ITEM_1X128, 0, 128, **one), item(fq.FP8Q_ITEM_128X128, 128, 0, **w)) == fq.FP8Q_OK
     assert ctypes.sizeof(fq.QuantItem) == 112
+
+
+@pytest.mark.skipif(subprocess.run(["which", "gcc"], capture_output=True).returncode != 0, reason="needs gcc")
+def test_binding_structs_match_the_header_layout(tmp_path):
+    """The ctypes mirrors have the size and field offsets that a C compiler gives the header's
+    argument structs (compiled from include/fp8q.h on the host)."""
+    exe = str(tmp_path / "abi_layout")
+    here = os.path.dirname(os.path.abspath(__file__))
+    subprocess.run(["gcc", "-std=c99", "-Wall", "-Werror", "-I", os.path.dirname(HEADER), "-o", exe,
+                    os.path.join(here, "host", "abi_layout.c")], check=True)
+    got = dict(line.split() for line in subprocess.run([exe], check=True, capture_output=True,
+                                                        text=True).stdout.splitlines())
+    for cname, cls in (("fp8q_gemm_args", fq.GemmArgs), ("fp8q_quant_item", fq.QuantItem)):
+        assert int(got[cname]) == ctypes.sizeof(cls), cname
+        for field, _ in cls._fields_:
+            assert int(got[f"{cname}.{field}"]) == getattr(cls, field).offset, (cname, field)
+        assert sum(k.startswith(cname + ".") for k in got) == len(cls._fields_), cname
+
+
+def test_gemm_workspace_bytes_is_zero_without_a_device_or_a_splittable_call(L):
+    """The workspace query never fails: NULL arguments, non-blockwise recipes and, here with no
+    GPU, every call report 0 (the GEMM then keeps its unsplit schedule)."""
+    assert L.fp8q_gemm_workspace_bytes(None) == 0
+    for recipe in (fq.FP8Q_BLOCKWISE, fq.FP8Q_MXFP8, fq.FP8Q_NVFP4):
+        assert fq.gemm_workspace_bytes(8192, 14336, 4096, recipe, fq.FP8Q_FPROP) == 0
+    assert fq.gemm_workspace_bytes(300, 19328, 2176, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, accumulate_fp32=True) == 0
+
+
+def test_gemm_workspace_argument_checked_before_anything_runs(L):
+    """A misaligned workspace given to a GEMM that could use one is an alignment error, found
+    on the host before any launch."""
+    a = fq.GemmArgs()
+    a.recipe, a.layout, a.M, a.N, a.K = fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, 256, 256, 512
+    a.a = a.b = a.a_scale = a.b_scale = a.c = 1 << 20
+    a.lda = a.ldb = 512
+    a.ld_sa, a.ld_sb, a.ldc = 256, 4, 256
+    a.workspace, a.workspace_bytes = (1 << 20) + 8, 1 << 20
+    assert fq.fp8q_gemm_blockscaled(a, None) == fq.FP8Q_ERR_ALIGN

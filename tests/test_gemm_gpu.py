@@ -262,6 +262,129 @@ def test_blockwise_partial_last_wave(cuda_lib, layout):
     assert fq.device_status() == 0
 
 
+def _pairs():
+    return torch.cuda.get_device_properties(0).multi_processor_count // 2
+
+
+def _split_tail_plan(M, N, K, pairs):
+    """The launcher's split of the last wave, restated: 256 x 256 pair tiles in its raster
+    order (groups of row tiles sweeping the columns when M <= N, else groups of column tiles
+    sweeping the rows, each group about 40 MB of the resident operand); the last
+    tiles % pairs tiles are split into s = min(pairs // tail, (K / 128) // 4) K ranges when they
+    fill at most half a wave, s >= 2 and the split saves at least 40 of the K / 128 chunks.
+    Returns the (row, column) origins of the split tiles and the workspace bytes (0: no split)."""
+    tm, tn = -(-M // 256), -(-N // 256)
+    tiles = tm * tn
+    tail = tiles % pairs
+    if tail == 0 or 2 * tail > pairs:
+        return [], 0
+    kb = K // 128
+    s = min(pairs // tail, kb // 4)
+    if s < 2 or kb - -(-kb // s) < 40:
+        return [], 0
+    g = (40 << 20) // (256 * K)
+    out = []
+    for t in range(tiles - tail, tiles):
+        if M <= N:
+            gm = max(1, min(g, tm))
+            per = gm * tn
+            grp, loc = divmod(t, per)
+            first = grp * gm
+            gsz = min(tm - first, gm)
+            rt, nt = first + loc % gsz, loc // gsz
+        else:
+            gn = max(1, min(g, tn))
+            per = gn * tm
+            grp, loc = divmod(t, per)
+            first = grp * gn
+            gsz = min(tn - first, gn)
+            nt, rt = first + loc % gsz, loc // gsz
+        out.append((rt * 256, nt * 256))
+    return out, tail * s * 256 * 256 * 4
+
+
+@pytest.mark.parametrize("layout", ["fprop", "dgrad", "wgrad"])
+def test_blockwise_split_last_wave(cuda_lib, layout):
+    """One full wave plus 4 tiles (6 row tiles, the last 240 rows; 13 column tiles, the last
+    128 wide; 74 pairs): the 4 tiles run as 12 K ranges of 4 chunks each with FP32 partial
+    sums in a workspace.  Every element is checked against the oracle, with and without the
+    split; the split result is the same on a second run."""
+    fq = cuda_lib
+    pairs = _pairs()
+    tn = -(-(pairs + 4) // 6)
+    M, N, K = 6 * 256 - 16, tn * 256 - 128, 6144     # M % 16 == 0: wgrad's colwise quantization
+    tiles, nbytes = _split_tail_plan(M, N, K, pairs)
+    assert nbytes > 0 and len(tiles) == 6 * tn - pairs
+    L = {"fprop": fq.FP8Q_FPROP, "dgrad": fq.FP8Q_DGRAD, "wgrad": fq.FP8Q_WGRAD}[layout]
+    assert fq.gemm_workspace_bytes(M, N, K, fq.FP8Q_BLOCKWISE, L) == nbytes
+    if layout == "fprop":
+        X, W = bf((M, K), 1.0, 71, 1e-3, 50.0), bf((K, N), 0.02, 72)
+        qx, qw = fq.quantize_1x128(X.cuda()), fq.quantize_128x128(W.cuda())
+        run = lambda split: fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, L, a_scale=qx["s_row"],  # noqa: E731
+                                    b_scale=qw["s"], split_tail=split)
+        ox, osx = Q.quantize_1x128_rowwise(workloads.bf16_bits(X))
+        _, owt, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(owt, osw, G.FPROP))
+    elif layout == "dgrad":
+        dY, W = bf((M, K), 1e-3, 73), bf((N, K), 0.02, 74)
+        qd, qw = fq.quantize_1x128(dY.cuda()), fq.quantize_128x128(W.cuda())
+        run = lambda split: fq.gemm(qd["q_row"], qw["q"], fq.FP8Q_BLOCKWISE, L, a_scale=qd["s_row"],  # noqa: E731
+                                    b_scale=qw["s"], ld_sb=N // 128, split_tail=split)
+        od, osd = Q.quantize_1x128_rowwise(workloads.bf16_bits(dY))
+        ow, _, osw = Q.quantize_128x128(workloads.bf16_bits(W))
+        ref, t = G.reference(G.dequant_a_1x128(od, osd), G.dequant_b_blockwise(ow, osw, G.DGRAD))
+    else:
+        X, dY = bf((K, M), 1.0, 75, 1e-3, 50.0), bf((K, N), 1e-3, 76)   # K tokens
+        qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
+        qd = fq.quantize_1x128(dY.cuda(), rowwise=False, colwise=True)
+        run = lambda split: fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, L, a_scale=qx["s_col"],  # noqa: E731
+                                    b_scale=qd["s_col"], split_tail=split)
+        ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
+        od, osd = Q.quantize_1x128_colwise(workloads.bf16_bits(dY))
+        ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od, osd, G.WGRAD))
+    c_split = run(True)
+    c_again = run(True)
+    c_whole = run(False)
+    assert fq.device_status() == 0
+    check(c_split, ref, t, f"{layout}, split last wave")
+    check(c_whole, ref, t, f"{layout}, unsplit")
+    assert torch.equal(c_split.view(torch.int16), c_again.view(torch.int16)), "split result not repeatable"
+    # outside the split tiles the two schedules run the same kernel on the same data
+    mask = torch.ones((M, N), dtype=torch.bool)
+    for m0, n0 in tiles:
+        mask[m0:m0 + 256, n0:n0 + 256] = False
+    assert torch.equal(c_split.cpu()[mask].view(torch.int16), c_whole.cpu()[mask].view(torch.int16))
+
+
+def test_llama8b_split_last_wave_tiles_fullsize(cuda_lib):
+    """At the bench's sizes only wgrad (896 tiles: 12 waves + 8, 64 chunks cut 9 ways) splits
+    its last wave; fprop (1792: 24 waves + 16, 32 chunks) and dgrad (512: 6 waves + 68) do not.
+    Every element of every split wgrad tile is checked against the oracle."""
+    fq = cuda_lib
+    pairs = _pairs()
+    for M, N, K, L in ((8192, 14336, 4096, fq.FP8Q_FPROP), (8192, 4096, 14336, fq.FP8Q_DGRAD),
+                       (4096, 14336, 8192, fq.FP8Q_WGRAD)):
+        assert fq.gemm_workspace_bytes(M, N, K, fq.FP8Q_BLOCKWISE, L) == _split_tail_plan(M, N, K, pairs)[1]
+    tiles, nb = _split_tail_plan(4096, 14336, 8192, pairs)
+    assert nb > 0 and len(tiles) == 896 % pairs
+    d = workloads.llama8b(device="cuda")
+    X, dY = d["X"], d["dY"]
+    qx = fq.quantize_1x128(X, rowwise=False, colwise=True)
+    qd = fq.quantize_1x128(dY, rowwise=False, colwise=True)
+    Xb, dYb = workloads.bf16_bits(X), workloads.bf16_bits(dY)
+    c = host(fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
+                     b_scale=qd["s_col"]).float())
+    for m0, n0 in tiles:
+        for dm in (0, 128):
+            for dn in (0, 128):
+                r, q = m0 + dm, n0 + dn
+                oa, sa = Q.quantize_1x128_colwise(Xb[:, r:r + 128])
+                ob, sb = Q.quantize_1x128_colwise(dYb[:, q:q + 128])
+                ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
+                check(c[r:r + 128, q:q + 128].astype(np.float64), ref, t, f"wgrad split tile {r},{q}")
+    assert fq.device_status() == 0
+
+
 def test_blockwise_more_tiles_than_sms(cuda_lib):
     """2048 x 4096 output = 256 tiles: every CTA runs the persistent loop more than once."""
     fq = cuda_lib
