@@ -148,8 +148,8 @@ class LlamaStep:
             return f
 
         def kernels(Mg, Ng, Kg, layout):
-            # a GEMM whose last wave is split runs three kernels (main tiles, split tail, sum)
-            return 3 if fq.gemm_workspace_bytes(Mg, Ng, Kg, fq.FP8Q_BLOCKWISE, layout) > 0 else 1
+            # a GEMM whose last wave is split runs two kernels (the tiles and K ranges, the sum)
+            return 2 if fq.gemm_workspace_bytes(Mg, Ng, Kg, fq.FP8Q_BLOCKWISE, layout) > 0 else 1
 
         if self.separate_quant:
             quant = [

@@ -490,7 +490,7 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
 def gemm_workspace_bytes(M, N, K, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, accumulate_fp32=False,
                          fused_quant=False, grouped=False):
     """Workspace bytes gemm() gives a call of this kind and size (0: the call launches one
-    kernel; otherwise three: the main tiles, the split last wave, the sum of its ranges)."""
+    kernel; otherwise two: the tiles with the last wave's K ranges, then the sum of the ranges)."""
     args = GemmArgs()
     args.recipe, args.layout = recipe, layout
     args.M, args.N, args.K = M, N, K

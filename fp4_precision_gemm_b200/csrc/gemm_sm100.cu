@@ -627,29 +627,26 @@ __device__ __forceinline__ void load_pair_groups(const GemmParams& p, int* prefi
 }
 
 // Work unit t of a launch: the raster index of its pair tile and its K chunks [kb0, kb1).
-// The main launch's units are whole tiles; a split tail's unit t is K range t % tail_splits
-// of tail tile t / tail_splits (raster index main_tiles + t / tail_splits).
-template <bool TAIL>
+// Units below main_tiles are whole tiles; with a split last wave, unit main_tiles + u is K
+// range u % tail_splits of tile main_tiles + u / tail_splits.
+template <bool RANGES>
 __device__ __forceinline__ int unit_tile(int t, const GemmParams& p) {
-  return TAIL ? p.main_tiles + t / p.tail_splits : t;
+  return (RANGES && t >= p.main_tiles) ? p.main_tiles + (t - p.main_tiles) / p.tail_splits : t;
 }
-template <bool TAIL>
+template <bool RANGES>
 __device__ __forceinline__ void unit_chunks(int t, const GemmParams& p, int KB, int& kb0, int& kb1) {
-  if (TAIL) {
-    const int r = t % p.tail_splits;
+  kb0 = 0;
+  kb1 = KB;
+  if (RANGES && t >= p.main_tiles) {
+    const int r = (t - p.main_tiles) % p.tail_splits;
     kb0 = r * KB / p.tail_splits;
     kb1 = (r + 1) * KB / p.tail_splits;
-  } else {
-    kb0 = 0;
-    kb1 = KB;
   }
 }
 
 }  // namespace
 
-// TAIL: a split tail's launch (FP32 epilogue, p.ws through tma_c): unit t's 256 x 256 partial
-// sum over its K range is stored (not added) at workspace rows [256 t, 256 t + 256).
-template <int L, bool GROUPED, int EPI, bool TAIL>
+template <int L, bool GROUPED, int EPI>
 __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     gemm_blockwise_kernel(const __grid_constant__ GemmParams p, const __grid_constant__ CUtensorMap tma_a,
                           const __grid_constant__ CUtensorMap tma_b, const __grid_constant__ CUtensorMap tma_sb,
@@ -657,7 +654,9 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
-  static_assert(!TAIL || (ACC32 && !GROUPED), "a split tail stores FP32 partial sums of whole tiles");
+  // BF16 output, not grouped: the last wave may be split into K ranges, whose FP32 partial
+  // sums go to the workspace (p.ws, through tma_q) instead of C
+  constexpr bool RANGES = (EPI == kEpiBf16) && !GROUPED;
   using C = BwCfg<L>;
   constexpr int kBwBN = C::BN, kBwHalfBN = C::HalfBN, kBwEpiWarps = C::EpiWarps;
   constexpr int kBwProducerWarp = C::ProducerWarp, kBwMmaWarp = C::MmaWarp;
@@ -713,8 +712,8 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
   const uint32_t tmem = *tmem_slot;
   const int row_tiles = GROUPED ? prefix[p.num_groups] : p.tiles_m;
   const int total = GROUPED ? row_tiles * p.tiles_n
-                    : TAIL  ? (p.tiles_m * p.tiles_n - p.main_tiles) * p.tail_splits
-                            : p.main_tiles;
+                    : RANGES ? p.main_tiles + (p.tiles_m * p.tiles_n - p.main_tiles) * p.tail_splits
+                             : p.main_tiles;
   const int cluster = (int)(blockIdx.x >> 1), n_clusters = (int)(gridDim.x >> 1);
 
   if (warp >= kBwEpiWarps) {
@@ -730,10 +729,10 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       uint32_t it = 0;
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
-        const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
+        const Tile T = pair_tile_of<kBwBN>(unit_tile<RANGES>(t, p), p, row_tiles, prefix, offs, rank);
         const int b_row = T.g * p.N + T.n0 + (int)rank * kBwHalfBN;
         int kb0, kb1;
-        unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+        unit_chunks<RANGES>(t, p, KB, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % kStages, ph = (it / kStages) & 1;
           if (!mbar_wait(&empty[s], ph ^ 1, abort_flag, kWaitLimitNs)) {
@@ -765,10 +764,10 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     uint32_t it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters) {
-      const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(unit_tile<RANGES>(t, p), p, row_tiles, prefix, offs, rank);
       const float* sbg = p.sb + (GROUPED ? (int64_t)T.g * ((p.N + kBM - 1) / kBM) * p.ld_sb : 0);
       int kb0, kb1;
-      unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+      unit_chunks<RANGES>(t, p, KB, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb, ++it) {
         const uint32_t r = it % kBwSb, rph = (it / kBwSb) & 1;
         int good = 1;
@@ -814,7 +813,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       bool ok = true;
       for (int t = cluster; t < total && ok; t += n_clusters) {
         int kb0, kb1;
-        unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+        unit_chunks<RANGES>(t, p, KB, kb0, kb1);
         for (int kb = kb0; kb < kb1; ++kb, ++it) {
           const uint32_t s = it % kStages, pb = it & 1;
           if (!mbar_wait(&go[it % kBwGo], (it / kBwGo) & 1, abort_flag, kWaitLimitNs)) {
@@ -847,13 +846,13 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
     uint32_t chunk = 0, tile_it = 0;
     bool ok = true;
     for (int t = cluster; t < total && ok; t += n_clusters, ++tile_it) {
-      const Tile T = pair_tile_of<kBwBN>(unit_tile<TAIL>(t, p), p, row_tiles, prefix, offs, rank);
+      const Tile T = pair_tile_of<kBwBN>(unit_tile<RANGES>(t, p), p, row_tiles, prefix, offs, rank);
       const int ncol0 = T.n0 + cgp * 64;
       float2 acc[32];
 #pragma unroll
       for (int i = 0; i < 32; ++i) acc[i] = make_float2(0.0f, 0.0f);
       int kb0, kb1;
-      unit_chunks<TAIL>(t, p, KB, kb0, kb1);
+      unit_chunks<RANGES>(t, p, KB, kb0, kb1);
       for (int kb = kb0; kb < kb1; ++kb) {
         const uint32_t rs = chunk % kBwSb;
         if (!mbar_wait(&sfull[rs], (chunk / kBwSb) & 1, abort_flag, kWaitLimitNs)) { raise_timeout(p, abort_flag); ok = false; break; }
@@ -929,6 +928,29 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
       constexpr int EC = S::epi_cols, CPR = EC / 8, RPI = 32 / CPR;
       auto swz = [](int r) { return CPR == 8 ? (r & 7) : ((r >> 1) & 3); };
       uint4* stg = reinterpret_cast<uint4*>(smem + S::cst + warp * S::stage_c);
+      if (RANGES && t >= p.main_tiles) {
+        // a K range of a split tile: its FP32 partial sum goes, in the same 32 x 16 boxes as
+        // the FP32-accumulate epilogue, to this unit's own workspace rows by TMA store
+        const int wrow = (t - p.main_tiles) * kBwPairM + (int)rank * kBM + q * 32;
+#pragma unroll
+        for (int h = 0; h < 4; ++h) {
+          if (lane == 0) bulk_wait_read();
+          __syncwarp();
+#pragma unroll
+          for (int c = 0; c < CPR; ++c) {
+            const float2* a2 = acc + h * 8 + c * 2;
+            stg[lane * CPR + (c ^ swz(lane))] = make_uint4(__float_as_uint(a2[0].x), __float_as_uint(a2[0].y),
+                                                           __float_as_uint(a2[1].x), __float_as_uint(a2[1].y));
+          }
+          fence_proxy_async();
+          __syncwarp();
+          if (lane == 0) {
+            tma_store_2d(&tma_q, stg, cgp * 64 + h * 16, wrow);
+            bulk_commit();
+          }
+        }
+        continue;
+      }
       if constexpr (!ACC32) {
         // BF16: the staged 32 x 32 box goes out by one TMA store and the warp moves on to the
         // next tile while the copy engine writes it (the swizzled staging layout is the tensor
@@ -984,10 +1006,7 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
             fence_proxy_async();
             __syncwarp();
             if (lane == 0) {
-              if constexpr (TAIL)   // this unit's own workspace rows: a store
-                tma_store_2d(&tma_c, stg, cgp * 64 + h * EC32, t * kBwPairM + (int)rank * kBM + q * 32);
-              else
-                tma_reduce_add_2d(&tma_c, stg, ncol0 + h * EC32, T.m0 + q * 32);
+              tma_reduce_add_2d(&tma_c, stg, ncol0 + h * EC32, T.m0 + q * 32);
               bulk_commit();
             }
             continue;
@@ -1085,17 +1104,17 @@ static void raster(GemmParams& q, int row_tiles, int tile_m, int tile_n) {
 
 // Launch configuration of one blockwise instantiation: its shared memory, the register check
 // of the register-moving (wgrad) form, and how many CTA pairs can be resident at once.
-template <int L, bool G, int EPI, bool TAIL>
+template <int L, bool G, int EPI>
 static cudaError_t blockwise_config(cudaLaunchConfig_t& cfg, cudaLaunchAttribute* attr, int num_sms, cudaStream_t s,
                                     int& pairs) {
-  auto kern = gemm_blockwise_kernel<L, G, EPI, TAIL>;
+  auto kern = gemm_blockwise_kernel<L, G, EPI>;
   using C = BwCfg<L>;
   // The register reallocation inside the wgrad kernel adds up to exactly the launch pool at
   // 96 registers per thread; with any other count an increase could wait forever, so refuse.
   if constexpr (C::Split) {
     static const int regs = [] {
       cudaFuncAttributes fa{};
-      return cudaFuncGetAttributes(&fa, gemm_blockwise_kernel<L, G, EPI, TAIL>) == cudaSuccess ? fa.numRegs : -1;
+      return cudaFuncGetAttributes(&fa, gemm_blockwise_kernel<L, G, EPI>) == cudaSuccess ? fa.numRegs : -1;
     }();
     if (regs != C::RegsLaunch) return cudaErrorInvalidConfiguration;
   }
@@ -1131,13 +1150,14 @@ static void blockwise_grid(GemmParams& q, bool grouped) {
 // Split of the last, partial wave: with `pairs` persistent CTA pairs, `tiles` tiles leave
 // tiles % pairs for a last wave in which most pairs are idle for a whole tile.  When that
 // wave is at most half full, its tiles are cut into `splits` K ranges of at least 4 chunks
-// (at most one range per pair), so the wave takes about 1 / splits of a tile's time; the
-// ranges' FP32 partial sums go to a workspace and a small kernel adds them and rounds to
-// BF16.  The second launch, its pipeline fill and the sum cost about as much as 25-30 chunks
-// of a tile (measured on the 256 x 256 tiles: a Llama-3-8B wgrad, 64 chunks cut 9 ways, gains
-// 3-4%; its fprop, 32 chunks cut 4 ways, loses 0.5%), so the split is taken only when it saves
-// at least kTailMinSaved chunks of the last wave.  Returns the workspace bytes (0: no split).
-constexpr int kTailMinSaved = 40;
+// (at most one range per pair), run after the whole tiles in the same launch, so the wave
+// takes about 1 / splits of a tile's time; the ranges' FP32 partial sums go to a workspace
+// and a small kernel adds them and rounds to BF16.  The ranges' FP32 stores, the sum kernel
+// and its launch cost about as much as 10-15 chunks of a tile (Llama-3-8B on 256 x 256
+// tiles: wgrad, 64 chunks cut 9 ways, -4.9%; fprop, 32 chunks cut 4 ways, -0.8%), so the
+// split is taken only when it saves at least kTailMinSaved chunks of the last wave.
+// Returns the workspace bytes (0: no split).
+constexpr int kTailMinSaved = 16;
 static int64_t tail_plan(int64_t tiles, int pairs, int KB, int& tail, int& splits) {
   tail = (int)(tiles % pairs);
   splits = 0;
@@ -1179,7 +1199,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   int pairs = 1;
-  cudaError_t e = blockwise_config<L, G, EPI, false>(cfg, attr, num_sms, s, pairs);
+  cudaError_t e = blockwise_config<L, G, EPI>(cfg, attr, num_sms, s, pairs);
   if (e != cudaSuccess) return e;
   GemmParams q = p;
   blockwise_grid(q, G);
@@ -1189,29 +1209,24 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   q.tail_splits = 0;
   int tail = 0, splits = 0;
   if constexpr (EPI == kEpiBf16 && !G) {
+    // the split ranges run as extra units of this launch, after the whole tiles
     const int64_t need = tail_plan(tiles, pairs, p.K / kBKB, tail, splits);
-    if (need > 0 && p.ws != nullptr && p.ws_bytes >= need) q.main_tiles = (int)(tiles - tail);
-    else splits = 0;
-  }
-  if (q.main_tiles > 0) {
-    cfg.gridDim = dim3(2 * (int)min((int64_t)pairs, (int64_t)q.main_tiles));
-    e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<L, G, EPI, false>, q, a, b, sb, c, qm);
-    if (e != cudaSuccess) return e;
-  }
-  if constexpr (EPI == kEpiBf16 && !G) {
-    if (splits > 0) {
-      cudaLaunchConfig_t tcfg;
-      cudaLaunchAttribute tattr[1];
-      int tpairs = 1;
-      e = blockwise_config<L, false, kEpiAcc32, true>(tcfg, tattr, num_sms, s, tpairs);
-      if (e != cudaSuccess) return e;
+    if (need > 0 && p.ws != nullptr && p.ws_bytes >= need) {
+      q.main_tiles = (int)(tiles - tail);
       q.tail_splits = splits;
-      tcfg.gridDim = dim3(2 * min(tpairs, tail * splits));
-      e = cudaLaunchKernelEx(&tcfg, gemm_blockwise_kernel<L, false, kEpiAcc32, true>, q, a, b, sb, ws, qm);
-      if (e != cudaSuccess) return e;
-      blockwise_tail_sum_kernel<<<tail * 32, 256, 0, s>>>(q);
-      return cudaGetLastError();
+    } else {
+      splits = 0;
     }
+  }
+  const int64_t units = q.main_tiles + (int64_t)tail * splits;
+  cfg.gridDim = dim3(2 * (int)min((int64_t)pairs, units));
+  // tma_q carries the workspace map when the last wave is split (the BF16 epilogue has no
+  // fused quantization)
+  e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<L, G, EPI>, q, a, b, sb, c, splits > 0 ? ws : qm);
+  if (e != cudaSuccess) return e;
+  if (splits > 0) {
+    blockwise_tail_sum_kernel<<<tail * 32, 256, 0, s>>>(q);
+    return cudaGetLastError();
   }
   return cudaSuccess;
 }
@@ -1222,9 +1237,9 @@ size_t blockwise_workspace_bytes(const GemmParams& p, int num_sms) {
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];
   int pairs = 1;
-  cudaError_t e = p.layout == kFprop   ? blockwise_config<kFprop, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs)
-                  : p.layout == kDgrad ? blockwise_config<kDgrad, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs)
-                                       : blockwise_config<kWgrad, false, kEpiBf16, false>(cfg, attr, num_sms, 0, pairs);
+  cudaError_t e = p.layout == kFprop   ? blockwise_config<kFprop, false, kEpiBf16>(cfg, attr, num_sms, 0, pairs)
+                  : p.layout == kDgrad ? blockwise_config<kDgrad, false, kEpiBf16>(cfg, attr, num_sms, 0, pairs)
+                                       : blockwise_config<kWgrad, false, kEpiBf16>(cfg, attr, num_sms, 0, pairs);
   if (e != cudaSuccess) return 0;
   GemmParams q = p;
   blockwise_grid(q, false);

@@ -271,7 +271,7 @@ def _split_tail_plan(M, N, K, pairs):
     order (groups of row tiles sweeping the columns when M <= N, else groups of column tiles
     sweeping the rows, each group about 40 MB of the resident operand); the last
     tiles % pairs tiles are split into s = min(pairs // tail, (K / 128) // 4) K ranges when they
-    fill at most half a wave, s >= 2 and the split saves at least 40 of the K / 128 chunks.
+    fill at most half a wave, s >= 2 and the split saves at least 16 of the K / 128 chunks.
     Returns the (row, column) origins of the split tiles and the workspace bytes (0: no split)."""
     tm, tn = -(-M // 256), -(-N // 256)
     tiles = tm * tn
@@ -280,7 +280,7 @@ def _split_tail_plan(M, N, K, pairs):
         return [], 0
     kb = K // 128
     s = min(pairs // tail, kb // 4)
-    if s < 2 or kb - -(-kb // s) < 40:
+    if s < 2 or kb - -(-kb // s) < 16:
         return [], 0
     g = (40 << 20) // (256 * K)
     out = []
@@ -306,8 +306,8 @@ def _split_tail_plan(M, N, K, pairs):
 @pytest.mark.parametrize("layout", ["fprop", "dgrad", "wgrad"])
 def test_blockwise_split_last_wave(cuda_lib, layout):
     """One full wave plus 4 tiles (6 row tiles, the last 240 rows; 13 column tiles, the last
-    128 wide; 74 pairs): the 4 tiles run as 12 K ranges of 4 chunks each with FP32 partial
-    sums in a workspace.  Every element is checked against the oracle, with and without the
+    128 wide; 74 pairs): the 4 tiles run as 12 K ranges of 4 chunks each, after the whole
+    tiles in the same launch, with FP32 partial sums in a workspace.  Every element is checked against the oracle, with and without the
     split; the split result is the same on a second run."""
     fq = cuda_lib
     pairs = _pairs()
@@ -357,28 +357,41 @@ def test_blockwise_split_last_wave(cuda_lib, layout):
 
 
 def test_llama8b_split_last_wave_tiles_fullsize(cuda_lib):
-    """At the bench's sizes only wgrad (896 tiles: 12 waves + 8, 64 chunks cut 9 ways) splits
-    its last wave; fprop (1792: 24 waves + 16, 32 chunks) and dgrad (512: 6 waves + 68) do not.
-    Every element of every split wgrad tile is checked against the oracle."""
+    """At the bench's sizes fprop (1792 tiles: 24 waves + 16, 32 chunks cut 4 ways) and wgrad
+    (896: 12 waves + 8, 64 chunks cut 9 ways) split their last wave; dgrad (512: 6 waves + 68)
+    does not.  Every element of every split tile is checked against the oracle."""
     fq = cuda_lib
     pairs = _pairs()
-    for M, N, K, L in ((8192, 14336, 4096, fq.FP8Q_FPROP), (8192, 4096, 14336, fq.FP8Q_DGRAD),
-                       (4096, 14336, 8192, fq.FP8Q_WGRAD)):
-        assert fq.gemm_workspace_bytes(M, N, K, fq.FP8Q_BLOCKWISE, L) == _split_tail_plan(M, N, K, pairs)[1]
+    assert fq.gemm_workspace_bytes(8192, 4096, 14336, fq.FP8Q_BLOCKWISE, fq.FP8Q_DGRAD) == 0
+    d = workloads.llama8b(device="cuda")
+    X, W, dY = d["X"], d["W"], d["dY"]
+    Xb, Wb, dYb = workloads.bf16_bits(X), workloads.bf16_bits(W), workloads.bf16_bits(dY)
+    # FPROP (8192, 4096, 14336)
+    tiles, nb = _split_tail_plan(8192, 14336, 4096, pairs)
+    assert nb > 0 and len(tiles) == 1792 % pairs
+    assert fq.gemm_workspace_bytes(8192, 14336, 4096, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP) == nb
+    qx = fq.quantize_1x128(X, rowwise=True, colwise=True)
+    qw = fq.quantize_128x128(W)
+    c = host(fq.gemm(qx["q_row"], qw["q_t"], fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, a_scale=qx["s_row"],
+                     b_scale=qw["s"]).float())
+    for m0, n0 in tiles:
+        for r in (m0, m0 + 128):
+            oa, sa = Q.quantize_1x128_rowwise(Xb[r:r + 128])
+            for q in (n0, n0 + 128):
+                _, owt, sw = Q.quantize_128x128(Wb[:, q:q + 128])
+                ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(owt, sw, G.FPROP))
+                check(c[r:r + 128, q:q + 128].astype(np.float64), ref, t, f"fprop split tile {r},{q}")
+    # WGRAD (4096, 8192, 14336)
     tiles, nb = _split_tail_plan(4096, 14336, 8192, pairs)
     assert nb > 0 and len(tiles) == 896 % pairs
-    d = workloads.llama8b(device="cuda")
-    X, dY = d["X"], d["dY"]
-    qx = fq.quantize_1x128(X, rowwise=False, colwise=True)
+    assert fq.gemm_workspace_bytes(4096, 14336, 8192, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD) == nb
     qd = fq.quantize_1x128(dY, rowwise=False, colwise=True)
-    Xb, dYb = workloads.bf16_bits(X), workloads.bf16_bits(dY)
     c = host(fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, a_scale=qx["s_col"],
                      b_scale=qd["s_col"]).float())
     for m0, n0 in tiles:
-        for dm in (0, 128):
-            for dn in (0, 128):
-                r, q = m0 + dm, n0 + dn
-                oa, sa = Q.quantize_1x128_colwise(Xb[:, r:r + 128])
+        for r in (m0, m0 + 128):
+            oa, sa = Q.quantize_1x128_colwise(Xb[:, r:r + 128])
+            for q in (n0, n0 + 128):
                 ob, sb = Q.quantize_1x128_colwise(dYb[:, q:q + 128])
                 ref, t = G.reference(G.dequant_a_1x128(oa, sa), G.dequant_b_blockwise(ob, sb, G.WGRAD))
                 check(c[r:r + 128, q:q + 128].astype(np.float64), ref, t, f"wgrad split tile {r},{q}")
