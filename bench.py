@@ -386,7 +386,9 @@ class WgradAccStep:
                 Launch("quantize_1x128 dY colwise", qcol(self.dY, self.qd_c, self.sd_c, N), "quantize",
                        bytes_=b_1x128_row(M, N)),
                 Launch("gemm blockwise wgrad FP32 accumulate", g, "gemm_blockwise_acc",
-                       flop=self.gemm_flop)]
+                       flop=self.gemm_flop,
+                       kernels=2 if fq.gemm_workspace_bytes(K, N, M, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD,
+                                                            accumulate_fp32=True) > 0 else 1)]
 
     def cpu_sample(self, tiles=1):
         """Oracle on a bounded sample: `tiles` sampled 128x128 tiles of dW, operands quantized

@@ -470,7 +470,7 @@ def gemm(a, b, recipe=FP8Q_BLOCKWISE, layout=FP8Q_FPROP, a_scale=None, b_scale=N
     accumulate_fp32 (BLOCKWISE): `out` is an FP32 (M, N) tensor updated in place, C += A . B^T.
     q_out (M, N) uint8 and s_out (N/128, M) float32 (BLOCKWISE): also receive the 1x128
     rowwise quantization of the BF16 C, made in the GEMM's epilogue.
-    split_tail (BLOCKWISE, BF16 output): give the call the workspace it asks for
+    split_tail (BLOCKWISE, not grouped, no q_out): give the call the workspace it asks for
     (fp8q_gemm_workspace_bytes), taken from torch's caching allocator on the call's stream, so
     that a mostly idle last wave is split into K ranges."""
     args, c = _gemm_args(a, b, recipe, layout, a_scale, b_scale, ld_sa, ld_sb, a_global, b_global, K, m_offsets,

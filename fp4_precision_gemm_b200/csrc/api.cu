@@ -497,8 +497,7 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
   p.s_out = qout ? a->s_out : nullptr;
   p.ld_q_out = a->ld_q_out;
   p.ld_s_out = a->ld_s_out;
-  if (a->workspace != nullptr && a->workspace_bytes >= 1024 && a->recipe == FP8Q_BLOCKWISE && !acc32 && !qout &&
-      !grouped) {
+  if (a->workspace != nullptr && a->workspace_bytes >= 1024 && a->recipe == FP8Q_BLOCKWISE && !qout && !grouped) {
     if (!aligned16(a->workspace)) return FP8Q_ERR_ALIGN;
     p.ws = static_cast<float*>(a->workspace);
     p.ws_bytes = a->workspace_bytes;
@@ -586,7 +585,7 @@ fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* a, void* stream) {
 
 size_t fp8q_gemm_workspace_bytes(const fp8q_gemm_args* a) {
   if (!a || a->recipe != FP8Q_BLOCKWISE || a->layout < FP8Q_FPROP || a->layout > FP8Q_WGRAD) return 0;
-  if (a->c_fp32_accumulate || a->q_out || a->s_out || a->num_groups != 0) return 0;
+  if (a->q_out || a->s_out || a->num_groups != 0) return 0;
   if (a->M <= 0 || a->N <= 0 || a->K <= 0 || a->K % 128 != 0) return 0;
   if (a->M >= (1ll << 31) || a->N >= (1ll << 31) || a->K >= (1ll << 31)) return 0;
   DeviceScratch* d = nullptr;

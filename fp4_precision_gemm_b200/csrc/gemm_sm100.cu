@@ -654,9 +654,9 @@ __global__ void __launch_bounds__(BwCfg<L>::Threads, 1)
   using S = BwSmem<L>;
   constexpr bool kWg = (L == kWgrad);
   constexpr bool ACC32 = EPI == kEpiAcc32, QOUT = EPI == kEpiQuant;
-  // BF16 output, not grouped: the last wave may be split into K ranges, whose FP32 partial
-  // sums go to the workspace (p.ws, through tma_q) instead of C
-  constexpr bool RANGES = (EPI == kEpiBf16) && !GROUPED;
+  // BF16 output or FP32 accumulation, not grouped: the last wave may be split into K ranges,
+  // whose FP32 partial sums go to the workspace (p.ws, through tma_q) instead of C
+  constexpr bool RANGES = (EPI == kEpiBf16 || EPI == kEpiAcc32) && !GROUPED;
   using C = BwCfg<L>;
   constexpr int kBwBN = C::BN, kBwHalfBN = C::HalfBN, kBwEpiWarps = C::EpiWarps;
   constexpr int kBwProducerWarp = C::ProducerWarp, kBwMmaWarp = C::MmaWarp;
@@ -1169,8 +1169,9 @@ static int64_t tail_plan(int64_t tiles, int pairs, int KB, int& tail, int& split
 }
 
 // Split tail, last step: each thread adds the K-range partial sums of 8 columns of one row of
-// a tail tile in range order (FP32) and stores them as BF16 into C, masked at M and N; a CTA
-// covers 8 rows, 32 CTAs a tile.
+// a tail tile in range order (FP32) and stores them as BF16 into C or, when accumulating in
+// FP32, adds the sum into C (one addition per element), masked at M and N; a CTA covers 8
+// rows, 32 CTAs a tile.
 __global__ void __launch_bounds__(256) blockwise_tail_sum_kernel(const __grid_constant__ GemmParams p) {
   const int u = blockIdx.x >> 5, r = (blockIdx.x & 31) * 8 + (threadIdx.x >> 5);
   int rt, nt;
@@ -1188,8 +1189,15 @@ __global__ void __launch_bounds__(256) blockwise_tail_sum_kernel(const __grid_co
     lo = make_float4(__fadd_rn(lo.x, a.x), __fadd_rn(lo.y, a.y), __fadd_rn(lo.z, a.z), __fadd_rn(lo.w, a.w));
     hi = make_float4(__fadd_rn(hi.x, b.x), __fadd_rn(hi.y, b.y), __fadd_rn(hi.z, b.z), __fadd_rn(hi.w, b.w));
   }
-  store8_bf16(p, m, n, make_uint4(pack_bf16(lo.x, lo.y), pack_bf16(lo.z, lo.w), pack_bf16(hi.x, hi.y),
-                                  pack_bf16(hi.z, hi.w)));
+  if (p.c32 != nullptr) {
+    add4_f32(p, m, n, make_uint4(__float_as_uint(lo.x), __float_as_uint(lo.y), __float_as_uint(lo.z),
+                                 __float_as_uint(lo.w)));
+    add4_f32(p, m, n + 4, make_uint4(__float_as_uint(hi.x), __float_as_uint(hi.y), __float_as_uint(hi.z),
+                                     __float_as_uint(hi.w)));
+  } else {
+    store8_bf16(p, m, n, make_uint4(pack_bf16(lo.x, lo.y), pack_bf16(lo.z, lo.w), pack_bf16(hi.x, hi.y),
+                                    pack_bf16(hi.z, hi.w)));
+  }
 }
 
 template <int L, bool G, int EPI = kEpiBf16>
@@ -1208,7 +1216,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   q.main_tiles = (int)tiles;
   q.tail_splits = 0;
   int tail = 0, splits = 0;
-  if constexpr (EPI == kEpiBf16 && !G) {
+  if constexpr ((EPI == kEpiBf16 || EPI == kEpiAcc32) && !G) {
     // the split ranges run as extra units of this launch, after the whole tiles
     const int64_t need = tail_plan(tiles, pairs, p.K / kBKB, tail, splits);
     if (need > 0 && p.ws != nullptr && p.ws_bytes >= need) {
@@ -1220,8 +1228,8 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
   }
   const int64_t units = q.main_tiles + (int64_t)tail * splits;
   cfg.gridDim = dim3(2 * (int)min((int64_t)pairs, units));
-  // tma_q carries the workspace map when the last wave is split (the BF16 epilogue has no
-  // fused quantization)
+  // tma_q carries the workspace map when the last wave is split (the BF16 and FP32-accumulate
+  // epilogues have no fused quantization)
   e = cudaLaunchKernelEx(&cfg, gemm_blockwise_kernel<L, G, EPI>, q, a, b, sb, c, splits > 0 ? ws : qm);
   if (e != cudaSuccess) return e;
   if (splits > 0) {
@@ -1232,7 +1240,7 @@ static cudaError_t launch_blockwise(const GemmParams& p, const CUtensorMap& a, c
 }
 
 size_t blockwise_workspace_bytes(const GemmParams& p, int num_sms) {
-  if (p.recipe != kBlockwise || p.c32 != nullptr || p.q_out != nullptr || p.num_groups > 0) return 0;
+  if (p.recipe != kBlockwise || p.q_out != nullptr || p.num_groups > 0) return 0;
   if (p.M <= 0 || p.N <= 0 || p.K <= 0) return 0;
   cudaLaunchConfig_t cfg;
   cudaLaunchAttribute attr[1];

@@ -110,7 +110,7 @@ struct GemmParams {
   float* s_out;            //   and their decode scales, s_out[(n / 128) * ld_s_out + m]
   int64_t ld_q_out, ld_s_out;
   uint32_t* status;        // device status word
-  // BLOCKWISE, BF16 output, not grouped (set by the launcher): units [0, main_tiles) are the
+  // BLOCKWISE, not grouped (set by the launcher): units [0, main_tiles) are the
   // whole raster tiles; with tail_splits > 0 the remaining tiles (the last, partial wave)
   // follow as tail_splits K ranges each, whose FP32 partial sums go to ws (256 x 256 floats
   // per range) and are then added by a second kernel.
@@ -126,7 +126,7 @@ cudaError_t launch_selftest_wait(uint32_t* status, uint64_t limit_ns, cudaStream
 // 32 x 32 boxes (stored), or FP32 with 16 x 32 boxes (added, FP32 accumulation); tma_q: the
 // fused quantization's E4M3 codes (64 x 32 boxes, stored); tma_ws: p.ws as FP32 rows of 256
 // (16 x 32 boxes, the same swizzle), used only when the last wave is split (in place of
-// tma_q, which a BF16 GEMM without the fused quantization does not use).
+// tma_q, which the BF16 and FP32-accumulate epilogues do not use).
 cudaError_t launch_gemm(const GemmParams& p, const CUtensorMap& tma_a, const CUtensorMap& tma_b,
                         const CUtensorMap& tma_sb, const CUtensorMap& tma_c, const CUtensorMap& tma_q,
                         const CUtensorMap& tma_ws, int num_sms, cudaStream_t s);

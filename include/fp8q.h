@@ -329,20 +329,21 @@ typedef struct {
 fp8q_status fp8q_gemm_blockscaled(const fp8q_gemm_args* args, void* stream);
 
 /* Workspace bytes that fp8q_gemm_blockscaled can use for `args` on the current device; 0 when
- * the call would use none.  Only BLOCKWISE GEMMs with BF16 output, not grouped and without the
- * fused quantization, use one: their kernel keeps one CTA pair per two SMs and walks the
- * 256 x 256 output tiles wave by wave, and when the last wave would leave more than half of
- * the pairs idle for a whole tile and the cut saves at least 16 of its chunks of 128, its tiles
- * are cut into K ranges of at least 4 chunks (one range per pair at most), run after the whole
- * tiles in the same launch, each storing its FP32 partial sum (the same promoted sum, over the
- * range's chunks only) into the workspace; a second small launch adds the ranges in order in
- * FP32 and rounds to BF16 into C.  The result is the
- * same FP32 sum, grouped by ranges, so it can differ from the unsplit schedule's by FP32
- * rounding, and it is the same on every run.  workspace (device memory, 16-byte aligned, or
- * NULL) with workspace_bytes: a NULL workspace, fewer bytes than this function returns, or
- * any other kind of GEMM keeps the unsplit schedule (no error).  The library only uses the
- * workspace in kernels enqueued on the call's stream; the caller must not use it
- * concurrently elsewhere before they complete.  Returns 0 for NULL or invalid arguments. */
+ * the call would use none.  Only BLOCKWISE GEMMs (BF16 output or FP32 accumulation), not
+ * grouped and without the fused quantization, use one.  Their kernel keeps one CTA pair per
+ * two SMs and walks the 256 x 256 output tiles wave by wave.  When the last wave would leave
+ * more than half of the pairs idle for a whole tile and the cut saves at least 16 of its
+ * chunks of 128, its tiles are cut into K ranges of at least 4 chunks (one range per pair at
+ * most), run after the whole tiles in the same launch, each storing its FP32 partial sum (the
+ * same promoted sum, over the range's chunks only) into the workspace; a second small launch
+ * adds the ranges in order in FP32 and rounds the sum to BF16 into C (with
+ * c_fp32_accumulate: adds it into C, still one addition per element).  The result is the same
+ * FP32 sum, grouped by ranges, so it can differ from the unsplit schedule's by FP32 rounding,
+ * and it is the same on every run.  workspace (device memory, 16-byte aligned, or NULL) with
+ * workspace_bytes: a NULL workspace, fewer bytes than this function returns, or any other
+ * kind of GEMM keeps the unsplit schedule (no error).  The library only uses the workspace in
+ * kernels enqueued on the call's stream; the caller must not use it concurrently elsewhere
+ * before they complete.  Returns 0 for NULL or invalid arguments. */
 size_t fp8q_gemm_workspace_bytes(const fp8q_gemm_args* args);
 
 /* Bytes of a scale-factor buffer: recipe MXFP8 (inner/32 scale columns) or NVFP4

@@ -291,7 +291,8 @@ def test_gemm_workspace_bytes_is_zero_without_a_device_or_a_splittable_call(L):
     assert L.fp8q_gemm_workspace_bytes(None) == 0
     for recipe in (fq.FP8Q_BLOCKWISE, fq.FP8Q_MXFP8, fq.FP8Q_NVFP4):
         assert fq.gemm_workspace_bytes(8192, 14336, 4096, recipe, fq.FP8Q_FPROP) == 0
-    assert fq.gemm_workspace_bytes(300, 19328, 2176, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, accumulate_fp32=True) == 0
+    assert fq.gemm_workspace_bytes(300, 19328, 6144, fq.FP8Q_BLOCKWISE, fq.FP8Q_WGRAD, accumulate_fp32=True) == 0
+    assert fq.gemm_workspace_bytes(300, 19328, 6144, fq.FP8Q_BLOCKWISE, fq.FP8Q_FPROP, fused_quant=True) == 0
 
 
 def test_gemm_workspace_argument_checked_before_anything_runs(L):

@@ -303,20 +303,23 @@ def _split_tail_plan(M, N, K, pairs):
     return out, tail * s * 256 * 256 * 4
 
 
-@pytest.mark.parametrize("layout", ["fprop", "dgrad", "wgrad"])
+@pytest.mark.parametrize("layout", ["fprop", "dgrad", "wgrad", "wgrad_acc32"])
 def test_blockwise_split_last_wave(cuda_lib, layout):
     """One full wave plus 4 tiles (6 row tiles, the last 240 rows; 13 column tiles, the last
     128 wide; 74 pairs): the 4 tiles run as 12 K ranges of 4 chunks each, after the whole
-    tiles in the same launch, with FP32 partial sums in a workspace.  Every element is checked against the oracle, with and without the
-    split; the split result is the same on a second run."""
+    tiles in the same launch, with FP32 partial sums in a workspace, in every layout and with
+    FP32 accumulation into C.  Every element is checked against the oracle, with and without
+    the split; the split result is the same on a second run."""
     fq = cuda_lib
     pairs = _pairs()
     tn = -(-(pairs + 4) // 6)
     M, N, K = 6 * 256 - 16, tn * 256 - 128, 6144     # M % 16 == 0: wgrad's colwise quantization
     tiles, nbytes = _split_tail_plan(M, N, K, pairs)
     assert nbytes > 0 and len(tiles) == 6 * tn - pairs
-    L = {"fprop": fq.FP8Q_FPROP, "dgrad": fq.FP8Q_DGRAD, "wgrad": fq.FP8Q_WGRAD}[layout]
-    assert fq.gemm_workspace_bytes(M, N, K, fq.FP8Q_BLOCKWISE, L) == nbytes
+    acc32 = layout == "wgrad_acc32"
+    L = {"fprop": fq.FP8Q_FPROP, "dgrad": fq.FP8Q_DGRAD, "wgrad": fq.FP8Q_WGRAD, "wgrad_acc32": fq.FP8Q_WGRAD}[layout]
+    assert fq.gemm_workspace_bytes(M, N, K, fq.FP8Q_BLOCKWISE, L, accumulate_fp32=acc32) == nbytes
+    c_in = torch.full((M, N), 0.5, dtype=torch.float32, device="cuda")
     if layout == "fprop":
         X, W = bf((M, K), 1.0, 71, 1e-3, 50.0), bf((K, N), 0.02, 72)
         qx, qw = fq.quantize_1x128(X.cuda()), fq.quantize_128x128(W.cuda())
@@ -338,7 +341,8 @@ def test_blockwise_split_last_wave(cuda_lib, layout):
         qx = fq.quantize_1x128(X.cuda(), rowwise=False, colwise=True)
         qd = fq.quantize_1x128(dY.cuda(), rowwise=False, colwise=True)
         run = lambda split: fq.gemm(qx["q_col"], qd["q_col"], fq.FP8Q_BLOCKWISE, L, a_scale=qx["s_col"],  # noqa: E731
-                                    b_scale=qd["s_col"], split_tail=split)
+                                    b_scale=qd["s_col"], split_tail=split,
+                                    out=c_in.clone() if acc32 else None, accumulate_fp32=acc32)
         ox, osx = Q.quantize_1x128_colwise(workloads.bf16_bits(X))
         od, osd = Q.quantize_1x128_colwise(workloads.bf16_bits(dY))
         ref, t = G.reference(G.dequant_a_1x128(ox, osx), G.dequant_b_blockwise(od, osd, G.WGRAD))
@@ -346,14 +350,20 @@ def test_blockwise_split_last_wave(cuda_lib, layout):
     c_again = run(True)
     c_whole = run(False)
     assert fq.device_status() == 0
-    check(c_split, ref, t, f"{layout}, split last wave")
-    check(c_whole, ref, t, f"{layout}, unsplit")
-    assert torch.equal(c_split.view(torch.int16), c_again.view(torch.int16)), "split result not repeatable"
+    for c, what in ((c_split, "split last wave"), (c_whole, "unsplit")):
+        if acc32:   # C_out - 0.5 against the product, plus half an FP32 ulp for the one addition
+            got = host(c).astype(np.float64)
+            excess = G.tolerance_violation(got - 0.5, ref, t) - np.abs(got) * 2.0 ** -24
+            assert float(excess.max()) <= 0, f"{layout}, {what}: {int((excess > 0).sum())} elements outside"
+        else:
+            check(c, ref, t, f"{layout}, {what}")
+    bits = torch.int32 if acc32 else torch.int16
+    assert torch.equal(c_split.view(bits), c_again.view(bits)), "split result not repeatable"
     # outside the split tiles the two schedules run the same kernel on the same data
     mask = torch.ones((M, N), dtype=torch.bool)
     for m0, n0 in tiles:
         mask[m0:m0 + 256, n0:n0 + 256] = False
-    assert torch.equal(c_split.cpu()[mask].view(torch.int16), c_whole.cpu()[mask].view(torch.int16))
+    assert torch.equal(c_split.cpu()[mask].view(bits), c_whole.cpu()[mask].view(bits))
 
 
 def test_llama8b_split_last_wave_tiles_fullsize(cuda_lib):
